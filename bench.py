@@ -1,0 +1,360 @@
+"""Benchmark of the C4 compressed-sparse-attention decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = the whole hot path over one synthetic batch: c4 compress of the
+blocks completed by this step (KV rows and index keys), rotation +
+quantisation of the index queries, indexer logits, top-512 page transform,
+sparse attention with the 128-token window.  The default workload is the
+batch-32 x 131072-token decode with the FP8 64x128 indexer, FP8 KV and 64
+query heads.  Inputs are drawn on the device before timing (seeded,
+synthetic).  Each timed step is one replay of a CUDA graph holding the step,
+bracketed by CUDA events on the launch stream; L2 is flushed (a 512 MiB
+write) between steps, outside the events.
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch
+(no data-path collective: requests are independent) and the time is the max
+over ranks.  `--impl reference` times the CPU oracle instead, on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA decode query-tok/s at 128K/1M ctx; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "query-tok/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="decode_128k")
+    p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def workload_config(w):
+    return {"workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
+            "c4_seq_len": int(w.c4_lens.max()), "query_tokens": w.num_q,
+            "indexer": f"{w.idx_fmt} {w.idx_heads}x{w.idx_dim}", "heads": w.heads,
+            "kv": w.kv_fmt, "window": w.window, "topk": w.topk, "page_size": 256,
+            "l2": "flushed between timed steps (512 MiB write)"}
+
+
+def index_bytes_per_key(w):
+    return {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}[w.idx_fmt]
+
+
+def indexer_alg_bytes(w):
+    """Bytes one indexer launch must move: every visible key (codes + scales)
+    once per query row, the query codes and weights, and the logits written."""
+    nv = np.concatenate([np.minimum(w.c4_lens[b], (np.arange(L - q, L) + 1) // 4)
+                         for b, (L, q) in enumerate(zip(w.seq_lens, w.q_lens))])
+    qb = {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}
+    return int(nv.sum() * (index_bytes_per_key(w) + 4) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4))
+
+
+def step_alg_bytes(w):
+    """Algorithmic bytes of one whole step (keys, q, selected + window rows,
+    attention q/out; logits excluded as an implementation detail)."""
+    row = 656 if w.kv_fmt == "fp8" else 1152
+    nv = np.concatenate([np.minimum(w.c4_lens[b], (np.arange(L - q, L) + 1) // 4)
+                         for b, (L, q) in enumerate(zip(w.seq_lens, w.q_lens))])
+    pos = np.concatenate([np.arange(L - q, L) for L, q in zip(w.seq_lens, w.q_lens)])
+    rows = np.minimum(nv, 512) + np.minimum(w.window, pos + 1)
+    qb = {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}
+    return int(nv.sum() * index_bytes_per_key(w) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4)
+               + rows.sum() * row + w.num_q * w.heads * (576 + 512) * 2)
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, data, pt, budget_s=20.0):
+    """The oracle, as it stands, timed on this host's cores over a bounded
+    sample: whole-step oracle runs of requests 0, 1, ... until ~budget_s."""
+    from oracle import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    done_q, reqs = 0, []
+    for b in range(w.bs):
+        oracle.step(w, data, pt, requests=[b])
+        done_q += int(w.q_lens[b])
+        reqs.append(b)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done_q / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"whole oracle step (compress, quantise caches, score, top-512, attention) "
+                      f"for {len(reqs)} of {w.bs} requests ({done_q} query tokens) in {dt:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, timed on this host, same workload."""
+    import torch
+    from compressed_sparse_attention_12_b200 import synth
+    from oracle import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.workload(args.workload)
+    # draw the sampled request's inputs on the host (small): one request's slice
+    data = synth.draw(w, "cuda" if torch.cuda.is_available() else "cpu")
+    pt = synth.page_table(w)
+    oracle.build()
+    for i in range(args.warmup):
+        oracle.step(w, data, pt, requests=[i % w.bs])
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.step(w, data, pt, requests=[i % w.bs])
+        times.append(time.perf_counter() - t0)
+    per = sum(times) / len(times)
+    q_per = float(np.mean(w.q_lens))
+    v = q_per / per
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": workload_config(w),
+           "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.num_threads(),
+                            "kind": "oracle",
+                            "sample": "each step: the whole oracle step for one request "
+                                      "(cycling through the batch)"},
+           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from compressed_sparse_attention_12_b200 import build, csa, pipeline, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    csa.lib()
+
+    w = synth.workload(args.workload)
+    w.seed += 1000 * rank                      # each rank its own batch
+    data = synth.draw(w, dev)
+    batch = pipeline.CsaBatch(w, data, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    # per-kernel events inside the graph around the indexer launch
+    ev_i0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev_i1 = torch.cuda.Event(enable_timing=True, external=True)
+    launches_per_step = 0
+
+    def step_body(s):
+        batch.compress(s)
+        batch_q = batch
+        from compressed_sparse_attention_12_b200 import csa as c
+        c.csa_hadamard_quant(batch_q.q_idx, batch_q.idx_fmt, batch_q.q_codes, batch_q.q_bsc,
+                             batch_q.q_scales, w_in=batch_q.w_head, w_out=batch_q.w_fold,
+                             status=batch_q.status, stream=s)
+        ev_i0.record(s)
+        c.csa_indexer_logits(batch_q.q_codes, batch_q.q_bsc, batch_q.w_fold, w.idx_heads,
+                             w.idx_dim, batch_q.idx_fmt, batch_q.k_codes, batch_q.k_bsc,
+                             batch_q.k_scales, batch_q.page_table, batch_q.c4_lens, batch_q.cu_q,
+                             batch_q.q_pos, batch_q.max_c4, batch_q.logits,
+                             status=batch_q.status, stream=s)
+        ev_i1.record(s)
+        batch.select(s)
+        batch.attend(s)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step_body(stream)
+        stream.synchronize()
+        batch.check_status()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step_body(stream)
+    # kernels per step: compress (2 when blocks complete), quantise, indexer, top-k (2),
+    # attention (1, +1 combine when split)
+    launches_per_step = (2 if batch.max_new >= 4 else 0) + 1 + 1 + 2 + \
+        (2 if csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, w.window, batch.decode) > 0 else 1)
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        g.replay()
+    torch.cuda.synchronize()
+    batch.check_status()
+
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    step_ms, idx_ms = [], []
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            step_ms.append(e0.elapsed_time(e1))
+            idx_ms.append(ev_i0.elapsed_time(ev_i1))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ck = clocks.stop()
+    batch.check_status()
+    t_step = sum(step_ms) / len(step_ms) / 1e3
+    t_idx = sum(idx_ms) / len(idx_ms) / 1e3
+    if world > 1:
+        t = torch.tensor([t_step, t_idx], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_step, t_idx = t.tolist()
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if True:
+        h_in = {k: data[k].cpu().pin_memory() for k in ("q_idx", "w", "q") if k in data}
+        for k in ("raw_kv", "gate", "raw_idx_k", "idx_gate"):
+            if data.get(k) is not None:
+                h_in[k] = data[k].cpu().pin_memory()
+        h_out = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
+        dst = {"q_idx": batch.q_idx, "w": batch.w_head, "q": batch.q, "raw_kv": batch.raw_kv,
+               "gate": batch.gate, "raw_idx_k": batch.raw_idx_k, "idx_gate": batch.idx_gate}
+        h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+        d2h = h_out.numel() * h_out.element_size()
+        e2e_ms = []
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup + args.steps):
+                flush.fill_(1)
+                e0.record(stream)
+                for k, v in h_in.items():
+                    dst[k].copy_(v, non_blocking=True)
+                g.replay()
+                h_out.copy_(batch.out, non_blocking=True)
+                e1.record(stream)
+                e1.synchronize()
+                if i >= args.warmup:
+                    e2e_ms.append(e0.elapsed_time(e1))
+        t_e2e = sum(e2e_ms) / len(e2e_ms) / 1e3
+        if world > 1:
+            t = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_e2e = t.item()
+        e2e = {"value": world * w.num_q / t_e2e, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": t_e2e * 1e3}
+
+    if rank == 0:
+        hbm, src = peaks()
+        ib = indexer_alg_bytes(w)
+        achieved = ib / t_idx / 1e9
+        sb = step_alg_bytes(w)
+        out = {"metric": METRIC, "value": world * w.num_q / t_step, "unit": UNIT, "n_gpus": world,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": f"{w.idx_fmt} indexer, bf16 attention", "data": "synthetic",
+               "config": workload_config(w),
+               "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
+                       "frac_of_8tbs": sb / t_step / 8e12, "frac_of_peak": sb / t_step / 1e9 / hbm},
+               "roofline": {"kernel": "indexer_logits", "bound": "hbm", "achieved": achieved,
+                            "peak": hbm, "peak_source": src, "unit": "GB/s",
+                            "frac": achieved / hbm, "traffic": None,
+                            "alg_bytes_per_launch": ib, "launch_ms": t_idx * 1e3},
+               "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": ck}
+        if not args.no_cpu_baseline and world == 1:
+            out["cpu_baseline"] = cpu_baseline(w, data, batch.pt_host)
+        print(json.dumps(out), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+// csa_api.cu -- the extern "C" entry points of libcsa.so (declared in
+// include/csa.h): host-side argument validation, then the launchers.
+#include <cuda_runtime.h>
+
+#include "../../include/csa.h"
+#include "launch.h"
+
+namespace {
+
+csa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool index_fmt_ok(int32_t fmt) {
+    return fmt == CSA_FMT_BF16 || fmt == CSA_FMT_FP8 || fmt == CSA_FMT_FP4;
+}
+
+bool kv_fmt_ok(int32_t fmt) { return fmt == CSA_FMT_BF16 || fmt == CSA_FMT_FP8; }
+
+// Scales that each index format needs next to its codes.
+bool index_arrays_ok(int32_t fmt, const void *codes, const void *block_scales,
+                     const void *scales) {
+    if (!codes) return false;
+    if (fmt == CSA_FMT_FP8 && !scales) return false;
+    if (fmt == CSA_FMT_FP4 && (!scales || !block_scales)) return false;
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *csa_status_string(csa_status_t s) {
+    switch (s) {
+        case CSA_OK: return "ok";
+        case CSA_ERR_INVALID: return "invalid argument";
+        case CSA_ERR_UNSUPPORTED: return "unsupported size or format";
+        case CSA_ERR_CUDA: return "CUDA error";
+        case CSA_ERR_TIMEOUT: return "device wait timed out";
+        case CSA_ERR_BOUNDS: return "index, slot or length out of range";
+        case CSA_ERR_NAN: return "NaN logit";
+        case CSA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int32_t csa_abi_version(void) { return 1; }
+
+int32_t csa_kv_row_bytes(int32_t kv_fmt) {
+    return kv_fmt == CSA_FMT_FP8 ? 656 : kv_fmt == CSA_FMT_BF16 ? 1152 : 0;
+}
+
+csa_status_t csa_kv_store(const float *rows, int64_t n, const int32_t *slots, int32_t kv_fmt,
+                          void *cache, int64_t num_slots, int32_t *status, void *stream) {
+    if (n < 0 || num_slots < 0) return CSA_ERR_INVALID;
+    if (!kv_fmt_ok(kv_fmt)) return CSA_ERR_UNSUPPORTED;
+    if (n == 0) return CSA_OK;
+    if (!rows || !slots || !cache) return CSA_ERR_INVALID;
+    return cuda_status(csa::launch_kv_store(rows, n, slots, kv_fmt, cache, num_slots, status,
+                                            as_stream(stream)));
+}
+
+csa_status_t csa_c4_compress(const float *x, const float *gate, const float *bias, int32_t dim,
+                             int32_t bs, const int32_t *cu_x, int64_t total_rows,
+                             const int32_t *start_pos, int32_t max_rows_per_req,
+                             const int32_t *page_table, int32_t page_table_stride,
+                             int32_t out_kind, void *out, uint8_t *out_block_scales,
+                             float *out_scales, int64_t num_slots, int32_t *status,
+                             void *stream) {
+    if (bs < 0 || total_rows < 0 || max_rows_per_req < 0 || page_table_stride < 0)
+        return CSA_ERR_INVALID;
+    const bool kv = out_kind == CSA_OUT_KV_BF16 || out_kind == CSA_OUT_KV_FP8;
+    const bool idx = out_kind == CSA_OUT_INDEX_BF16 || out_kind == CSA_OUT_INDEX_FP8 ||
+                     out_kind == CSA_OUT_INDEX_FP4;
+    if (!kv && !idx) return CSA_ERR_UNSUPPORTED;
+    if (kv && dim != CSA_KV_DIM) return CSA_ERR_UNSUPPORTED;
+    if (idx && dim != 64 && dim != 128) return CSA_ERR_UNSUPPORTED;
+    if (bs == 0 || total_rows == 0 || max_rows_per_req < 4) return CSA_OK;
+    if (!x || !gate || !bias || !cu_x || !start_pos || !page_table || !out) return CSA_ERR_INVALID;
+    if (out_kind == CSA_OUT_INDEX_FP8 && !out_scales) return CSA_ERR_INVALID;
+    if (out_kind == CSA_OUT_INDEX_FP4 && (!out_scales || !out_block_scales)) return CSA_ERR_INVALID;
+    if (bs > 65535) return CSA_ERR_UNSUPPORTED;
+    return cuda_status(csa::launch_c4_compress(x, gate, bias, dim, bs, cu_x, start_pos,
+                                               max_rows_per_req, page_table, page_table_stride,
+                                               out_kind, out, out_block_scales, out_scales,
+                                               num_slots, status, as_stream(stream)));
+}
+
+csa_status_t csa_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                                int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
+                                void *codes, uint8_t *block_scales, float *scales,
+                                const float *w_in, float *w_out, int32_t *status, void *stream) {
+    if (rows < 0) return CSA_ERR_INVALID;
+    if (x_dtype != CSA_FMT_BF16 && x_dtype != CSA_FMT_F32) return CSA_ERR_UNSUPPORTED;
+    if (dim != 64 && dim != 128) return CSA_ERR_UNSUPPORTED;
+    if (!index_fmt_ok(fmt)) return CSA_ERR_UNSUPPORTED;
+    if (rows == 0) return CSA_OK;
+    if (!x || !index_arrays_ok(fmt, codes, block_scales, scales)) return CSA_ERR_INVALID;
+    if ((w_in == nullptr) != (w_out == nullptr)) return CSA_ERR_INVALID;
+    if (row_map && num_out_rows < 0) return CSA_ERR_INVALID;
+    return cuda_status(csa::launch_hadamard_quant(x, x_dtype, rows, dim, fmt, row_map,
+                                                  num_out_rows, codes, block_scales, scales,
+                                                  w_in, w_out, status, as_stream(stream)));
+}
+
+csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
+                                const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                const uint8_t *k_block_scales, const float *k_scales,
+                                int64_t num_slots, const int32_t *page_table,
+                                int32_t page_table_stride, const int32_t *c4_seq_lens,
+                                int32_t bs, const int32_t *cu_q, const int32_t *q_pos,
+                                int32_t max_c4_len, float *logits, int64_t logits_stride,
+                                int32_t *status, void *stream) {
+    if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (!index_fmt_ok(fmt)) return CSA_ERR_UNSUPPORTED;
+    if (idx_dim != 64 && idx_dim != 128) return CSA_ERR_UNSUPPORTED;
+    if (idx_heads < 1 || idx_heads > 128) return CSA_ERR_UNSUPPORTED;
+    if (num_q == 0 || max_c4_len == 0) return CSA_OK;
+    if (bs < 1 || !q_codes || !q_weights || !page_table || !c4_seq_lens || !cu_q || !logits)
+        return CSA_ERR_INVALID;
+    if (fmt == CSA_FMT_FP4 && !q_block_scales) return CSA_ERR_INVALID;
+    if (!index_arrays_ok(fmt, k_codes, k_block_scales, k_scales)) return CSA_ERR_INVALID;
+    if (logits_stride < max_c4_len) return CSA_ERR_INVALID;
+    if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
+    csa::IndexerArgs a{q_codes, q_block_scales, q_weights, num_q, idx_heads, idx_dim, fmt,
+                       k_codes, k_block_scales, k_scales, num_slots, page_table,
+                       page_table_stride, c4_seq_lens, bs, cu_q, q_pos, max_c4_len, logits,
+                       logits_stride, status};
+    return cuda_status(csa::launch_indexer(a, as_stream(stream)));
+}
+
+size_t csa_topk512_workspace_size(int32_t num_q, int32_t max_c4_len) {
+    if (num_q <= 0) return 0;
+    return csa::topk_workspace_bytes(num_q, max_c4_len);
+}
+
+csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stride,
+                                        int32_t num_q, const int32_t *c4_seq_lens, int32_t bs,
+                                        const int32_t *cu_q, const int32_t *q_pos,
+                                        const int32_t *page_table, int32_t page_table_stride,
+                                        int64_t num_slots, int32_t c4_page_size,
+                                        int32_t max_c4_len, int32_t *c4_sparse_page_indices,
+                                        int32_t *raw_indices, void *workspace,
+                                        size_t workspace_bytes, int32_t *status, void *stream) {
+    if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (c4_page_size != CSA_C4_PAGE_SIZE) return CSA_ERR_INVALID;
+    if (num_q == 0) return CSA_OK;
+    if (bs < 1 || !c4_seq_lens || !cu_q || !page_table || !c4_sparse_page_indices)
+        return CSA_ERR_INVALID;
+    if (max_c4_len > 0 && (!logits || logits_stride < max_c4_len)) return CSA_ERR_INVALID;
+    if (!workspace || workspace_bytes < csa_topk512_workspace_size(num_q, max_c4_len))
+        return CSA_ERR_WORKSPACE;
+    if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
+    csa::TopkArgs a{logits, logits_stride, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,
+                    page_table_stride, num_slots, max_c4_len, c4_sparse_page_indices,
+                    raw_indices, workspace, status};
+    return cuda_status(csa::launch_topk512(a, as_stream(stream)));
+}
+
+size_t csa_sparse_mqa_workspace_size(int32_t num_q, int32_t heads, int32_t window,
+                                     int32_t decode) {
+    if (num_q <= 0 || heads <= 0) return 0;
+    return csa::attn_workspace_bytes(num_q, heads, window, decode != 0);
+}
+
+static csa_status_t sparse_mqa(const void *q, int32_t num_q, int32_t heads,
+                               const void *c4_cache, const void *raw_cache, int32_t kv_fmt,
+                               int64_t num_c4_slots, int64_t num_raw_slots, const int32_t *idx,
+                               const int32_t *page_table, int32_t page_table_stride,
+                               const int32_t *seq_lens, int32_t bs, const int32_t *cu_q,
+                               const int32_t *q_pos, int32_t window, float sm_scale, void *out,
+                               float *lse, void *workspace, size_t workspace_bytes,
+                               int32_t *status, void *stream, bool decode) {
+    if (num_q < 0 || bs < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (!kv_fmt_ok(kv_fmt)) return CSA_ERR_UNSUPPORTED;
+    if (heads != 16 && heads != 32 && heads != 64 && heads != 128) return CSA_ERR_UNSUPPORTED;
+    if (window < 0 || window > 1024) return CSA_ERR_UNSUPPORTED;
+    if (num_q == 0) return CSA_OK;
+    if (bs < 1 || !q || !idx || !page_table || !cu_q || !out || !seq_lens) return CSA_ERR_INVALID;
+    if (!c4_cache && num_c4_slots > 0) return CSA_ERR_INVALID;
+    if (window > 0 && !raw_cache) return CSA_ERR_INVALID;
+    if (!q_pos && num_q != bs) return CSA_ERR_INVALID;
+    const size_t need = csa::attn_workspace_bytes(num_q, heads, window, decode);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return CSA_ERR_WORKSPACE;
+    if (num_q > 2147483647 / 2) return CSA_ERR_UNSUPPORTED;
+    csa::AttnArgs a{q, num_q, heads, c4_cache, raw_cache, kv_fmt, num_c4_slots, num_raw_slots,
+                    idx, page_table, page_table_stride, seq_lens, bs, cu_q, q_pos, window,
+                    sm_scale, out, lse, workspace, status};
+    return cuda_status(csa::launch_sparse_mqa(a, decode, as_stream(stream)));
+}
+
+csa_status_t csa_sparse_mqa_decode(const void *q, int32_t num_q, int32_t heads,
+                                   const void *c4_cache, const void *raw_cache, int32_t kv_fmt,
+                                   int64_t num_c4_slots, int64_t num_raw_slots,
+                                   const int32_t *c4_sparse_page_indices,
+                                   const int32_t *page_table, int32_t page_table_stride,
+                                   const int32_t *seq_lens, int32_t bs, const int32_t *cu_q,
+                                   const int32_t *q_pos, int32_t window, float sm_scale,
+                                   void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, int32_t *status, void *stream) {
+    return sparse_mqa(q, num_q, heads, c4_cache, raw_cache, kv_fmt, num_c4_slots, num_raw_slots,
+                      c4_sparse_page_indices, page_table, page_table_stride, seq_lens, bs, cu_q,
+                      q_pos, window, sm_scale, out, lse, workspace, workspace_bytes, status,
+                      stream, true);
+}
+
+csa_status_t csa_sparse_mqa_prefill(const void *q, int32_t num_q, int32_t heads,
+                                    const void *c4_cache, const void *raw_cache, int32_t kv_fmt,
+                                    int64_t num_c4_slots, int64_t num_raw_slots,
+                                    const int32_t *c4_sparse_page_indices,
+                                    const int32_t *page_table, int32_t page_table_stride,
+                                    const int32_t *seq_lens, int32_t bs, const int32_t *cu_q,
+                                    const int32_t *q_pos, int32_t window, float sm_scale,
+                                    void *out, float *lse, void *workspace,
+                                    size_t workspace_bytes, int32_t *status, void *stream) {
+    return sparse_mqa(q, num_q, heads, c4_cache, raw_cache, kv_fmt, num_c4_slots, num_raw_slots,
+                      c4_sparse_page_indices, page_table, page_table_stride, seq_lens, bs, cu_q,
+                      q_pos, window, sm_scale, out, lse, workspace, workspace_bytes, status,
+                      stream, false);
+}
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// launch.h -- internal launchers behind the C ABI (host side, namespace csa).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace csa {
+
+// Raises a kernel's dynamic shared-memory limit once per device (the call is
+// not a stream operation, so it is kept out of CUDA-graph captures after the
+// first eager launch).  `done` is a per-kernel table indexed by device.
+inline cudaError_t ensure_max_smem(const void *fn, int bytes, int *done) {
+    int d = 0;
+    cudaError_t e = cudaGetDevice(&d);
+    if (e != cudaSuccess) return e;
+    if (d < 0 || d >= 64) return cudaErrorInvalidDevice;
+    if (done[d] >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[d] = bytes;
+    return e;
+}
+
+cudaError_t launch_kv_store(const float *rows, int64_t n, const int32_t *slots, int fmt,
+                            void *cache, int64_t num_slots, int32_t *status, cudaStream_t s);
+
+cudaError_t launch_hadamard_quant(const void *x, int x_dtype, int64_t rows, int dim, int fmt,
+                                  const int32_t *row_map, int64_t num_out_rows, void *codes,
+                                  uint8_t *block_scales, float *scales, const float *w_in,
+                                  float *w_out, int32_t *status, cudaStream_t s);
+
+cudaError_t launch_c4_compress(const float *x, const float *gate, const float *bias, int dim,
+                               int bs, const int32_t *cu_x, const int32_t *start_pos,
+                               int max_rows, const int32_t *page_table, int pt_stride,
+                               int out_kind, void *out, uint8_t *out_block_scales,
+                               float *out_scales, int64_t num_slots, int32_t *status,
+                               cudaStream_t s);
+
+// Shape of one indexer launch (validated by the caller).
+struct IndexerArgs {
+    const void *q_codes;
+    const uint8_t *q_block_scales;
+    const float *q_weights;
+    int num_q, heads, dim, fmt;
+    const void *k_codes;
+    const uint8_t *k_block_scales;
+    const float *k_scales;
+    int64_t num_slots;
+    const int32_t *page_table;
+    int pt_stride;
+    const int32_t *c4_seq_lens;
+    int bs;
+    const int32_t *cu_q;
+    const int32_t *q_pos;
+    int max_c4_len;
+    float *logits;
+    int64_t logits_stride;
+    int32_t *status;
+};
+cudaError_t launch_indexer(const IndexerArgs &a, cudaStream_t s);
+
+// Top-512: candidates per (query row, chunk) live in the workspace.
+size_t topk_workspace_bytes(int num_q, int max_c4_len);
+struct TopkArgs {
+    const float *logits;
+    int64_t logits_stride;
+    int num_q;
+    const int32_t *c4_seq_lens;
+    int bs;
+    const int32_t *cu_q;
+    const int32_t *q_pos;
+    const int32_t *page_table;
+    int pt_stride;
+    int64_t num_slots;
+    int max_c4_len;
+    int32_t *out_phys;
+    int32_t *out_raw;
+    void *workspace;
+    int32_t *status;
+};
+cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s);
+
+struct AttnArgs {
+    const void *q;
+    int num_q, heads;
+    const void *c4_cache, *raw_cache;
+    int kv_fmt;
+    int64_t num_c4_slots, num_raw_slots;
+    const int32_t *idx;
+    const int32_t *page_table;
+    int pt_stride;
+    const int32_t *seq_lens;
+    int bs;
+    const int32_t *cu_q;
+    const int32_t *q_pos;
+    int window;
+    float sm_scale;
+    void *out;
+    float *lse;
+    void *workspace;
+    int32_t *status;
+};
+size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode);
+cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s);
+
+}  // namespace csa

@@ -1,0 +1,302 @@
+// topk.cu -- step 3, the fixed-k top-512 with the paged index transform
+// ("Token 的一生：DSV4 架构与 DSpark" §3.2 topk_transform_512, page arithmetic
+// of §2.2).
+//
+// Selection is exact on order-preserving 32-bit keys of the float logits
+// (-0 folded onto +0, NaN recorded and ordered below -inf).  The order is
+// (logit descending, logical index ascending); outputs are listed in
+// ascending logical index and padded with -1.
+//
+// Two launches, no inter-CTA waits:
+//   stage 1: each CTA takes a chunk of 8192 logits of one query row into
+//            shared memory, finds the chunk's 512th key by a 3-pass radix
+//            select (12/12/8-bit digits, shared-memory histograms, block
+//            suffix scan), and writes the chunk's top-512 (key, index) pairs
+//            in index order to the workspace.
+//   stage 2: one CTA per query row repeats the select over the row's
+//            concatenated candidates (every element of the global top-512 is
+//            in its chunk's top-512 under the same total order) and writes
+//            physical slots page_table[s/64]*64 + s%64 and raw indices.
+#include "common.cuh"
+#include "launch.h"
+
+namespace csa {
+
+constexpr int kTkThreads = 512;
+constexpr int kTkChunk = 8192;
+constexpr int kTkWarps = kTkThreads / 32;
+constexpr int kHistBins = 4096;
+
+__device__ __forceinline__ uint32_t order_key(float f, int32_t *status) {
+    uint32_t u = __float_as_uint(f);
+    if (f != f) {  // NaN
+        report(status, CSA_ERR_NAN);
+        return 0u;
+    }
+    if (f == 0.0f) u = 0u;                        // -0 -> +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct TkShared {
+    uint32_t hist[kHistBins];
+    uint32_t warp_a[kTkWarps];
+    uint32_t warp_b[kTkWarps];
+    uint32_t digit, above;
+};
+
+// Exclusive scan of one value per thread over the block; returns the prefix
+// and writes the block total to *total.  Uses sh.warp_a.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total, TkShared &sh) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) sh.warp_a[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kTkWarps; w++) {
+        const uint32_t x = sh.warp_a[w];
+        before += (w < warp) ? x : 0u;
+        tot += x;
+    }
+    __syncthreads();
+    *total = tot;
+    return before + incl - v;
+}
+
+// Finds the K-th largest key T among keys[0..n) (K <= n) and how many keys
+// equal to T belong to the top K (need_eq >= 1).  keys may point to shared
+// or global memory.
+__device__ void radix_threshold(const uint32_t *keys, int n, int K, TkShared &sh,
+                                uint32_t *T_out, int *need_eq_out) {
+    const int shifts[3] = {20, 8, 0};
+    const int widths[3] = {12, 12, 8};
+    uint32_t prefix = 0;
+    int remaining = K;
+#pragma unroll 1
+    for (int p = 0; p < 3; p++) {
+        const int shift = shifts[p], bits = widths[p];
+        const uint32_t nb = 1u << bits;
+        const uint64_t hi_mask64 = ~((1ull << (shift + bits)) - 1ull);
+        const uint32_t hi_mask = (uint32_t)hi_mask64;
+        for (uint32_t i = threadIdx.x; i < nb; i += kTkThreads) sh.hist[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += kTkThreads) {
+            const uint32_t k = keys[i];
+            if ((k & hi_mask) == (prefix & hi_mask))
+                atomicAdd(&sh.hist[(k >> shift) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+        // Suffix scan from the top bin: thread i owns bins nb-1-8i .. nb-8-8i.
+        const int per = (int)nb / kTkThreads;  // 8 (4096 bins) or 0 (256 bins)
+        uint32_t mine = 0;
+        uint32_t c[8];
+        if (per == 8) {
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                c[j] = sh.hist[nb - 1 - (threadIdx.x * 8 + j)];
+                mine += c[j];
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; j++) c[j] = 0;
+            if (threadIdx.x < nb) c[0] = sh.hist[nb - 1 - threadIdx.x];
+            mine = c[0];
+        }
+        uint32_t total;
+        const uint32_t excl = block_excl_scan(mine, &total, sh);
+        if (excl < (uint32_t)remaining && (uint32_t)remaining <= excl + mine) {
+            uint32_t acc = excl;
+            const int cnt = per == 8 ? 8 : 1;
+            for (int j = 0; j < cnt; j++) {
+                if (acc + c[j] >= (uint32_t)remaining) {
+                    sh.digit = per == 8 ? nb - 1 - (threadIdx.x * 8 + j) : nb - 1 - threadIdx.x;
+                    sh.above = acc;
+                    break;
+                }
+                acc += c[j];
+            }
+        }
+        __syncthreads();
+        prefix |= sh.digit << shift;
+        remaining -= (int)sh.above;
+        __syncthreads();
+    }
+    *T_out = prefix;
+    *need_eq_out = remaining;
+}
+
+// Walks keys[0..n) in index order and calls emit(pos, i, key) for the
+// selected ones: key > T, or key == T among the first need_eq such keys.
+template <typename Emit>
+__device__ void ordered_compact(const uint32_t *keys, int n, uint32_t T, int need_eq, int K,
+                                TkShared &sh, Emit emit) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t base_eq = 0, base_out = 0;
+    for (int r0 = 0; r0 < n && base_out < (uint32_t)K; r0 += kTkThreads) {
+        const int i = r0 + threadIdx.x;
+        const uint32_t k = i < n ? keys[i] : 0u;
+        const bool eq = i < n && k == T;
+        const bool gt = i < n && k > T;
+        const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) sh.warp_a[warp] = __popc(beq);
+        __syncthreads();
+        uint32_t eq_before = 0, eq_total = 0;
+#pragma unroll
+        for (int w = 0; w < kTkWarps; w++) {
+            const uint32_t x = sh.warp_a[w];
+            eq_before += (w < warp) ? x : 0u;
+            eq_total += x;
+        }
+        const uint32_t eq_rank = base_eq + eq_before + __popc(beq & lt);
+        const bool take = gt || (eq && eq_rank < (uint32_t)need_eq);
+        const uint32_t btk = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) sh.warp_b[warp] = __popc(btk);
+        __syncthreads();
+        uint32_t tk_before = 0, tk_total = 0;
+#pragma unroll
+        for (int w = 0; w < kTkWarps; w++) {
+            const uint32_t x = sh.warp_b[w];
+            tk_before += (w < warp) ? x : 0u;
+            tk_total += x;
+        }
+        if (take) emit((int)(base_out + tk_before + __popc(btk & lt)), i, k);
+        base_eq += eq_total;
+        base_out += tk_total;
+        __syncthreads();
+    }
+}
+
+struct RowInfo {
+    int b, n_vis;
+};
+
+__device__ __forceinline__ RowInfo row_info(int t, const int32_t *cu_q, int bs,
+                                            const int32_t *q_pos, const int32_t *c4_lens,
+                                            int max_c4_len, int pt_stride, int32_t *status,
+                                            bool leader) {
+    int lo = 0, hi = bs - 1;
+    while (lo < hi) {  // last b with cu_q[b] <= t
+        const int mid = (lo + hi + 1) >> 1;
+        if (cu_q[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    RowInfo r;
+    r.b = lo;
+    int n = c4_lens[lo];
+    if (q_pos) n = min(n, (q_pos[t] + 1) / 4);
+    const int cap = min(max_c4_len, pt_stride * kC4Page);
+    if (n > cap) {
+        if (leader) report(status, CSA_ERR_BOUNDS);
+        n = cap;
+    }
+    r.n_vis = max(n, 0);
+    return r;
+}
+
+__global__ void __launch_bounds__(kTkThreads)
+topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens,
+                   int bs, const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
+                   int pt_stride, int max_chunks, uint32_t *cand_key, int32_t *cand_idx,
+                   int32_t *status) {
+    extern __shared__ __align__(16) uint8_t tk_smem[];
+    TkShared &sh = *reinterpret_cast<TkShared *>(tk_smem);
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(tk_smem + sizeof(TkShared));
+    const int t = blockIdx.y, c = blockIdx.x;
+    const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
+                                threadIdx.x == 0 && c == 0);
+    const int lo = c * kTkChunk;
+    if (lo >= ri.n_vis) return;
+    const int len = min(kTkChunk, ri.n_vis - lo);
+    const float *row = logits + (int64_t)t * stride + lo;
+    for (int i = threadIdx.x; i < len; i += kTkThreads) skeys[i] = order_key(row[i], status);
+    __syncthreads();
+    const int K = min(kTopK, len);
+    uint32_t T = 0;
+    int need_eq = len;
+    if (len > kTopK) radix_threshold(skeys, len, K, sh, &T, &need_eq);
+    uint32_t *ok = cand_key + ((int64_t)t * max_chunks + c) * kTopK;
+    int32_t *oi = cand_idx + ((int64_t)t * max_chunks + c) * kTopK;
+    ordered_compact(skeys, len, T, need_eq, K, sh, [&](int pos, int i, uint32_t k) {
+        ok[pos] = k;
+        oi[pos] = lo + i;
+    });
+}
+
+__global__ void __launch_bounds__(kTkThreads)
+topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const int32_t *q_pos,
+                   int max_c4_len, const int32_t *page_table, int pt_stride, int64_t num_slots,
+                   int max_chunks, const uint32_t *cand_key, const int32_t *cand_idx,
+                   int32_t *out_phys, int32_t *out_raw, int32_t *status) {
+    __shared__ TkShared sh;
+    const int t = blockIdx.x;
+    const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
+                                false);
+    const int n = ri.n_vis;
+    int total = 0;
+    if (n > 0) {
+        const int nch = (n + kTkChunk - 1) / kTkChunk;
+        total = (nch - 1) * kTopK + min(kTopK, n - (nch - 1) * kTkChunk);
+    }
+    const int K = min(kTopK, total);
+    const uint32_t *keys = cand_key + (int64_t)t * max_chunks * kTopK;
+    const int32_t *idx = cand_idx + (int64_t)t * max_chunks * kTopK;
+    const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
+    uint32_t T = 0;
+    int need_eq = total;
+    if (total > kTopK) radix_threshold(keys, total, K, sh, &T, &need_eq);
+    int32_t *op = out_phys + (int64_t)t * kTopK;
+    int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
+    ordered_compact(keys, total, T, need_eq, K, sh, [&](int pos, int i, uint32_t) {
+        const int32_t s = idx[i];
+        const int32_t page = pt_row[s / kC4Page];
+        const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
+        int32_t phys = (int32_t)slot;
+        if (page < 0 || slot >= num_slots) {
+            report(status, CSA_ERR_BOUNDS);
+            phys = -1;
+        }
+        op[pos] = phys;
+        if (orw) orw[pos] = s;
+    });
+    for (int p = K + threadIdx.x; p < kTopK; p += kTkThreads) {
+        op[p] = -1;
+        if (orw) orw[p] = -1;
+    }
+}
+
+static int topk_max_chunks(int max_c4_len) {
+    return max_c4_len <= 0 ? 1 : (max_c4_len + kTkChunk - 1) / kTkChunk;
+}
+
+size_t topk_workspace_bytes(int num_q, int max_c4_len) {
+    return (size_t)num_q * topk_max_chunks(max_c4_len) * kTopK * 8;
+}
+
+cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
+    if (a.num_q == 0) return cudaSuccess;
+    const int mc = topk_max_chunks(a.max_c4_len);
+    uint32_t *ck = (uint32_t *)a.workspace;
+    int32_t *ci = (int32_t *)((uint8_t *)a.workspace + (size_t)a.num_q * mc * kTopK * 4);
+    const size_t smem1 = sizeof(TkShared) + kTkChunk * sizeof(uint32_t);
+    static int done[64] = {0};
+    cudaError_t e0 = ensure_max_smem((const void *)topk_stage1_kernel, (int)smem1, done);
+    if (e0 != cudaSuccess) return e0;
+    dim3 g1(mc, a.num_q);
+    topk_stage1_kernel<<<g1, kTkThreads, smem1, s>>>(a.logits, a.logits_stride, a.c4_seq_lens, a.bs,
+                                                 a.cu_q, a.q_pos, a.max_c4_len, a.pt_stride, mc,
+                                                 ck, ci, a.status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    topk_stage2_kernel<<<a.num_q, kTkThreads, 0, s>>>(a.c4_seq_lens, a.bs, a.cu_q, a.q_pos,
+                                                      a.max_c4_len, a.page_table, a.pt_stride,
+                                                      a.num_slots, mc, ck, ci, a.out_phys,
+                                                      a.out_raw, a.status);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

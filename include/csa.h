@@ -1,0 +1,275 @@
+/*
+ * csa.h -- C ABI of libcsa.so: C4 compressed sparse attention (DeepSeek-V4
+ * style) for NVIDIA B200 (sm_100a).
+ *
+ * The pages this library follows, cited by title and section:
+ *   [T] "Token 的一生：DSV4 架构与 DSpark" (SGLang DSV4 internals article):
+ *       §1 从 DSA 到 DSV4, §2.1 什么是 C4, §2.2 C4 KV Cache 的尺寸,
+ *       §3.1 FP4 量化支持, §3.2 Top-512 变换, §4 Hadamard 旋转
+ *   [H] "DeepSeek-V4 的交錯壓縮注意力（CSA/HCA）：將百萬標記長上下文變為可用資源":
+ *       section "Compressed Sparse Attention（CSA）" and section
+ *       "低精度與儲存策略的配合"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is DEVICE memory owned by the caller, unless its
+ *    comment says otherwise.  The library never allocates device memory;
+ *    scratch space comes from a caller-provided workspace whose size the
+ *    matching *_workspace_size() call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream.
+ *  - Return value: CSA_OK once the work is enqueued.  Arguments that are
+ *    wrong on their face (null required pointer, unsupported size, format or
+ *    page size) return CSA_ERR_INVALID / CSA_ERR_UNSUPPORTED before anything is
+ *    launched; a failed launch returns CSA_ERR_CUDA.
+ *  - `status` (nullable, one int32 in device memory): problems only the
+ *    device can see -- a page id or slot out of range, a NaN logit, a length
+ *    above the stated maximum -- are recorded there as a csa_status_t (the
+ *    first one wins) and the offending element is skipped.  No kernel traps.
+ *    The caller zeroes *status and reads it after synchronising.
+ *  - Paging ([T] §2.2): a page holds PAGE_SIZE = 256 raw tokens; physical
+ *    page p of the compressed cache holds the 64 compressed rows of raw page
+ *    p, so one page table [bs, page_table_stride] (int32 physical page ids)
+ *    serves both caches.  Raw position r of request b lives in raw slot
+ *      page_table[b*stride + r/256]*256 + r%256,
+ *    compressed index s in compressed slot
+ *      page_table[b*stride + s/64]*64 + s%64.
+ *  - A request with L raw tokens (its query tokens included) has
+ *    c4_seq_lens[b] = floor(L/4) compressed rows ([T] §2.2).  A query at raw
+ *    position p sees the compressed rows s < floor((p+1)/4) (blocks whose four
+ *    tokens are all at or before p) and the raw window [max(0,p-W+1), p].
+ *  - Query tokens are packed request-major: request b owns query rows
+ *    cu_q[b] .. cu_q[b+1]-1 (cu_q has bs+1 entries, cu_q[0] = 0).  q_pos
+ *    [num_q] gives each query row's raw position.  Where a call accepts
+ *    q_pos = NULL, every request has exactly one query row, the decode token
+ *    at position L-1, so that it sees all floor(L/4) compressed rows.
+ *
+ * Storage formats
+ * ---------------
+ *  KV row ([H] "低精度與儲存策略的配合": FP8 for most entries, BF16 for RoPE),
+ *  576 channels = 512 latent + 64 RoPE; values are the 512 latent channels:
+ *    CSA_FMT_FP8 : 656 bytes = 512 E4M3 codes | 4 fp32 scales (one per 128
+ *                  latent channels, scale = amax/448, 1 for an all-zero block)
+ *                  | 64 bf16 RoPE values
+ *    CSA_FMT_BF16: 1152 bytes = 576 bf16 values
+ *  Index rows (queries and keys after the Hadamard rotation, [T] §3.1, §4),
+ *  dim Di in {64, 128}; each array is indexed by row (query row or slot):
+ *    CSA_FMT_BF16: codes = Di bf16;            no scales
+ *    CSA_FMT_FP8 : codes = Di E4M3 bytes;       scales[row] fp32 = amax/448
+ *    CSA_FMT_FP4 : codes = Di/2 bytes, two E2M1 codes per byte (element 2i in
+ *                  the low nibble); block_scales = Di/16 unsigned-E4M3 bytes,
+ *                  sb = RN(amax_blk/(6*s)); scales[row] fp32 s = amax/2688
+ *  Every quantised value is rounded to nearest, ties to even, saturating.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID = 1,      /* bad argument found on the host; nothing launched   */
+    CSA_ERR_UNSUPPORTED = 2,  /* well-formed but unsupported size/format            */
+    CSA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed        */
+    CSA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up                 */
+    CSA_ERR_BOUNDS = 5,       /* device saw an index/slot/length out of range       */
+    CSA_ERR_NAN = 6,          /* device saw a NaN logit (ordered as -inf)           */
+    CSA_ERR_WORKSPACE = 7     /* workspace pointer null or smaller than required    */
+} csa_status_t;
+
+typedef enum {
+    CSA_FMT_BF16 = 0,
+    CSA_FMT_FP8 = 1,          /* E4M3 */
+    CSA_FMT_FP4 = 2,          /* E2M1 with block-16 unsigned-E4M3 scales */
+    CSA_FMT_F32 = 3           /* input-only: float32 */
+} csa_fmt_t;
+
+/* What csa_c4_compress writes. */
+typedef enum {
+    CSA_OUT_KV_BF16 = 0,      /* dim 576, KV row in CSA_FMT_BF16 into the compressed KV cache */
+    CSA_OUT_KV_FP8 = 1,       /* dim 576, KV row in CSA_FMT_FP8                               */
+    CSA_OUT_INDEX_BF16 = 2,   /* dim 64/128, rotated index key, bf16 codes                    */
+    CSA_OUT_INDEX_FP8 = 3,    /* dim 64/128, rotated index key, FP8 codes + row scale          */
+    CSA_OUT_INDEX_FP4 = 4     /* dim 64/128, rotated index key, FP4 codes + block/row scales   */
+} csa_out_kind_t;
+
+enum { CSA_TOPK = 512, CSA_PAGE_SIZE = 256, CSA_C4_PAGE_SIZE = 64, CSA_C4_RATIO = 4,
+       CSA_KV_DIM = 576, CSA_KV_LATENT = 512, CSA_KV_ROPE = 64 };
+
+/* Human-readable name of a status code (static storage). */
+const char *csa_status_string(csa_status_t s);
+
+/* ABI version of this header (bumped on any signature change). */
+int32_t csa_abi_version(void);
+
+/* Bytes of one KV row in `kv_fmt` (656 or 1152), 0 for an unknown format. */
+int32_t csa_kv_row_bytes(int32_t kv_fmt);
+
+/*
+ * csa_kv_store -- write raw or compressed KV rows into a paged KV cache.
+ * ([H] "低精度與儲存策略的配合": FP8 latent with BF16 RoPE.)
+ *   rows      [n, 576] float32, row-major
+ *   slots     [n] int32 destination row of each input row; negative = skip
+ *   kv_fmt    CSA_FMT_FP8 or CSA_FMT_BF16
+ *   cache     [num_slots, csa_kv_row_bytes(kv_fmt)] bytes
+ * A slot >= num_slots records CSA_ERR_BOUNDS and is skipped.
+ */
+csa_status_t csa_kv_store(const float *rows, int64_t n, const int32_t *slots, int32_t kv_fmt,
+                          void *cache, int64_t num_slots, int32_t *status, void *stream);
+
+/*
+ * csa_c4_compress -- step 1, the C4 compressor ([T] §2.1; [H] "Compressed
+ * Sparse Attention（CSA）": softmax-gated pooling with a learned positional
+ * bias).  Block j of a request pools raw rows 4j..4j+3:
+ *   alpha_i[c] = softmax_i(gate[4j+i][c] + bias[i][c]),  y[j][c] = sum_i alpha_i[c] x[4j+i][c]
+ * computed in float32 and rounded once into the output format.  Only
+ * complete blocks are written (a block is compressed when its fourth token
+ * arrives); trailing rows of an incomplete block are ignored.
+ *   x, gate   [cu_x[bs], dim] float32: the new raw rows of every request,
+ *             request b owning rows cu_x[b] .. cu_x[b+1]-1 (host copy of the
+ *             total: total_rows)
+ *   bias      [4, dim] float32, indexed by position inside the block
+ *   start_pos [bs] raw position of each request's first new row; must be a
+ *             multiple of 4 (else CSA_ERR_BOUNDS for that request)
+ *   max_rows_per_req  host upper bound on cu_x[b+1]-cu_x[b]; rows beyond it
+ *             record CSA_ERR_BOUNDS and are not compressed
+ *   out_kind  see csa_out_kind_t.  KV kinds need dim = 576 and write `out`
+ *             as KV rows of a compressed KV cache.  INDEX kinds need dim 64 or
+ *             128 and apply the Hadamard rotation (1/sqrt(dim)) H x ([T] §4)
+ *             before quantising into the index-key arrays out (codes),
+ *             out_block_scales (FP4 only) and out_scales (FP8/FP4).
+ *   Compressed index j of request b is written to compressed slot
+ *   page_table[b*stride + j/64]*64 + j%64 (< num_slots).
+ */
+csa_status_t csa_c4_compress(const float *x, const float *gate, const float *bias, int32_t dim,
+                             int32_t bs, const int32_t *cu_x, int64_t total_rows,
+                             const int32_t *start_pos, int32_t max_rows_per_req,
+                             const int32_t *page_table, int32_t page_table_stride,
+                             int32_t out_kind, void *out, uint8_t *out_block_scales,
+                             float *out_scales, int64_t num_slots, int32_t *status, void *stream);
+
+/*
+ * csa_hadamard_quant -- the rotation and quantisation of index queries or
+ * keys ([T] §3.1 fused_q_indexer_rope_hadamard[_fp4]_quant, §4; the RoPE step
+ * is upstream of this call): x' = (1/sqrt(dim)) H_dim x per row, then
+ * quantised to `fmt` as described above.
+ *   x         [rows, dim] in x_dtype (CSA_FMT_BF16 or CSA_FMT_F32)
+ *   dim       64 or 128
+ *   row_map   nullable [rows] int32: output row of input row r (for writing
+ *             keys straight into a paged index cache); NULL = identity.
+ *             Negative = skip; >= num_out_rows records CSA_ERR_BOUNDS.
+ *   codes, block_scales, scales: output arrays indexed by output row
+ *   w_in/w_out nullable [rows] float32, indexed by INPUT row: the head-gate
+ *             fusion of [T] §3.1: w_out[r] = w_in[r] * scales[r] (the row
+ *             scale is positive, so it commutes with the indexer's ReLU);
+ *             for bf16 w_out = w_in.
+ */
+csa_status_t csa_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                                int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
+                                void *codes, uint8_t *block_scales, float *scales,
+                                const float *w_in, float *w_out, int32_t *status, void *stream);
+
+/*
+ * csa_indexer_logits -- step 2, the C4 indexer scores ([T] §1, §3.1;
+ * [H] "Compressed Sparse Attention（CSA）": a light indexer in low precision):
+ *   logits[t][s] = k_scale[s] * sum_h w'[t][h] * ReLU(qhat[t][h] . khat[s])
+ * where qhat/khat are the stored codes' values (FP4: times their block
+ * scales) and w' = w * q_scale already folds the query's row scale in
+ * (csa_hadamard_quant's w_out).  Accumulation in float32.
+ *   q_codes        [num_q, idx_heads, code bytes of one row]
+ *   q_block_scales [num_q, idx_heads, dim/16] (FP4 only, else NULL)
+ *   q_weights      [num_q, idx_heads] float32 (w')
+ *   k_codes, k_block_scales, k_scales: the index-key arrays, indexed by
+ *                  compressed slot (< num_slots)
+ *   q_pos          nullable [num_q]: query raw positions (causal visibility
+ *                  n_vis = min(c4_seq_lens[b], floor((p+1)/4))); NULL means
+ *                  n_vis = c4_seq_lens[b]
+ *   max_c4_len     host upper bound on c4_seq_lens[] (grid sizing); longer
+ *                  rows record CSA_ERR_BOUNDS and are truncated
+ *   logits         [num_q, logits_stride] float32; entries s >= n_vis of a
+ *                  row are not written
+ */
+csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
+                                const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                const uint8_t *k_block_scales, const float *k_scales,
+                                int64_t num_slots, const int32_t *page_table,
+                                int32_t page_table_stride, const int32_t *c4_seq_lens,
+                                int32_t bs, const int32_t *cu_q, const int32_t *q_pos,
+                                int32_t max_c4_len, float *logits, int64_t logits_stride,
+                                int32_t *status, void *stream);
+
+/*
+ * csa_topk512_page_transform -- step 3, topk_transform_512 ([T] §3.2, with
+ * the page arithmetic of §2.2).  For each query row t of request b: among
+ * the first n_vis logits (n_vis as in csa_indexer_logits) select the
+ * min(512, n_vis) largest, ties broken toward the lower index (-0 == +0;
+ * a NaN records CSA_ERR_NAN and ranks below -inf), and write them in
+ * ascending logical order followed by -1 padding:
+ *   c4_sparse_page_indices[t][i] = page_table[b*stride + s/64]*64 + s%64
+ *   raw_indices[t][i]            = s            (nullable output)
+ *   c4_page_size   must be 64 (= 256/4)
+ *   workspace      >= csa_topk512_workspace_size(num_q, max_c4_len) bytes
+ */
+size_t csa_topk512_workspace_size(int32_t num_q, int32_t max_c4_len);
+csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stride,
+                                        int32_t num_q, const int32_t *c4_seq_lens, int32_t bs,
+                                        const int32_t *cu_q, const int32_t *q_pos,
+                                        const int32_t *page_table, int32_t page_table_stride,
+                                        int64_t num_slots, int32_t c4_page_size,
+                                        int32_t max_c4_len, int32_t *c4_sparse_page_indices,
+                                        int32_t *raw_indices, void *workspace,
+                                        size_t workspace_bytes, int32_t *status, void *stream);
+
+/*
+ * csa_sparse_mqa_decode / csa_sparse_mqa_prefill -- step 4, sparse attention
+ * over the selected compressed rows joined with the sliding window of raw
+ * rows under ONE softmax ([T] §1; [H] "Compressed Sparse Attention（CSA）").
+ * For query t of request b at raw position p and head h, with key rows
+ *   S = { compressed slot c4_sparse_page_indices[t][i] >= 0 }
+ *     U { raw slot of r : max(0, p-window+1) <= r <= p }:
+ *   z_r = sm_scale * q[t][h] . key_r (576 dims),
+ *   out[t][h] = sum_r softmax(z)_r * key_r[0:512],  lse[t][h] = ln sum_r exp(z_r).
+ * A raw token may appear both in the window and inside a selected
+ * compressed row; both count.
+ *   q         [num_q, heads, 576] bf16;  heads in {16, 32, 64, 128}
+ *   c4_cache  [num_c4_slots, row bytes]; raw_cache [num_raw_slots, row bytes]
+ *   seq_lens  [bs] raw lengths L (q_pos NULL => one query per request at L-1)
+ *   window    0..1024
+ *   out       [num_q, heads, 512] bf16;  lse nullable [num_q, heads] float32
+ *   workspace >= csa_sparse_mqa_workspace_size(num_q, heads, window, decode)
+ * The two entry points compute the same function; _decode splits each
+ * query's rows across CTAs (few queries, many rows each), _prefill gives each
+ * query its own CTA (many queries).
+ */
+size_t csa_sparse_mqa_workspace_size(int32_t num_q, int32_t heads, int32_t window,
+                                     int32_t decode);
+csa_status_t csa_sparse_mqa_decode(const void *q, int32_t num_q, int32_t heads,
+                                   const void *c4_cache, const void *raw_cache, int32_t kv_fmt,
+                                   int64_t num_c4_slots, int64_t num_raw_slots,
+                                   const int32_t *c4_sparse_page_indices,
+                                   const int32_t *page_table, int32_t page_table_stride,
+                                   const int32_t *seq_lens, int32_t bs, const int32_t *cu_q,
+                                   const int32_t *q_pos, int32_t window, float sm_scale,
+                                   void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, int32_t *status, void *stream);
+csa_status_t csa_sparse_mqa_prefill(const void *q, int32_t num_q, int32_t heads,
+                                    const void *c4_cache, const void *raw_cache, int32_t kv_fmt,
+                                    int64_t num_c4_slots, int64_t num_raw_slots,
+                                    const int32_t *c4_sparse_page_indices,
+                                    const int32_t *page_table, int32_t page_table_stride,
+                                    const int32_t *seq_lens, int32_t bs, const int32_t *cu_q,
+                                    const int32_t *q_pos, int32_t window, float sm_scale,
+                                    void *out, float *lse, void *workspace,
+                                    size_t workspace_bytes, int32_t *status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -382,3 +382,78 @@ def window_positions(pos: int, window: int) -> np.ndarray:
 def raw_slot(page_table_row: np.ndarray, pos: np.ndarray, page_size: int = PAGE_SIZE):
     pos = np.asarray(pos, dtype=np.int64)
     return page_table_row[pos // page_size].astype(np.int64) * page_size + pos % page_size
+
+
+# ---------------------------------------------------------------- whole step
+
+def _t2n(x):
+    """A torch tensor or numpy array as float64 numpy (exact for bf16/f32)."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu()
+        if str(x.dtype) == "torch.bfloat16":
+            x = x.float()
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def step(w, data, page_table, requests=None, sm_scale=None):
+    """One decode/prefill step of C4 compressed sparse attention, composed from
+    the steps above in the pages' order ([T] §1-§4; [H] "Compressed Sparse
+    Attention（CSA）"), for the requests listed (default: all).
+
+    w is the workload's shape record and data its drawn inputs (the same
+    buffers the GPU path reads).  The oracle keeps its own copies of the
+    caches, quantised by its own codecs.  Returns a dict keyed by query row
+    with the logical top-k indices, the logits, the output and the lse."""
+    import math
+    sm_scale = 1.0 / math.sqrt(KV_DIM) if sm_scale is None else sm_scale
+    fp8_kv = w.kv_fmt == "fp8"
+    bs = w.bs
+    requests = range(bs) if requests is None else requests
+    direct = np.asarray(w.direct_c4_lens)
+    d_off = np.concatenate([[0], np.cumsum(direct)])
+    n_off = np.asarray(w.cu_new)
+    q_off = np.asarray(w.cu_q)
+    q_pos = np.asarray(w.q_pos)
+    raw_req = np.asarray(data["raw_req"])
+    raw_pos = np.asarray(data["raw_pos"])
+    out = {}
+    for b in requests:
+        L = int(w.seq_lens[b])
+        # compressed rows: drawn directly, then the compressor's blocks ([T] §2.1)
+        kv = _t2n(data["kv_c4"][d_off[b]:d_off[b + 1]])
+        ik = _t2n(data["idx_k"][d_off[b]:d_off[b + 1]])
+        if w.new_tokens[b] >= 4:
+            sl = slice(n_off[b], n_off[b + 1])
+            kv = np.concatenate([kv, c4_compress(_t2n(data["raw_kv"][sl]), _t2n(data["gate"][sl]),
+                                                 _t2n(data["bias"]))])
+            ik = np.concatenate([ik, c4_compress(_t2n(data["raw_idx_k"][sl]),
+                                                 _t2n(data["idx_gate"][sl]),
+                                                 _t2n(data["idx_bias"]))])
+        n_c4 = c4_len(L)
+        assert kv.shape[0] == n_c4 and ik.shape[0] == n_c4
+        kv_deq = kv_decode_rows(kv_encode_rows(kv, fp8_kv), fp8_kv)
+        k_deq = index_quantise(ik, w.idx_fmt)["deq"]
+        # raw rows of this request, by position
+        sel = raw_req == b
+        raw_rows = dict(zip(raw_pos[sel].tolist(),
+                            kv_decode_rows(kv_encode_rows(_t2n(data["kv_raw"][sel]), fp8_kv),
+                                           fp8_kv)))
+        qs = slice(q_off[b], q_off[b + 1])
+        qi = index_quantise(_t2n(data["q_idx"][qs]), w.idx_fmt)["deq"]
+        ww = _t2n(data["w"][qs])
+        pos = q_pos[qs]
+        nv = np.array([min(n_c4, n_visible(int(p))) for p in pos], dtype=np.int64)
+        lg = indexer_logits(qi, ww, k_deq, nv) if n_c4 else np.zeros((len(pos), 0))
+        qa = _t2n(data["q"][qs])
+        for j, p in enumerate(pos):
+            t = int(q_off[b] + j)
+            phys, logical = topk_transform(lg[j], int(nv[j]), page_table[b], 1 << 40, k=w.topk)
+            chosen = logical[logical >= 0]
+            win = window_positions(int(p), w.window)
+            rows = np.concatenate([kv_deq[chosen].reshape(-1, KV_DIM),
+                                   np.array([raw_rows[int(r)] for r in win]).reshape(-1, KV_DIM)])
+            o, lse = sparse_attention(qa[j], rows, sm_scale)
+            out[t] = {"logical": logical, "phys": phys, "logits": lg[j, :nv[j]], "out": o,
+                      "lse": lse, "n_vis": int(nv[j])}
+    return out

@@ -1,0 +1,64 @@
+"""Helpers for the GPU parity tests: lay out oracle-produced codes in the
+library's array formats (a test-side marshalling step; the arithmetic
+stays on each side) and compare results."""
+import numpy as np
+import torch
+
+from oracle import oracle as orc
+
+
+def dev(a):
+    return torch.as_tensor(np.ascontiguousarray(a), device="cuda")
+
+
+def code_bytes(fmt, dim):
+    return {"bf16": 2 * dim, "fp8": dim, "fp4": dim // 2}[fmt]
+
+
+def index_arrays(q, fmt, dim, n_rows, rows=None):
+    """Oracle index quantisation result `q` (orc.index_quantise) written into
+    [n_rows] library arrays at row indices `rows` (default 0..)."""
+    n = q["deq"].reshape(-1, dim).shape[0]
+    rows = np.arange(n) if rows is None else np.asarray(rows)
+    codes = np.zeros((n_rows, code_bytes(fmt, dim)), dtype=np.uint8)
+    bsc = np.zeros((n_rows, dim // 16), dtype=np.uint8) if fmt == "fp4" else None
+    sc = np.ones(n_rows, dtype=np.float32) if fmt != "bf16" else None
+    if fmt == "bf16":
+        codes[rows] = q["codes"].reshape(n, dim).astype(np.uint16).view(np.uint8).reshape(n, -1)
+    elif fmt == "fp8":
+        codes[rows] = q["codes"].reshape(n, dim)
+        sc[rows] = q["scales"].reshape(n)
+    else:
+        codes[rows] = q["packed"].reshape(n, dim // 2)
+        bsc[rows] = q["block_scales"].reshape(n, dim // 16)
+        sc[rows] = q["scales"].reshape(n)
+    return (dev(codes), dev(bsc) if bsc is not None else None,
+            dev(sc) if sc is not None else None)
+
+
+def decode_index_rows(codes, bsc, sc, fmt, dim):
+    """Oracle-side decode of library index arrays (host numpy) to float64."""
+    codes = np.asarray(codes)
+    if fmt == "bf16":
+        return orc.bf16_to_f64(codes.view(np.uint16).reshape(-1, dim))
+    if fmt == "fp8":
+        return orc.dequant_fp8_rows(codes, sc)
+    return orc.dequant_fp4_rows(orc.unpack_fp4(codes), bsc, sc)
+
+
+def code_values(codes, fmt, dim):
+    """Per-element code values (no scales) of library arrays, float64."""
+    codes = np.asarray(codes)
+    if fmt == "bf16":
+        return orc.bf16_to_f64(codes.view(np.uint16).reshape(-1, dim))
+    if fmt == "fp8":
+        return orc.e4m3_table()[codes]
+    return orc.e2m1_table()[orc.unpack_fp4(codes)]
+
+
+def rel_close(got, ref, rel, floor_frac=1e-3, axis=-1):
+    """|got-ref| <= rel * max(|ref|, floor_frac * max|ref| along axis)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = np.maximum(np.abs(ref), floor_frac * np.abs(ref).max(axis=axis, keepdims=True))
+    return np.abs(got - ref) <= rel * scale + 1e-30

@@ -1,0 +1,124 @@
+"""The C ABI library loads on a machine without a GPU, exports every entry
+point include/csa.h declares, and rejects malformed arguments on the host
+before any launch (no GPU calls are made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from compressed_sparse_attention_12_b200 import build, csa
+    build.build()
+    return csa.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    from compressed_sparse_attention_12_b200 import csa
+    assert set(names) <= set(csa.EXPORTED) | {"csa_status_string"}
+
+
+def test_status_strings_and_constants(L):
+    from compressed_sparse_attention_12_b200 import csa
+    assert csa.status_string(0) == "ok"
+    for c in range(1, 8):
+        assert csa.status_string(c) not in ("ok", "unknown status")
+    assert csa.status_string(99) == "unknown status"
+    assert csa.csa_abi_version() == 1
+    assert csa.csa_kv_row_bytes(csa.CSA_FMT_FP8) == 656
+    assert csa.csa_kv_row_bytes(csa.CSA_FMT_BF16) == 1152
+    assert csa.csa_kv_row_bytes(7) == 0
+
+
+def test_workspace_sizes(L):
+    from compressed_sparse_attention_12_b200 import csa
+    assert csa.csa_topk512_workspace_size(0, 100) == 0
+    # one chunk of 8192 candidates per row, (key, index) pairs of 512
+    assert csa.csa_topk512_workspace_size(3, 8192) == 3 * 1 * 512 * 8
+    assert csa.csa_topk512_workspace_size(3, 8193) == 3 * 2 * 512 * 8
+    assert csa.csa_topk512_workspace_size(8, 262144) == 8 * 32 * 512 * 8
+    assert csa.csa_sparse_mqa_workspace_size(4096, 64, 128, 0) == 0
+    assert csa.csa_sparse_mqa_workspace_size(32, 64, 128, 1) > 0
+
+
+def _p(v=1):
+    return ctypes.c_void_p(v * 256)   # never dereferenced: host checks fail first
+
+
+def test_host_validation_rejects_before_launch(L):
+    from compressed_sparse_attention_12_b200 import csa
+    # page size other than 64
+    r = L.csa_topk512_page_transform(_p(), 64, 1, _p(), 1, _p(), None, _p(), 4, 256, 32, 64,
+                                     _p(), None, _p(), 1 << 20, None, None)
+    assert r == csa.CSA_ERR_INVALID
+    # workspace too small
+    r = L.csa_topk512_page_transform(_p(), 64, 1, _p(), 1, _p(), None, _p(), 4, 256, 64, 64,
+                                     _p(), None, _p(), 8, None, None)
+    assert r == csa.CSA_ERR_WORKSPACE
+    # unsupported index dim / format / heads
+    r = L.csa_hadamard_quant(_p(), csa.CSA_FMT_BF16, 4, 96, csa.CSA_FMT_FP8, None, 0, _p(), None,
+                             _p(), None, None, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    r = L.csa_hadamard_quant(_p(), csa.CSA_FMT_BF16, 4, 128, 9, None, 0, _p(), None, _p(), None,
+                             None, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    # FP4 without block scales
+    r = L.csa_hadamard_quant(_p(), csa.CSA_FMT_BF16, 4, 128, csa.CSA_FMT_FP4, None, 0, _p(), None,
+                             _p(), None, None, None, None)
+    assert r == csa.CSA_ERR_INVALID
+    r = L.csa_indexer_logits(_p(), None, _p(), 1, 200, 128, csa.CSA_FMT_FP8, _p(), None, _p(), 64,
+                             _p(), 1, _p(), 1, _p(), None, 64, _p(), 64, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    # logits row stride shorter than the longest row
+    r = L.csa_indexer_logits(_p(), None, _p(), 1, 64, 128, csa.CSA_FMT_FP8, _p(), None, _p(), 64,
+                             _p(), 1, _p(), 1, _p(), None, 100, _p(), 64, None, None)
+    assert r == csa.CSA_ERR_INVALID
+    # KV compress needs dim 576; index compress needs 64/128
+    r = L.csa_c4_compress(_p(), _p(), _p(), 512, 1, _p(), 8, _p(), 8, _p(), 4,
+                          csa.CSA_OUT_KV_FP8, _p(), None, None, 64, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    r = L.csa_c4_compress(_p(), _p(), _p(), 576, 1, _p(), 8, _p(), 8, _p(), 4,
+                          csa.CSA_OUT_INDEX_FP8, _p(), None, None, 64, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    # attention: heads not a multiple of 16, window out of range, bad KV format
+    args = [_p(), 1, 24, _p(), _p(), csa.CSA_FMT_FP8, 64, 256, _p(), _p(), 1, _p(), 1, _p(), None,
+            128, 0.1, _p(), None, _p(), 1 << 30, None, None]
+    assert L.csa_sparse_mqa_decode(*args) == csa.CSA_ERR_UNSUPPORTED
+    args[2] = 64
+    args[15] = 5000
+    assert L.csa_sparse_mqa_decode(*args) == csa.CSA_ERR_UNSUPPORTED
+    args[15] = 128
+    args[5] = csa.CSA_FMT_FP4
+    assert L.csa_sparse_mqa_prefill(*args) == csa.CSA_ERR_UNSUPPORTED
+    # q_pos NULL needs one query per request
+    args[5] = csa.CSA_FMT_FP8
+    args[1] = 3
+    assert L.csa_sparse_mqa_prefill(*args) == csa.CSA_ERR_INVALID
+    # empty work is a no-op
+    assert L.csa_kv_store(None, 0, None, csa.CSA_FMT_FP8, None, 0, None, None) == csa.CSA_OK
+    assert L.csa_kv_store(None, 4, None, 5, None, 0, None, None) == csa.CSA_ERR_UNSUPPORTED
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The library package never imports or loads the oracle."""
+    pkg = os.path.join(ROOT, "compressed_sparse_attention_12_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"(import|from)\s+oracle|liboracle|csa_oracle", txt), f
