@@ -12,10 +12,14 @@
 //
 // One CTA (4 warps) owns one query, 16 heads and a contiguous range of the
 // query's row list (a "split").  Rows are gathered 64 at a time into shared
-// memory as bf16 (FP8 rows dequantised on the way in); S = Q K^T and O += P V
-// run on bf16 mma.sync tensor-core instructions with an online softmax in
-// float32 (base-2 exponent).  Splits write unnormalised partials that a
-// second kernel merges; a single split finalises in place.
+// memory as bf16: BF16 rows as stored, FP8 rows as their E4M3 codes (exact in
+// bf16) with the four per-128-channel scales kept aside in float32.
+// S = Q K^T runs on bf16 mma.sync tensor-core instructions per 128-channel
+// block, each block's partial sum scaled by its row scale in float32; the
+// online softmax is float32 (base-2 exponent); O += P V splits P (times the
+// value block's row scale) into a bf16 high part and a bf16 remainder so the
+// probabilities keep ~16 significant bits.  Splits write unnormalised
+// partials that a second kernel merges; a single split finalises in place.
 #include "common.cuh"
 #include "launch.h"
 
@@ -25,13 +29,14 @@ constexpr int kAtThreads = 128;
 constexpr int kAtRows = 64;                 // rows per tile
 constexpr int kAtHeads = 16;                // heads per CTA
 constexpr int kAtStride = kKvDim + 8;       // bf16 elements per smem row (bank-conflict pad)
-constexpr int kAtPStride = kAtRows + 8;
+constexpr int kAtPStride = kAtRows + 8;   // floats per P row
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AtSmem {
     __nv_bfloat16 q[kAtHeads * kAtStride];
     __nv_bfloat16 kv[kAtRows * kAtStride];
-    __nv_bfloat16 p[kAtHeads * kAtPStride];
+    float p[kAtHeads * kAtPStride];         // probabilities of the tile, float32
+    float rscale[kAtRows][4];               // per-row scales of the 4 latent blocks
     float red_max[4][kAtHeads];
     float red_sum[4][kAtHeads];
     int32_t slot[kAtRows];                  // >= 0: row slot; -1: masked
@@ -122,6 +127,10 @@ __device__ void load_tile(const AttnArgs &a, const AtQuery &qq, int t, int r0, A
     const uint8_t *c4 = reinterpret_cast<const uint8_t *>(a.c4_cache);
     const uint8_t *rc = reinterpret_cast<const uint8_t *>(a.raw_cache);
     if (a.kv_fmt == CSA_FMT_BF16) {
+        if (tid < kAtRows) {
+            const float one = sm.slot[tid] >= 0 ? 1.0f : 0.0f;
+            sm.rscale[tid][0] = sm.rscale[tid][1] = sm.rscale[tid][2] = sm.rscale[tid][3] = one;
+        }
         // 72 chunks of 16 B per row
         for (int u = tid; u < kAtRows * 72; u += kAtThreads) {
             const int r = u / 72, c = u % 72;
@@ -136,7 +145,18 @@ __device__ void load_tile(const AttnArgs &a, const AtQuery &qq, int t, int r0, A
         }
         cp_async_wait_all();
     } else {
-        // 32 code chunks (16 E4M3 -> 16 bf16) + 8 RoPE chunks per row
+        if (tid < kAtRows) {
+            const int32_t slot = sm.slot[tid];
+            float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (slot >= 0)
+                sc = *reinterpret_cast<const float4 *>((sm.is_raw[tid] ? rc : c4) +
+                                                       (int64_t)slot * row_bytes + 512);
+            sm.rscale[tid][0] = sc.x;
+            sm.rscale[tid][1] = sc.y;
+            sm.rscale[tid][2] = sc.z;
+            sm.rscale[tid][3] = sc.w;
+        }
+        // 32 code chunks (16 E4M3 codes -> 16 exact bf16) + 8 RoPE chunks per row
         for (int u = tid; u < kAtRows * 40; u += kAtThreads) {
             const int r = u / 40, c = u % 40;
             const int32_t slot = sm.slot[r];
@@ -149,15 +169,14 @@ __device__ void load_tile(const AttnArgs &a, const AtQuery &qq, int t, int r0, A
             const uint8_t *row = (sm.is_raw[r] ? rc : c4) + (int64_t)slot * row_bytes;
             if (c < 32) {
                 const uint4 u4 = *reinterpret_cast<const uint4 *>(row + c * 16);
-                const float sc = *reinterpret_cast<const float *>(row + 512 + 4 * (c / 8));
                 const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
                 uint32_t o[8];
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     const float2 lo = e4m3x2_to_f32x2((uint16_t)(w[j] & 0xFFFF));
                     const float2 hi = e4m3x2_to_f32x2((uint16_t)(w[j] >> 16));
-                    o[2 * j] = pack_bf16(lo.x * sc, lo.y * sc);
-                    o[2 * j + 1] = pack_bf16(hi.x * sc, hi.y * sc);
+                    o[2 * j] = pack_bf16(lo.x, lo.y);
+                    o[2 * j + 1] = pack_bf16(hi.x, hi.y);
                 }
                 *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
                 *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
@@ -210,7 +229,9 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
         }
         load_tile(a, qq, t, r0, sm);
 
-        // S = Q K^T: warp w covers rows 16w..16w+15 (two n-tiles of 8)
+        // S = Q K^T: warp w covers rows 16w..16w+15 (two n-tiles of 8).  Each
+        // 128-channel latent block accumulates separately and is folded in
+        // with its row scale; the RoPE block has scale 1.
         float s[2][4];
 #pragma unroll
         for (int i = 0; i < 2; i++) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.0f;
@@ -220,13 +241,29 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
         const uint32_t k_base = smem_u32(sm.kv) +
                                 (uint32_t)((warp * 16 + (lane & 7) + (lane >> 4) * 8) * kAtStride +
                                            ((lane >> 3) & 1) * 8) * 2;
+#pragma unroll 1
+        for (int blk = 0; blk < 5; blk++) {
+            float acc[2][4];
+#pragma unroll
+            for (int i = 0; i < 2; i++) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+            const int k0 = blk * 8, nk = blk < 4 ? 8 : 4;
 #pragma unroll 4
-        for (int kk = 0; kk < kKvDim / 16; kk++) {
-            uint32_t af[4], bf[4];
-            ldsm_x4(af, q_base + kk * 32);
-            ldsm_x4(bf, k_base + kk * 32);
-            mma16816(s[0], af, bf[0], bf[1]);
-            mma16816(s[1], af, bf[2], bf[3]);
+            for (int kk = k0; kk < k0 + nk; kk++) {
+                uint32_t af[4], bf[4];
+                ldsm_x4(af, q_base + kk * 32);
+                ldsm_x4(bf, k_base + kk * 32);
+                mma16816(acc[0], af, bf[0], bf[1]);
+                mma16816(acc[1], af, bf[2], bf[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; nt++) {
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int row = warp * 16 + nt * 8 + 2 * tq + (j & 1);
+                    const float sc = blk < 4 ? sm.rscale[row][blk] : 1.0f;
+                    s[nt][j] = fmaf(acc[nt][j], sc, s[nt][j]);
+                }
+            }
         }
         // scale, mask, per-head tile max
         float tmax[2] = {-INFINITY, -INFINITY};
@@ -270,9 +307,9 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
                 psum[h] += pv;
             }
             const int col = warp * 16 + nt * 8 + 2 * tq;
-            *reinterpret_cast<uint32_t *>(sm.p + gq * kAtPStride + col) = pack_bf16(s[nt][0], s[nt][1]);
-            *reinterpret_cast<uint32_t *>(sm.p + (gq + 8) * kAtPStride + col) =
-                pack_bf16(s[nt][2], s[nt][3]);
+            *reinterpret_cast<float2 *>(sm.p + gq * kAtPStride + col) = make_float2(s[nt][0], s[nt][1]);
+            *reinterpret_cast<float2 *>(sm.p + (gq + 8) * kAtPStride + col) =
+                make_float2(s[nt][2], s[nt][3]);
         }
 #pragma unroll
         for (int h = 0; h < 2; h++) {
@@ -299,23 +336,42 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             o[i][2] *= alpha[1];
             o[i][3] *= alpha[1];
         }
-        // O[:, 128w:128w+128] += P V
-        const uint32_t p_base = smem_u32(sm.p) +
-                                (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtPStride +
-                                           (lane >> 4) * 8) * 2;
+        // O[:, 128w:128w+128] += (P * rowscale_w) V, P split into bf16 hi + lo
+        // (this warp's output columns are exactly latent block w).
+        __syncthreads();
         const uint32_t v_base = smem_u32(sm.kv) +
                                 (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
                                            warp * 128 + (lane >> 4) * 8) * 2;
 #pragma unroll
         for (int ks = 0; ks < kAtRows / 16; ks++) {
-            uint32_t af[4];
-            ldsm_x4(af, p_base + ks * 32);
+            const int r0k = ks * 16 + 2 * tq;
+            float pv[8];
+            const float2 p00 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k);
+            const float2 p10 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k);
+            const float2 p01 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k + 8);
+            const float2 p11 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k + 8);
+            const float c0 = sm.rscale[r0k][warp], c1 = sm.rscale[r0k + 1][warp];
+            const float c8 = sm.rscale[r0k + 8][warp], c9 = sm.rscale[r0k + 9][warp];
+            pv[0] = p00.x * c0; pv[1] = p00.y * c1;     // a0: head g,   rows r, r+1
+            pv[2] = p10.x * c0; pv[3] = p10.y * c1;     // a1: head g+8, rows r, r+1
+            pv[4] = p01.x * c8; pv[5] = p01.y * c9;     // a2: head g,   rows r+8, r+9
+            pv[6] = p11.x * c8; pv[7] = p11.y * c9;     // a3: head g+8, rows r+8, r+9
+            uint32_t ah[4], al[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const uint16_t h0 = f32_to_bf16_bits(pv[2 * i]), h1 = f32_to_bf16_bits(pv[2 * i + 1]);
+                ah[i] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                al[i] = pack_bf16(pv[2 * i] - bf16_bits_to_f32(h0),
+                                  pv[2 * i + 1] - bf16_bits_to_f32(h1));
+            }
 #pragma unroll
             for (int np = 0; np < 8; np++) {
                 uint32_t bf[4];
                 ldsm_x4_t(bf, v_base + (uint32_t)(ks * 16 * kAtStride + np * 16) * 2);
-                mma16816(o[2 * np], af, bf[0], bf[1]);
-                mma16816(o[2 * np + 1], af, bf[2], bf[3]);
+                mma16816(o[2 * np], ah, bf[0], bf[1]);
+                mma16816(o[2 * np], al, bf[0], bf[1]);
+                mma16816(o[2 * np + 1], ah, bf[2], bf[3]);
+                mma16816(o[2 * np + 1], al, bf[2], bf[3]);
             }
         }
         __syncthreads();   // smem tile reused by the next load

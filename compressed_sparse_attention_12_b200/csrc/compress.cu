@@ -198,8 +198,12 @@ __device__ __forceinline__ int64_t compress_target(int b, int blk, const int32_t
                                                    int64_t num_slots, int32_t *status,
                                                    int64_t *row0, bool leader) {
     const int32_t x0 = cu_x[b], n = cu_x[b + 1] - x0;
+    if (n < 4) {                      // no complete block: nothing to compress
+        if (n < 0 && leader && blk == 0) report(status, CSA_ERR_BOUNDS);
+        return -1;
+    }
     const int32_t sp = start_pos[b];
-    if (n < 0 || sp < 0 || (sp & 3) != 0) {
+    if (sp < 0 || (sp & 3) != 0) {
         if (leader && blk == 0) report(status, CSA_ERR_BOUNDS);
         return -1;
     }

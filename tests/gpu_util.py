@@ -62,3 +62,18 @@ def rel_close(got, ref, rel, floor_frac=1e-3, axis=-1):
     ref = np.asarray(ref, dtype=np.float64)
     scale = np.maximum(np.abs(ref), floor_frac * np.abs(ref).max(axis=axis, keepdims=True))
     return np.abs(got - ref) <= rel * scale + 1e-30
+
+
+def bf16_bound(ref, rel=2e-3, floor=None):
+    """Error bound for a value computed in float32 and rounded once to bf16:
+    the stated relative tolerance, or half a bf16 ulp of the reference where
+    that is larger (2e-3 lies below bf16's half-ulp in the lower part of
+    every binade, up to 2^-8 relative), plus an optional absolute term for
+    the float32 error of the value before its rounding (cancellation)."""
+    ref = np.abs(np.asarray(ref, dtype=np.float64))
+    e = np.floor(np.log2(np.where(ref > 0, ref, 1.0)))
+    half_ulp = np.where(ref > 0, 2.0 ** (e - 8), 0.0) * (1 + 2.0 ** -10)
+    b = np.maximum(rel * ref, half_ulp)
+    if floor is not None:
+        b = b + floor    # float32 rounding before the bf16 rounding adds to it
+    return b

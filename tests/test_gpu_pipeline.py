@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import dev, index_arrays, rel_close
+from gpu_util import bf16_bound, dev, index_arrays, rel_close
 from oracle import oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -59,7 +59,7 @@ def test_step_end_to_end(name, scale):
         assert np.array_equal(phys[t][:len(g)], batch.pt_host[b, g // 64] * 64 + g % 64)
         if got == want:
             exact += 1
-            assert np.abs(out[t] - r["out"]).max() <= tol, t
+            assert (np.abs(out[t] - r["out"]) - bf16_bound(r["out"], rel=0.0)).max() <= tol, t
     print(f"\n{name}: mean top-512 overlap {np.mean(overlaps):.5f}, "
           f"min {np.min(overlaps):.5f}, identical sets {exact}/{len(ref)}")
     assert np.mean(overlaps) >= 0.98
@@ -150,7 +150,7 @@ def _full_index_check(name, sample_q):
     go_ = o.float().cpu().numpy()
     tol = 2e-2 if fp8 else 5e-3
     for b, (ro, rl) in want.items():
-        assert np.abs(go_[b] - ro).max() <= tol, b
+        assert (np.abs(go_[b] - ro) - bf16_bound(ro, rel=0.0)).max() <= tol, b
         assert np.abs(lse.cpu().numpy()[b] - rl).max() <= 2e-2, b
 
 

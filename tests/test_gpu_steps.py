@@ -19,7 +19,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import code_values, dev, index_arrays, rel_close
+from gpu_util import bf16_bound, code_values, dev, index_arrays, rel_close
 from oracle import oracle as orc
 
 pytestmark = pytest.mark.gpu
@@ -195,6 +195,7 @@ def test_c4_compress_kv(fmt):
     assert st.item() == 0
     got = cache.cpu().numpy()
     written = np.zeros(n_slots, dtype=bool)
+    rne_mismatch, n_el = 0, 0
     for b in range(len(new)):
         xb, gb = x[cu[b]:cu[b + 1]].astype(np.float64), gate[cu[b]:cu[b + 1]].astype(np.float64)
         y = orc.c4_compress(xb, gb, bias.astype(np.float64))
@@ -205,7 +206,9 @@ def test_c4_compress_kv(fmt):
             gr = orc.kv_decode_rows(got[slot], fmt == "fp8")[0]
             blk = np.abs(xb[4 * i:4 * i + 4]).max(0)
             if fmt == "bf16":
-                assert (np.abs(gr - y[i]) <= 2e-3 * np.maximum(np.abs(y[i]), blk)).all()
+                assert (np.abs(gr - y[i]) <= bf16_bound(y[i], floor=1e-6 * blk)).all()
+                rne_mismatch += int((orc.kv_encode_rows(y[i:i + 1], False)[0] != got[slot]).sum())
+                n_el += 1152
             else:
                 s = got[slot, 512:528].copy().view(np.float32).astype(np.float64)
                 ref_row = orc.kv_encode_rows(y[i:i + 1], True)[0]
@@ -214,9 +217,12 @@ def test_c4_compress_kv(fmt):
                 lat = np.abs(gr[:512] - y[i, :512])
                 bound = 2.0 ** -3 * np.abs(y[i, :512]) + np.repeat(s, 128) * 2.0 ** -9
                 assert (lat <= bound).all()
-                assert (np.abs(gr[512:] - y[i, 512:]) <= 2e-3 * np.maximum(np.abs(y[i, 512:]),
-                                                                          blk[512:])).all()
+                assert (np.abs(gr[512:] - y[i, 512:]) <= bf16_bound(y[i, 512:],
+                                                                   floor=1e-6 * blk[512:])).all()
     assert (got[~written] == 0xCD).all()
+    # the single float32 rounding agrees with the oracle's bf16 rounding except
+    # where float32 and float64 straddle a rounding midpoint
+    assert rne_mismatch <= 1e-3 * max(n_el, 1)
 
 
 def test_c4_compress_one_hot_gate_copies_rows():
@@ -559,8 +565,10 @@ def test_sparse_mqa(kv_fmt, heads, decode):
         rows = np.concatenate([c["c4_rows"][b][c["chosen"][t]].reshape(-1, 576),
                                np.array([c["raw_rows"][b][int(r)] for r in win]).reshape(-1, 576)])
         ro, rl = orc.sparse_attention(qf[t], rows, sm_scale)
-        err = np.abs(go[t] - ro).max()
-        assert err <= tol, (t, err)
+        # outputs are bf16: the bound is the tolerance plus half a bf16 ulp of
+        # the reference (only matters for |out| > 1, as in the x3 request)
+        err = np.abs(go[t] - ro) - bf16_bound(ro, rel=0.0)
+        assert err.max() <= tol, (t, err.max())
         assert np.abs(gl[t] - rl).max() <= 2e-2, t
 
 
@@ -581,7 +589,7 @@ def test_sparse_mqa_window_only_and_zero_window():
         win = orc.window_positions(int(c["q_pos"][t]), 128)
         rows = np.array([c["raw_rows"][t][int(r)] for r in win])
         ro, _ = orc.sparse_attention(qf[t], rows, 0.05)
-        assert np.abs(go[t] - ro).max() <= 5e-3
+        assert (np.abs(go[t] - ro) - bf16_bound(ro, rel=0.0)).max() <= 5e-3
     csa.csa_sparse_mqa_decode(c["q"].cuda(), dev(c["c4_cache"]), dev(c["raw_cache"]), 0,
                               dev(c["idx"]), dev(c["pt"]), dev(c["L"].astype(np.int32)),
                               dev(c["cu_q"]), None, 0, 0.05, out, lse)
@@ -590,4 +598,4 @@ def test_sparse_mqa_window_only_and_zero_window():
     for t in range(c["nq"]):
         rows = c["c4_rows"][t][c["chosen"][t]]
         ro, _ = orc.sparse_attention(qf[t], rows, 0.05)
-        assert np.abs(go[t] - ro).max() <= 5e-3
+        assert (np.abs(go[t] - ro) - bf16_bound(ro, rel=0.0)).max() <= 5e-3
