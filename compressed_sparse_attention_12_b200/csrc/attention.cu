@@ -11,9 +11,11 @@
 // with V = the rows' 512 latent dims; lse = ln sum exp z.
 //
 // One CTA (4 warps) owns one query, 16 heads and a contiguous range of the
-// query's row list (a "split").  Rows are gathered 64 at a time into shared
-// memory as bf16: BF16 rows as stored, FP8 rows as their E4M3 codes (exact in
-// bf16) with the four per-128-channel scales kept aside in float32.
+// query's row list (a "split").  Rows are gathered 32 at a time by cp.async
+// into a two-stage ring (the next tile's rows land while the current one is
+// computed); FP8 rows are then expanded into a bf16 tile as their E4M3 codes
+// (exact in bf16) with the four per-128-channel scales kept aside in float32,
+// BF16 rows are gathered straight into their tile.
 // S = Q K^T runs on bf16 mma.sync tensor-core instructions per 128-channel
 // block, each block's partial sum scaled by its row scale in float32; the
 // online softmax is float32 (base-2 exponent); O += P V splits P (times the
@@ -26,22 +28,30 @@
 namespace csa {
 
 constexpr int kAtThreads = 128;
-constexpr int kAtRows = 64;                 // rows per tile
+constexpr int kAtRows = 32;                 // rows per tile
 constexpr int kAtHeads = 16;                // heads per CTA
 constexpr int kAtStride = kKvDim + 8;       // bf16 elements per smem row (bank-conflict pad)
-constexpr int kAtPStride = kAtRows + 8;   // floats per P row
+constexpr int kAtPStride = kAtRows + 8;     // floats per P row
+constexpr int kAtMaxTiles = (kTopK + 1024 + kAtRows - 1) / kAtRows;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kTileBytes = kAtRows * kAtStride * 2;             // one bf16 tile
+constexpr int kStageBytes = kAtRows * kFp8RowBytes;             // one FP8 staging buffer
+constexpr int kRegionBytes = 2 * kStageBytes + kTileBytes;      // >= 2 bf16 tiles
 
 struct AtSmem {
     __nv_bfloat16 q[kAtHeads * kAtStride];
-    __nv_bfloat16 kv[kAtRows * kAtStride];
+    // FP8: [staging 0 | staging 1 | tile];  BF16: [tile 0 | tile 1]
+    alignas(16) uint8_t region[kRegionBytes];
     float p[kAtHeads * kAtPStride];         // probabilities of the tile, float32
-    float rscale[kAtRows][4];               // per-row scales of the 4 latent blocks
+    float rscale[2][kAtRows][4];            // per-row scales of the 4 latent blocks
     float red_max[4][kAtHeads];
     float red_sum[4][kAtHeads];
-    int32_t slot[kAtRows];                  // >= 0: row slot; -1: masked
-    int32_t is_raw[kAtRows];
+    int32_t slot[2][kAtRows];               // >= 0: row slot; -1: masked
+    int32_t is_raw[2][kAtRows];
+    int16_t tiles[kAtMaxTiles];             // non-empty tiles of this split
+    int32_t n_tiles;
 };
+static_assert(2 * kTileBytes <= kRegionBytes, "region holds two bf16 tiles");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -69,8 +79,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src));
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -94,83 +108,100 @@ __device__ __forceinline__ AtQuery at_query(const AttnArgs &a, int t) {
     return q;
 }
 
-// Gather rows [r0, r0+64) of the query's row list into smem as bf16.
-__device__ void load_tile(const AttnArgs &a, const AtQuery &qq, int t, int r0, AtSmem &sm) {
-    const int tid = threadIdx.x;
-    const int row_bytes = a.kv_fmt == CSA_FMT_FP8 ? kFp8RowBytes : kBf16RowBytes;
-    if (tid < kAtRows) {
-        const int r = r0 + tid;
-        int32_t slot = -1, raw = 0;
-        if (r < kTopK) {
-            slot = a.idx[(int64_t)t * kTopK + r];
-            if (slot >= a.num_c4_slots) {
-                report(a.status, CSA_ERR_BOUNDS);
-                slot = -1;
-            }
-        } else if (r - kTopK < qq.nw) {
-            const int pos = qq.p - qq.nw + 1 + (r - kTopK);
-            const int32_t page = pos / kPage < a.pt_stride
-                                     ? a.page_table[(int64_t)qq.b * a.pt_stride + pos / kPage]
-                                     : -1;
-            const int64_t s = (int64_t)page * kPage + pos % kPage;
-            if (page < 0 || s >= a.num_raw_slots) {
-                report(a.status, CSA_ERR_BOUNDS);
-            } else {
-                slot = (int32_t)s;
-                raw = 1;
-            }
+// Slot of entry r of the query's row list (-1: masked).  Entries 0..511 are
+// the selected compressed rows, then the window's raw positions in order.
+__device__ __forceinline__ int32_t row_slot(const AttnArgs &a, const AtQuery &qq, int t, int r,
+                                            int32_t *raw) {
+    *raw = 0;
+    if (r < kTopK) {
+        int32_t slot = a.idx[(int64_t)t * kTopK + r];
+        if (slot >= a.num_c4_slots) {
+            report(a.status, CSA_ERR_BOUNDS);
+            slot = -1;
         }
-        sm.slot[tid] = slot;
-        sm.is_raw[tid] = raw;
+        return slot < 0 ? -1 : slot;
     }
-    __syncthreads();
+    if (r - kTopK >= qq.nw) return -1;
+    const int pos = qq.p - qq.nw + 1 + (r - kTopK);
+    const int32_t page = pos / kPage < a.pt_stride
+                             ? a.page_table[(int64_t)qq.b * a.pt_stride + pos / kPage]
+                             : -1;
+    const int64_t s = (int64_t)page * kPage + pos % kPage;
+    if (page < 0 || s >= a.num_raw_slots) {
+        report(a.status, CSA_ERR_BOUNDS);
+        return -1;
+    }
+    *raw = 1;
+    return (int32_t)s;
+}
+
+// Fills the slot table of stage `st` for tile `tile` (threads 0..31).
+__device__ __forceinline__ void fill_slots(const AttnArgs &a, const AtQuery &qq, int t, int tile,
+                                           int st, AtSmem &sm) {
+    if (threadIdx.x < kAtRows) {
+        int32_t raw;
+        const int32_t slot = row_slot(a, qq, t, tile * kAtRows + threadIdx.x, &raw);
+        sm.slot[st][threadIdx.x] = slot;
+        sm.is_raw[st][threadIdx.x] = raw;
+    }
+}
+
+__device__ __forceinline__ __nv_bfloat16 *tile_ptr(int fmt, int st, AtSmem &sm) {
+    return reinterpret_cast<__nv_bfloat16 *>(
+        sm.region + (fmt == CSA_FMT_FP8 ? 2 * kStageBytes : st * kTileBytes));
+}
+
+// Issues the cp.async gathers of stage `st` (slots already filled and visible).
+__device__ __forceinline__ void issue_loads(const AttnArgs &a, int st, AtSmem &sm) {
     const uint8_t *c4 = reinterpret_cast<const uint8_t *>(a.c4_cache);
     const uint8_t *rc = reinterpret_cast<const uint8_t *>(a.raw_cache);
     if (a.kv_fmt == CSA_FMT_BF16) {
-        if (tid < kAtRows) {
-            const float one = sm.slot[tid] >= 0 ? 1.0f : 0.0f;
-            sm.rscale[tid][0] = sm.rscale[tid][1] = sm.rscale[tid][2] = sm.rscale[tid][3] = one;
-        }
-        // 72 chunks of 16 B per row
-        for (int u = tid; u < kAtRows * 72; u += kAtThreads) {
+        __nv_bfloat16 *tile = tile_ptr(CSA_FMT_BF16, st, sm);
+        for (int u = threadIdx.x; u < kAtRows * 72; u += kAtThreads) {
             const int r = u / 72, c = u % 72;
-            __nv_bfloat16 *dst = sm.kv + r * kAtStride + c * 8;
-            const int32_t slot = sm.slot[r];
-            if (slot < 0) {
+            __nv_bfloat16 *dst = tile + r * kAtStride + c * 8;
+            const int32_t slot = sm.slot[st][r];
+            if (slot < 0)
                 *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-            } else {
-                const uint8_t *src = (sm.is_raw[r] ? rc : c4) + (int64_t)slot * row_bytes + c * 16;
-                cp_async16(dst, src);
-            }
+            else
+                cp_async16(dst, (sm.is_raw[st][r] ? rc : c4) + (int64_t)slot * kBf16RowBytes + c * 16);
         }
-        cp_async_wait_all();
     } else {
-        if (tid < kAtRows) {
-            const int32_t slot = sm.slot[tid];
-            float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
+        uint8_t *stage = sm.region + st * kStageBytes;
+        for (int u = threadIdx.x; u < kAtRows * 41; u += kAtThreads) {
+            const int r = u / 41, c = u % 41;
+            const int32_t slot = sm.slot[st][r];
             if (slot >= 0)
-                sc = *reinterpret_cast<const float4 *>((sm.is_raw[tid] ? rc : c4) +
-                                                       (int64_t)slot * row_bytes + 512);
-            sm.rscale[tid][0] = sc.x;
-            sm.rscale[tid][1] = sc.y;
-            sm.rscale[tid][2] = sc.z;
-            sm.rscale[tid][3] = sc.w;
+                cp_async16(stage + r * kFp8RowBytes + c * 16,
+                           (sm.is_raw[st][r] ? rc : c4) + (int64_t)slot * kFp8RowBytes + c * 16);
         }
-        // 32 code chunks (16 E4M3 codes -> 16 exact bf16) + 8 RoPE chunks per row
-        for (int u = tid; u < kAtRows * 40; u += kAtThreads) {
-            const int r = u / 40, c = u % 40;
-            const int32_t slot = sm.slot[r];
-            __nv_bfloat16 *dst = sm.kv + r * kAtStride + (c < 32 ? c * 16 : 512 + (c - 32) * 8);
-            if (slot < 0) {
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-                if (c < 32) *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(0, 0, 0, 0);
-                continue;
-            }
-            const uint8_t *row = (sm.is_raw[r] ? rc : c4) + (int64_t)slot * row_bytes;
-            if (c < 32) {
+    }
+    cp_async_commit();
+}
+
+// FP8: expands staging `st` into the bf16 tile (exact codes) and the row scales.
+__device__ __forceinline__ void expand_fp8(int st, AtSmem &sm) {
+    const uint8_t *stage = sm.region + st * kStageBytes;
+    __nv_bfloat16 *tile = tile_ptr(CSA_FMT_FP8, st, sm);
+    if (threadIdx.x < kAtRows) {
+        const int r = threadIdx.x;
+        float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (sm.slot[st][r] >= 0) sc = *reinterpret_cast<const float4 *>(stage + r * kFp8RowBytes + 512);
+        sm.rscale[st][r][0] = sc.x;
+        sm.rscale[st][r][1] = sc.y;
+        sm.rscale[st][r][2] = sc.z;
+        sm.rscale[st][r][3] = sc.w;
+    }
+    for (int u = threadIdx.x; u < kAtRows * 40; u += kAtThreads) {
+        const int r = u / 40, c = u % 40;
+        __nv_bfloat16 *dst = tile + r * kAtStride + (c < 32 ? c * 16 : 512 + (c - 32) * 8);
+        const uint8_t *row = stage + r * kFp8RowBytes;
+        const bool valid = sm.slot[st][r] >= 0;
+        if (c < 32) {
+            uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (valid) {
                 const uint4 u4 = *reinterpret_cast<const uint4 *>(row + c * 16);
                 const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
-                uint32_t o[8];
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     const float2 lo = e4m3x2_to_f32x2((uint16_t)(w[j] & 0xFFFF));
@@ -178,15 +209,15 @@ __device__ void load_tile(const AttnArgs &a, const AtQuery &qq, int t, int r0, A
                     o[2 * j] = pack_bf16(lo.x, lo.y);
                     o[2 * j + 1] = pack_bf16(hi.x, hi.y);
                 }
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
-            } else {
-                *reinterpret_cast<uint4 *>(dst) =
-                    *reinterpret_cast<const uint4 *>(row + 528 + (c - 32) * 16);
             }
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+        } else {
+            *reinterpret_cast<uint4 *>(dst) =
+                valid ? *reinterpret_cast<const uint4 *>(row + 528 + (c - 32) * 16)
+                      : make_uint4(0, 0, 0, 0);
         }
     }
-    __syncthreads();
 }
 
 // One CTA: query t, head group g (16 heads), split sp over the row list.
@@ -198,12 +229,32 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
     const int t = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
+    const bool fp8 = a.kv_fmt == CSA_FMT_FP8;
     const AtQuery qq = at_query(a, t);
     const int n_rows = kTopK + qq.nw;
     const int tile0 = sp * tiles_per_split;
     const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
 
-    // Q: heads 16g..16g+15 of query t
+    // non-empty tiles of this split (compressed tiles whose entries are all -1 are skipped)
+    if (tid == 0) sm.n_tiles = 0;
+    __syncthreads();
+    for (int tile = tile0 + warp; tile < tile1; tile += 4) {
+        const int r = tile * kAtRows + lane;
+        bool any = r >= kTopK ? (r - kTopK) < qq.nw : a.idx[(int64_t)t * kTopK + r] >= 0;
+        any = __any_sync(0xffffffffu, any);
+        if (lane == 0) sm.tiles[tile - tile0] = any ? 1 : 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int n = 0;
+        for (int tile = tile0; tile < tile1; tile++)
+            if (sm.tiles[tile - tile0]) sm.tiles[n++] = (int16_t)tile;
+        sm.n_tiles = n;
+    }
+    __syncthreads();
+    const int nt = sm.n_tiles;
+
+    // prologue: Q (heads 16g..16g+15) and the first two tiles
     {
         const __nv_bfloat16 *qsrc = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                                     ((int64_t)t * a.heads + g * kAtHeads) * kKvDim;
@@ -211,7 +262,14 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             const int h = u / 72, c = u % 72;
             cp_async16(sm.q + h * kAtStride + c * 8, qsrc + h * kKvDim + c * 8);
         }
-        cp_async_wait_all();
+    }
+    for (int j = 0; j < 2; j++) {
+        if (j < nt) fill_slots(a, qq, t, sm.tiles[j], j, sm);
+    }
+    __syncthreads();
+    for (int j = 0; j < 2; j++) {
+        if (j < nt) issue_loads(a, j, sm);
+        else cp_async_commit();
     }
 
     const float scale2 = a.sm_scale * kLog2e;
@@ -219,63 +277,57 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
 #pragma unroll
     for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    const uint32_t q_base = smem_u32(sm.q) +
+                            (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
+                                       (lane >> 4) * 8) * 2;
 
-    for (int tile = tile0; tile < tile1; tile++) {
-        const int r0 = tile * kAtRows;
-        // skip tiles whose compressed entries are all padding
-        if (r0 + kAtRows <= kTopK) {
-            const int32_t v = a.idx[(int64_t)t * kTopK + r0 + (tid & 63)];
-            if (__syncthreads_or(v >= 0) == 0) continue;
+    for (int j = 0; j < nt; j++) {
+        const int st = j & 1;
+        if (j + 1 < nt) cp_async_wait<1>(); else cp_async_wait<0>();
+        __syncthreads();
+        if (fp8) {
+            expand_fp8(st, sm);
+        } else if (tid < kAtRows) {
+            const float one = sm.slot[st][tid] >= 0 ? 1.0f : 0.0f;
+            sm.rscale[st][tid][0] = sm.rscale[st][tid][1] = one;
+            sm.rscale[st][tid][2] = sm.rscale[st][tid][3] = one;
         }
-        load_tile(a, qq, t, r0, sm);
+        __syncthreads();
+        const __nv_bfloat16 *tile = tile_ptr(a.kv_fmt, st, sm);
 
-        // S = Q K^T: warp w covers rows 16w..16w+15 (two n-tiles of 8).  Each
-        // 128-channel latent block accumulates separately and is folded in
-        // with its row scale; the RoPE block has scale 1.
-        float s[2][4];
-#pragma unroll
-        for (int i = 0; i < 2; i++) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.0f;
-        const uint32_t q_base = smem_u32(sm.q) +
-                                (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
-                                           (lane >> 4) * 8) * 2;
-        const uint32_t k_base = smem_u32(sm.kv) +
-                                (uint32_t)((warp * 16 + (lane & 7) + (lane >> 4) * 8) * kAtStride +
-                                           ((lane >> 3) & 1) * 8) * 2;
+        // S = Q K^T: warp w covers rows 8w..8w+7.  Each 128-channel latent block
+        // accumulates separately and is folded in with its row scale.
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t k_base = smem_u32(tile) +
+                                (uint32_t)((warp * 8 + (lane & 7)) * kAtStride + (lane >> 3) * 8) * 2;
 #pragma unroll 1
         for (int blk = 0; blk < 5; blk++) {
-            float acc[2][4];
-#pragma unroll
-            for (int i = 0; i < 2; i++) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
             const int k0 = blk * 8, nk = blk < 4 ? 8 : 4;
-#pragma unroll 4
-            for (int kk = k0; kk < k0 + nk; kk++) {
-                uint32_t af[4], bf[4];
-                ldsm_x4(af, q_base + kk * 32);
+#pragma unroll 2
+            for (int kk = k0; kk < k0 + nk; kk += 2) {
+                uint32_t a0[4], a1[4], bf[4];
+                ldsm_x4(a0, q_base + kk * 32);
+                ldsm_x4(a1, q_base + (kk + 1) * 32);
                 ldsm_x4(bf, k_base + kk * 32);
-                mma16816(acc[0], af, bf[0], bf[1]);
-                mma16816(acc[1], af, bf[2], bf[3]);
+                mma16816(acc, a0, bf[0], bf[1]);
+                mma16816(acc, a1, bf[2], bf[3]);
             }
 #pragma unroll
-            for (int nt = 0; nt < 2; nt++) {
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const int row = warp * 16 + nt * 8 + 2 * tq + (j & 1);
-                    const float sc = blk < 4 ? sm.rscale[row][blk] : 1.0f;
-                    s[nt][j] = fmaf(acc[nt][j], sc, s[nt][j]);
-                }
+            for (int jj = 0; jj < 4; jj++) {
+                const int row = warp * 8 + 2 * tq + (jj & 1);
+                const float sc = blk < 4 ? sm.rscale[st][row][blk] : 1.0f;
+                s[jj] = fmaf(acc[jj], sc, s[jj]);
             }
         }
         // scale, mask, per-head tile max
         float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int nt = 0; nt < 2; nt++) {
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int row = warp * 16 + nt * 8 + 2 * tq + (j & 1);
-                const float v = sm.slot[row] >= 0 ? s[nt][j] * scale2 : -INFINITY;
-                s[nt][j] = v;
-                tmax[j >> 1] = fmaxf(tmax[j >> 1], v);
-            }
+        for (int jj = 0; jj < 4; jj++) {
+            const int row = warp * 8 + 2 * tq + (jj & 1);
+            const float v = sm.slot[st][row] >= 0 ? s[jj] * scale2 : -INFINITY;
+            s[jj] = v;
+            tmax[jj >> 1] = fmaxf(tmax[jj >> 1], v);
         }
 #pragma unroll
         for (int h = 0; h < 2; h++) {
@@ -291,25 +343,23 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             const int hh = gq + 8 * h;
-            float mx = fmaxf(fmaxf(sm.red_max[0][hh], sm.red_max[1][hh]),
-                             fmaxf(sm.red_max[2][hh], sm.red_max[3][hh]));
+            const float mx = fmaxf(fmaxf(sm.red_max[0][hh], sm.red_max[1][hh]),
+                                   fmaxf(sm.red_max[2][hh], sm.red_max[3][hh]));
             m_new[h] = fmaxf(m_run[h], mx);
             alpha[h] = m_new[h] == -INFINITY ? 1.0f : exp2f(m_run[h] - m_new[h]);
         }
         float psum[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int nt = 0; nt < 2; nt++) {
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int h = j >> 1;
-                const float pv = m_new[h] == -INFINITY ? 0.0f : exp2f(s[nt][j] - m_new[h]);
-                s[nt][j] = pv;
-                psum[h] += pv;
-            }
-            const int col = warp * 16 + nt * 8 + 2 * tq;
-            *reinterpret_cast<float2 *>(sm.p + gq * kAtPStride + col) = make_float2(s[nt][0], s[nt][1]);
-            *reinterpret_cast<float2 *>(sm.p + (gq + 8) * kAtPStride + col) =
-                make_float2(s[nt][2], s[nt][3]);
+        for (int jj = 0; jj < 4; jj++) {
+            const int h = jj >> 1;
+            const float pv = m_new[h] == -INFINITY ? 0.0f : exp2f(s[jj] - m_new[h]);
+            s[jj] = pv;
+            psum[h] += pv;
+        }
+        {
+            const int col = warp * 8 + 2 * tq;
+            *reinterpret_cast<float2 *>(sm.p + gq * kAtPStride + col) = make_float2(s[0], s[1]);
+            *reinterpret_cast<float2 *>(sm.p + (gq + 8) * kAtPStride + col) = make_float2(s[2], s[3]);
         }
 #pragma unroll
         for (int h = 0; h < 2; h++) {
@@ -338,8 +388,7 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
         }
         // O[:, 128w:128w+128] += (P * rowscale_w) V, P split into bf16 hi + lo
         // (this warp's output columns are exactly latent block w).
-        __syncthreads();
-        const uint32_t v_base = smem_u32(sm.kv) +
+        const uint32_t v_base = smem_u32(tile) +
                                 (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
                                            warp * 128 + (lane >> 4) * 8) * 2;
 #pragma unroll
@@ -350,8 +399,8 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             const float2 p10 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k);
             const float2 p01 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k + 8);
             const float2 p11 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k + 8);
-            const float c0 = sm.rscale[r0k][warp], c1 = sm.rscale[r0k + 1][warp];
-            const float c8 = sm.rscale[r0k + 8][warp], c9 = sm.rscale[r0k + 9][warp];
+            const float c0 = sm.rscale[st][r0k][warp], c1 = sm.rscale[st][r0k + 1][warp];
+            const float c8 = sm.rscale[st][r0k + 8][warp], c9 = sm.rscale[st][r0k + 9][warp];
             pv[0] = p00.x * c0; pv[1] = p00.y * c1;     // a0: head g,   rows r, r+1
             pv[2] = p10.x * c0; pv[3] = p10.y * c1;     // a1: head g+8, rows r, r+1
             pv[4] = p01.x * c8; pv[5] = p01.y * c9;     // a2: head g,   rows r+8, r+9
@@ -374,7 +423,14 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
                 mma16816(o[2 * np + 1], al, bf[2], bf[3]);
             }
         }
-        __syncthreads();   // smem tile reused by the next load
+        __syncthreads();   // stage `st` and the tile are free again
+        if (j + 2 < nt) {
+            fill_slots(a, qq, t, sm.tiles[j + 2], st, sm);
+            __syncthreads();
+            issue_loads(a, st, sm);
+        } else {
+            cp_async_commit();
+        }
     }
 
     const int h0 = g * kAtHeads;
@@ -386,10 +442,10 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +
                                   ((int64_t)t * a.heads + h0 + hh) * kLatent;
 #pragma unroll
-            for (int nt = 0; nt < 16; nt++) {
-                const int col = warp * 128 + nt * 8 + 2 * tq;
+            for (int n8 = 0; n8 < 16; n8++) {
+                const int col = warp * 128 + n8 * 8 + 2 * tq;
                 *reinterpret_cast<uint32_t *>(orow + col) =
-                    pack_bf16(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
+                    pack_bf16(o[n8][2 * h] * inv, o[n8][2 * h + 1] * inv);
             }
             if (a.lse && warp == 0 && tq == 0)
                 a.lse[(int64_t)t * a.heads + h0 + hh] =
@@ -403,9 +459,9 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             const int hh = gq + 8 * h;
             float *prow = part_o + (pbase + hh) * kLatent;
 #pragma unroll
-            for (int nt = 0; nt < 16; nt++) {
-                const int col = warp * 128 + nt * 8 + 2 * tq;
-                *reinterpret_cast<float2 *>(prow + col) = make_float2(o[nt][2 * h], o[nt][2 * h + 1]);
+            for (int n8 = 0; n8 < 16; n8++) {
+                const int col = warp * 128 + n8 * 8 + 2 * tq;
+                *reinterpret_cast<float2 *>(prow + col) = make_float2(o[n8][2 * h], o[n8][2 * h + 1]);
             }
             if (warp == 0 && tq == 0) {
                 part_ml[(pbase + hh) * 2] = m_run[h];
@@ -415,40 +471,45 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
     }
 }
 
-// Merge the splits of one (query, head group): grid (num_q, groups), 256 threads.
-__global__ void __launch_bounds__(256)
+// Merge the splits of one (query, head): grid num_q * heads, 128 threads,
+// four output columns per thread.
+__global__ void __launch_bounds__(128)
 sparse_mqa_combine_kernel(const AttnArgs a, int splits, const float *part_o,
                           const float *part_ml) {
-    const int t = blockIdx.x, g = blockIdx.y;
-    const int64_t base = ((int64_t)t * gridDim.y + g) * splits;
-    for (int u = threadIdx.x; u < kAtHeads * (kLatent / 2); u += blockDim.x) {
-        const int hh = u / (kLatent / 2), c = (u % (kLatent / 2)) * 2;
-        float M = -INFINITY;
+    const int t = blockIdx.x / a.heads, head = blockIdx.x % a.heads;
+    const int g = head / kAtHeads, hh = head % kAtHeads;
+    const int groups = a.heads / kAtHeads;
+    const int64_t base = ((int64_t)t * groups + g) * splits;
+    float M = -INFINITY;
+    for (int sp = 0; sp < splits; sp++) {
+        const int64_t r = (base + sp) * kAtHeads + hh;
+        if (part_ml[r * 2 + 1] > 0.0f) M = fmaxf(M, part_ml[r * 2]);
+    }
+    float L = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int c = threadIdx.x * 4;
+    if (M != -INFINITY) {
         for (int sp = 0; sp < splits; sp++) {
             const int64_t r = (base + sp) * kAtHeads + hh;
-            if (part_ml[r * 2 + 1] > 0.0f) M = fmaxf(M, part_ml[r * 2]);
+            const float l = part_ml[r * 2 + 1];
+            if (!(l > 0.0f)) continue;
+            const float w = exp2f(part_ml[r * 2] - M);
+            L += l * w;
+            const float4 v = *reinterpret_cast<const float4 *>(part_o + r * kLatent + c);
+            acc.x += v.x * w;
+            acc.y += v.y * w;
+            acc.z += v.z * w;
+            acc.w += v.w * w;
         }
-        float L = 0.0f, o0 = 0.0f, o1 = 0.0f;
-        if (M != -INFINITY) {
-            for (int sp = 0; sp < splits; sp++) {
-                const int64_t r = (base + sp) * kAtHeads + hh;
-                const float l = part_ml[r * 2 + 1];
-                if (!(l > 0.0f)) continue;
-                const float w = exp2f(part_ml[r * 2] - M);
-                L += l * w;
-                const float2 v = *reinterpret_cast<const float2 *>(part_o + r * kLatent + c);
-                o0 += v.x * w;
-                o1 += v.y * w;
-            }
-        }
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +
-                              ((int64_t)t * a.heads + g * kAtHeads + hh) * kLatent;
-        *reinterpret_cast<uint32_t *>(orow + c) = pack_bf16(o0 * inv, o1 * inv);
-        if (a.lse && c == 0)
-            a.lse[(int64_t)t * a.heads + g * kAtHeads + hh] =
-                L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +
+                          ((int64_t)t * a.heads + head) * kLatent;
+    *reinterpret_cast<uint2 *>(orow + c) =
+        make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+    if (a.lse && threadIdx.x == 0)
+        a.lse[(int64_t)t * a.heads + head] =
+            L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
 static int at_tiles(int window) { return (kTopK + window + kAtRows - 1) / kAtRows; }
@@ -459,7 +520,7 @@ static int at_splits(int num_q, int heads, int window, bool decode) {
     int sp = (2 * 148 * 2 + ctas - 1) / ctas;
     sp = sp < 1 ? 1 : sp;
     const int nt = at_tiles(window);
-    sp = sp > 4 ? 4 : sp;
+    sp = sp > 5 ? 5 : sp;
     return sp > nt ? nt : sp;
 }
 
@@ -488,7 +549,7 @@ cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s) {
     sparse_mqa_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
     e = cudaGetLastError();
     if (e != cudaSuccess || sp == 1) return e;
-    sparse_mqa_combine_kernel<<<dim3(a.num_q, groups), 256, 0, s>>>(a, sp, po, pml);
+    sparse_mqa_combine_kernel<<<a.num_q * a.heads, 128, 0, s>>>(a, sp, po, pml);
     return cudaGetLastError();
 }
 

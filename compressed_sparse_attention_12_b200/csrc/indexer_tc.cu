@@ -17,8 +17,12 @@
 //           accumulator to the epilogue,
 //   warps 2-5 epilogue: tcgen05.ld of the key's row, ReLU, head-weighted sum
 //           per query, times the key's scale, one coalesced float store.
-// Formats: FP8 E4M3 (kind::f8f6f4) and bf16 (kind::f16).  All waits are
-// bounded; a timeout records CSA_ERR_TIMEOUT and the CTA unwinds.
+// Formats: FP8 E4M3 (kind::f8f6f4), bf16 (kind::f16), and FP4 E2M1 with
+// unsigned-E4M3 block-16 scales (kind::mxf4nvf4 block-scaled): warp 0's other
+// lanes gather each tile's key block scales into the 128-row scale-factor
+// layout in shared memory, the MMA thread moves them into TMEM with
+// tcgen05.cp, and the query's block scales are placed in TMEM once.  All
+// waits are bounded; a timeout records CSA_ERR_TIMEOUT and the CTA unwinds.
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
@@ -55,15 +59,19 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     // 1024-byte aligned carve-up: stages | q tile | w' | nv | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    constexpr bool kFp4 = FMT == CSA_FMT_FP4;
     uint8_t *stage_buf = base;
     uint8_t *q_buf = stage_buf + p.stages * G::kStageBytes;
-    float *w_s = reinterpret_cast<float *>(q_buf + ((p.n * RB + 1023) & ~1023));
+    uint8_t *sfa_buf = q_buf + ((p.n * RB + 1023) & ~1023);            // [stages][ksteps][512]
+    uint8_t *sfb_buf = sfa_buf + (kFp4 ? p.stages * G::kKSteps * 512 : 0);  // [ksteps][512]
+    float *w_s = reinterpret_cast<float *>(sfb_buf + (kFp4 ? G::kKSteps * 512 : 0));
     int *nv_s = reinterpret_cast<int *>(w_s + 256);
     uint64_t *bars = reinterpret_cast<uint64_t *>(nv_s + 16);
     uint64_t *full = bars, *empty = bars + p.stages, *tfull = bars + 2 * p.stages;
     uint64_t *tempty = tfull + 2, *drain = tempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *pg_s = const_cast<int *>(abort_flag) + 4;     // page ids of this CTA's tiles (-1: none)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -107,7 +115,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     if (warp == 0) tc::tmem_alloc(tc::saddr(tmem_slot), (uint32_t)p.tmem_cols);
     if (threadIdx.x == 32) {
         for (int s = 0; s < p.stages; s++) {
-            tc::mbar_init(tc::saddr(&full[s]), 1);
+            // FP4: the TMA transaction and the block-scale gather both arrive
+            tc::mbar_init(tc::saddr(&full[s]), kFp4 ? 2 : 1);
             tc::mbar_init(tc::saddr(&empty[s]), 1);
         }
         for (int i = 0; i < 2; i++) {
@@ -119,6 +128,12 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         tc::fence_mbar_init();
     }
     if (threadIdx.x < 4) nv_s[threadIdx.x] = nv_q[threadIdx.x];
+    for (int u = threadIdx.x; u < 2 * my_tiles; u += kTcThreads) {
+        const int pidx = tile_begin * 2 + u;
+        int page = -1;
+        if (pidx * kC4Page < nv_max && pidx < a.pt_stride) page = pt_row[pidx];
+        pg_s[u] = page;
+    }
     // query tile: row n = qi*hi_pad + h (K-major, swizzled like the key tiles)
     {
         const uint8_t *qc = reinterpret_cast<const uint8_t *>(a.q_codes);
@@ -138,6 +153,20 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             const int qi = n / p.hi_pad, h = n % p.hi_pad;
             w_s[n] = (qi < nq && h < a.heads) ? a.q_weights[(int64_t)(t0 + qi) * a.heads + h] : 0.f;
         }
+        if constexpr (kFp4) {
+            // scale-factor layout of 128 rows: row n = m0 + 32*m1 keeps its four
+            // block scales of K-step ks at byte ks*512 + m0*16 + m1*4
+            constexpr int nsf = RB / 4;      // block scales per row (Di/16)
+            for (int u = threadIdx.x; u < 128 * G::kKSteps; u += kTcThreads) {
+                const int n = u % 128, ks = u / 128;
+                const int qi = n / p.hi_pad, h = n % p.hi_pad;
+                uint32_t wv = 0;
+                if (n < p.n && qi < nq && h < a.heads)
+                    wv = *reinterpret_cast<const uint32_t *>(
+                        a.q_block_scales + ((int64_t)(t0 + qi) * a.heads + h) * nsf + ks * 4);
+                *reinterpret_cast<uint32_t *>(sfb_buf + ks * 512 + (n & 31) * 16 + (n >> 5) * 4) = wv;
+            }
+        }
     }
     tc::fence_proxy_async();
     tc::fence_before_sync();
@@ -146,24 +175,27 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- TMA producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < my_tiles; i++) {
-                const int s = i % p.stages;
-                const uint32_t ph = (uint32_t)((i / p.stages) & 1);
-                if (!tc::mbar_wait(tc::saddr(&empty[s]), ph ^ 1u, abort_flag)) {
+        // ---------------- TMA producer (lane 0) and FP4 block-scale gather (all lanes)
+        int issued = 0;
+        for (int i = 0; i < my_tiles; i++) {
+            const int s = i % p.stages;
+            const uint32_t ph = (uint32_t)((i / p.stages) & 1);
+            int ok = 1;
+            if (lane == 0) {
+                ok = tc::mbar_wait(tc::saddr(&empty[s]), ph ^ 1u, abort_flag) ? 1 : 0;
+                if (!ok) {
                     if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
                     *abort_flag = 1;
-                    break;
                 }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            const int tile = tile_begin + i;
+            if (lane == 0) {
                 tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
-                const int tile = tile_begin + i;
 #pragma unroll
                 for (int half = 0; half < 2; half++) {
-                    const int pidx = tile * 2 + half;
-                    int page = 0;
-                    if (pidx * kC4Page < nv_max && pidx < a.pt_stride) page = pt_row[pidx];
+                    int page = pg_s[i * 2 + half];
                     if (page < 0 || page >= p.num_pages) page = 0;   // epilogue reports visible keys
 #pragma unroll
                     for (int c = 0; c < G::kChunks; c++)
@@ -172,17 +204,56 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                                         &kmap, c * G::kSpan, page * kC4Page,
                                         tc::saddr(&full[s]));
                 }
-                issued++;
             }
-            // before leaving, every load issued must have landed
+            if constexpr (kFp4) {
+                // key m = lane + 32*m1 of the tile; its block scales for K-step ks
+                constexpr int nsf = RB / 4;
+                uint32_t wv[G::kKSteps][4];
+#pragma unroll
+                for (int m1 = 0; m1 < 4; m1++) {
+                    const int m = lane + 32 * m1;
+                    const int sk = tile * kTcTile + m;
+                    int64_t slot = -1;
+                    if (sk < nv_max) {
+                        const int32_t page = pg_s[i * 2 + (m >> 6)];
+                        if (page >= 0 && page < p.num_pages) slot = (int64_t)page * kC4Page + (m & 63);
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < G::kKSteps; ks++)
+                        wv[ks][m1] = slot >= 0 ? *reinterpret_cast<const uint32_t *>(
+                                                     a.k_block_scales + slot * nsf + ks * 4)
+                                               : 0u;
+                }
+#pragma unroll
+                for (int ks = 0; ks < G::kKSteps; ks++)
+                    *reinterpret_cast<uint4 *>(sfa_buf + (s * G::kKSteps + ks) * 512 + lane * 16) =
+                        make_uint4(wv[ks][0], wv[ks][1], wv[ks][2], wv[ks][3]);
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(tc::saddr(&full[s]));
+            }
+            issued++;
+        }
+        // before leaving, every load issued must have landed
+        if (lane == 0)
             for (int i = max(0, issued - p.stages); i < issued; i++)
                 tc::mbar_wait(tc::saddr(&full[i % p.stages]), (uint32_t)((i / p.stages) & 1), nullptr);
-        }
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = FMT == CSA_FMT_FP8 ? tc::idesc_m128(0, 0, p.n)
-                                                      : tc::idesc_m128(1, 1, p.n);
+            const uint32_t idesc = FMT == CSA_FMT_FP8  ? tc::idesc_m128(0, 0, p.n)
+                                   : FMT == CSA_FMT_BF16 ? tc::idesc_m128(1, 1, p.n)
+                                                         : tc::idesc_mxf4_m128(p.n);
+            // TMEM columns: [0, 2n) accumulators, then two sets of key block
+            // scales (4 columns per K-step), then the query block scales
+            const uint32_t sfa_col = (uint32_t)(2 * p.n);
+            const uint32_t sfb_col = sfa_col + 8u * G::kKSteps;
+            if constexpr (kFp4) {
+#pragma unroll
+                for (int ks = 0; ks < G::kKSteps; ks++)
+                    tc::tmem_cp_32x128b_x4(tmem_base + sfb_col + 4 * ks,
+                                           tc::rows16_desc(tc::saddr(sfb_buf + ks * 512)));
+            }
             for (int i = 0; i < my_tiles; i++) {
                 const int s = i % p.stages;
                 const int acc = i & 1;
@@ -197,13 +268,23 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 const uint32_t d = tmem_base + (uint32_t)(acc * p.n);
                 const uint32_t sa = tc::saddr(stage_buf + s * G::kStageBytes);
                 const uint32_t sb = tc::saddr(q_buf);
+                const uint32_t sfa = tmem_base + sfa_col + (uint32_t)(acc * 4 * G::kKSteps);
+                if constexpr (kFp4) {
+#pragma unroll
+                    for (int ks = 0; ks < G::kKSteps; ks++)
+                        tc::tmem_cp_32x128b_x4(
+                            sfa + 4 * ks,
+                            tc::rows16_desc(tc::saddr(sfa_buf + (s * G::kKSteps + ks) * 512)));
+                }
 #pragma unroll
                 for (int k = 0; k < G::kKSteps; k++) {
                     const int c = (k * 32) / G::kSpan, off = (k * 32) % G::kSpan;
                     const uint64_t ad = tc::kmajor_desc(sa + c * kTcTile * G::kSpan + off, G::kSpan);
                     const uint64_t bd = tc::kmajor_desc(sb + c * p.n * G::kSpan + off, G::kSpan);
-                    if (FMT == CSA_FMT_FP8) tc::mma_f8f6f4(d, ad, bd, idesc, k > 0);
-                    else tc::mma_f16(d, ad, bd, idesc, k > 0);
+                    if constexpr (FMT == CSA_FMT_FP8) tc::mma_f8f6f4(d, ad, bd, idesc, k > 0);
+                    else if constexpr (FMT == CSA_FMT_BF16) tc::mma_f16(d, ad, bd, idesc, k > 0);
+                    else tc::mma_mxf4nvf4(d, ad, bd, idesc, sfa + 4 * k, tmem_base + sfb_col + 4 * k,
+                                          k > 0);
                 }
                 tc::mma_commit(tc::saddr(&empty[s]));
                 tc::mma_commit(tc::saddr(&tfull[acc]));
@@ -218,19 +299,28 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float *lg = a.logits;
+        // key scale of this thread's row, fetched one tile ahead of its use
+        auto key_scale = [&](int i, bool &valid) -> float {
+            const int sk = (tile_begin + i) * kTcTile + row;
+            valid = false;
+            if (sk >= nv_max) return 0.0f;
+            const int32_t page = pg_s[i * 2 + (row >> 6)];
+            const int64_t slot = (int64_t)page * kC4Page + (row & 63);
+            valid = page >= 0 && page < p.num_pages && slot < a.num_slots;
+            if (!valid) {
+                report(a.status, CSA_ERR_BOUNDS);
+                return 0.0f;
+            }
+            return FMT == CSA_FMT_BF16 ? 1.0f : __ldg(a.k_scales + slot);
+        };
+        bool valid_next = false;
+        float kscale_next = key_scale(0, valid_next);
         for (int i = 0; i < my_tiles; i++) {
             const int acc = i & 1;
-            const int tile = tile_begin + i;
-            const int sk = tile * kTcTile + row;
-            float kscale = 0.0f;
-            bool valid = false;
-            if (sk < nv_max) {
-                const int32_t page = pt_row[sk / kC4Page];
-                const int64_t slot = (int64_t)page * kC4Page + sk % kC4Page;
-                valid = page >= 0 && slot < a.num_slots && page < p.num_pages;
-                if (!valid) report(a.status, CSA_ERR_BOUNDS);
-                else kscale = FMT == CSA_FMT_BF16 ? 1.0f : a.k_scales[slot];
-            }
+            const int sk = (tile_begin + i) * kTcTile + row;
+            const float kscale = kscale_next;
+            const bool valid = valid_next;
+            if (i + 1 < my_tiles) kscale_next = key_scale(i + 1, valid_next);
             if (!tc::mbar_wait(tc::saddr(&tfull[acc]), (uint32_t)((i >> 1) & 1), abort_flag)) {
                 if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
                 *abort_flag = 1;
@@ -308,20 +398,23 @@ static bool make_key_map(CUtensorMap *m, const void *codes, int64_t num_slots, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t tc_smem_bytes(int rb, const TcParams &p) {
+static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p) {
+    const size_t ks = rb / 32;
     return 1024 + (size_t)p.stages * kTcTile * rb + (((size_t)p.n * rb + 1023) & ~(size_t)1023) +
-           256 * 4 + 16 * 4 + (2 * p.stages + 5) * 8 + 16;
+           (fp4 ? (p.stages + 1) * ks * 512 : 0) + 256 * 4 + 16 * 4 + (2 * p.stages + 5) * 8 + 32 +
+           (size_t)2 * p.tiles_per_cta * 4;
 }
 
 bool indexer_tc_supported(const IndexerArgs &a) {
-    const bool fmt_ok = (a.fmt == CSA_FMT_FP8 && (a.dim == 64 || a.dim == 128)) ||
-                        (a.fmt == CSA_FMT_BF16 && (a.dim == 64 || a.dim == 128));
+    const bool fmt_ok = (a.dim == 64 || a.dim == 128) &&
+                        (a.fmt == CSA_FMT_FP8 || a.fmt == CSA_FMT_BF16);
     return fmt_ok && a.heads <= 128 && (a.num_slots % kC4Page) == 0 && a.num_slots >= kC4Page &&
            (reinterpret_cast<uintptr_t>(a.k_codes) % 16) == 0 && encode_fn() != nullptr;
 }
 
 cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
-    const int rb = a.fmt == CSA_FMT_FP8 ? a.dim : 2 * a.dim;
+    const bool fp4 = a.fmt == CSA_FMT_FP4;
+    const int rb = a.fmt == CSA_FMT_FP8 ? a.dim : fp4 ? a.dim / 2 : 2 * a.dim;
     TcParams p;
     p.hi_pad = (a.heads + 15) / 16 * 16;
     // queries of one request share the key tiles: group up to 4 of them
@@ -329,12 +422,14 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
     p.qg = a.num_q <= a.bs ? 1 : 128 / p.hi_pad;
     if (p.qg < 1) p.qg = 1;
     if (p.qg > 4) p.qg = 4;
+    if (fp4 && p.qg * p.hi_pad > 64) p.qg = p.hi_pad >= 64 ? 1 : 64 / p.hi_pad;
     p.n = p.qg * p.hi_pad;
     int cols = 32;
-    while (cols < 2 * p.n) cols <<= 1;
+    const int need = 2 * p.n + (fp4 ? 12 * (rb / 32) : 0);
+    while (cols < need) cols <<= 1;
     p.tmem_cols = cols;
     p.num_pages = (int)(a.num_slots / kC4Page);
-    p.stages = rb >= 128 ? 4 : 6;
+    p.stages = rb >= 128 ? 4 : rb == 64 ? 8 : 12;     // ~64 KB of key tiles in flight
     const int tiles_max = (a.max_c4_len + kTcTile - 1) / kTcTile;
     const int groups = (a.num_q + p.qg - 1) / p.qg;
     const int ctas_per_sm = 512 / cols < 3 ? 512 / cols : 3;
@@ -347,7 +442,7 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
 
     CUtensorMap map;
     if (!make_key_map(&map, a.k_codes, a.num_slots, rb)) return cudaErrorInvalidValue;
-    const size_t smem = tc_smem_bytes(rb, p);
+    const size_t smem = tc_smem_bytes(rb, fp4, p);
     dim3 grid(chunks, a.num_q);
 #define CSA_TC(F, R)                                                                        \
     do {                                                                                    \
@@ -358,6 +453,8 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
     } while (0)
     if (a.fmt == CSA_FMT_FP8 && rb == 128) CSA_TC(CSA_FMT_FP8, 128);
     else if (a.fmt == CSA_FMT_FP8) CSA_TC(CSA_FMT_FP8, 64);
+    else if (fp4 && rb == 64) CSA_TC(CSA_FMT_FP4, 64);
+    else if (fp4) CSA_TC(CSA_FMT_FP4, 32);
     else if (rb == 128) CSA_TC(CSA_FMT_BF16, 128);
     else CSA_TC(CSA_FMT_BF16, 256);
 #undef CSA_TC

@@ -136,6 +136,35 @@ __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint
         : "memory");
 }
 
+// Block-scaled FP4 (E2M1 x E2M1, one unsigned-E4M3 scale per 16 elements of
+// K on each side); scale factors are read from TMEM at sfa / sfb.
+__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Copies a 32-row x 128-bit block from shared memory (rows 16 bytes apart)
+// into 4 TMEM columns of lanes 0-31 of every lane quadrant.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// Descriptor of an unswizzled K-major source whose rows are 16 bytes apart
+// (8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t addr) {
+    uint64_t d = (uint64_t)((addr & 0x3FFFF) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(128 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
 // 16 consecutive 32-bit columns of this warp's 32 TMEM lanes (one per thread).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
@@ -175,6 +204,12 @@ __device__ __forceinline__ uint32_t swz(int row, int byte, int span) {
     const uint32_t o = (uint32_t)(row * span + byte);
     const uint32_t mask = (uint32_t)(span / 16 - 1);
     return o ^ (((o >> 7) & mask) << 4);
+}
+
+// Instruction descriptor of the block-scaled FP4 MMA: A, B E2M1, scales
+// unsigned E4M3, both K-major, M = 128, K = 64, scale-factor ids 0.
+__host__ __device__ constexpr uint32_t idesc_mxf4_m128(int n) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
 // Instruction descriptor: D float32, A/B formats, both K-major, M = 128.
