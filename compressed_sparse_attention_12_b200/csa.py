@@ -22,6 +22,7 @@ CSA_FMT_BF16, CSA_FMT_FP8, CSA_FMT_FP4, CSA_FMT_F32 = 0, 1, 2, 3
 CSA_OUT_KV_BF16, CSA_OUT_KV_FP8 = 0, 1
 CSA_OUT_INDEX_BF16, CSA_OUT_INDEX_FP8, CSA_OUT_INDEX_FP4 = 2, 3, 4
 TOPK, PAGE_SIZE, C4_PAGE_SIZE, KV_DIM, KV_LATENT = 512, 256, 64, 576, 512
+TOPK_NOALLOC_MAX_BYTES = 16 << 20
 
 FMT = {"bf16": CSA_FMT_BF16, "fp8": CSA_FMT_FP8, "fp4": CSA_FMT_FP4}
 
@@ -49,6 +50,9 @@ _SIGS = {
     "csa_topk512_workspace_size": (_SZ, [_I32, _I32]),
     "csa_topk512_page_transform": (ctypes.c_int, [_P, _I64, _I32, _P, _I32, _P, _P, _P, _I32,
                                                   _I64, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
+    "csa_topk512_page_transform_noalloc": (ctypes.c_int, [_P, _I64, _I32, _P, _I32, _P, _P, _P,
+                                                         _I32, _I64, _I32, _I32, _P, _P, _P,
+                                                         _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
     "csa_sparse_mqa_decode": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _P,
                                              _I32, _P, _I32, _P, _P, _I32, _F, _P, _P, _P, _SZ,
@@ -165,6 +169,18 @@ def csa_topk512_page_transform(logits, c4_seq_lens, cu_q, q_pos, page_table, num
         _ptr(q_pos), _ptr(page_table), page_table.shape[1], int(num_slots), int(c4_page_size),
         int(max_c4_len), _ptr(out_indices), _ptr(raw_indices), _ptr(workspace),
         workspace.numel(), _ptr(status), _stream(stream)))
+
+
+def csa_topk512_page_transform_noalloc(logits, c4_seq_lens, cu_q, q_pos, page_table, num_slots,
+                                       max_c4_len, out_indices, raw_indices=None,
+                                       c4_page_size=C4_PAGE_SIZE, status=None, stream=None):
+    """Top-512 page transform whose scratch is the library's own device array
+    (no workspace, no allocation); see include/csa.h."""
+    num_q = out_indices.shape[0]
+    _check("csa_topk512_page_transform_noalloc", lib().csa_topk512_page_transform_noalloc(
+        _ptr(logits), logits.shape[1], num_q, _ptr(c4_seq_lens), c4_seq_lens.shape[0], _ptr(cu_q),
+        _ptr(q_pos), _ptr(page_table), page_table.shape[1], int(num_slots), int(c4_page_size),
+        int(max_c4_len), _ptr(out_indices), _ptr(raw_indices), _ptr(status), _stream(stream)))
 
 
 def csa_sparse_mqa_workspace_size(num_q, heads, window, decode) -> int:

@@ -158,6 +158,30 @@ csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stri
     return cuda_status(csa::launch_topk512(a, as_stream(stream)));
 }
 
+csa_status_t csa_topk512_page_transform_noalloc(const float *logits, int64_t logits_stride,
+                                                int32_t num_q, const int32_t *c4_seq_lens,
+                                                int32_t bs, const int32_t *cu_q,
+                                                const int32_t *q_pos, const int32_t *page_table,
+                                                int32_t page_table_stride, int64_t num_slots,
+                                                int32_t c4_page_size, int32_t max_c4_len,
+                                                int32_t *c4_sparse_page_indices,
+                                                int32_t *raw_indices, int32_t *status,
+                                                void *stream) {
+    if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (c4_page_size != CSA_C4_PAGE_SIZE) return CSA_ERR_INVALID;
+    if (num_q == 0) return CSA_OK;
+    if (bs < 1 || !c4_seq_lens || !cu_q || !page_table || !c4_sparse_page_indices)
+        return CSA_ERR_INVALID;
+    if (max_c4_len > 0 && (!logits || logits_stride < max_c4_len)) return CSA_ERR_INVALID;
+    if (csa_topk512_workspace_size(num_q, max_c4_len) > (size_t)CSA_TOPK_NOALLOC_MAX_BYTES)
+        return CSA_ERR_WORKSPACE;
+    if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
+    csa::TopkArgs a{logits, logits_stride, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,
+                    page_table_stride, num_slots, max_c4_len, c4_sparse_page_indices,
+                    raw_indices, nullptr, status};
+    return cuda_status(csa::launch_topk512_noalloc(a, as_stream(stream)));
+}
+
 size_t csa_sparse_mqa_workspace_size(int32_t num_q, int32_t heads, int32_t window,
                                      int32_t decode) {
     if (num_q <= 0 || heads <= 0) return 0;

@@ -79,6 +79,8 @@ struct TopkArgs {
     int32_t *status;
 };
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s);
+// Same, with the scratch in the library's own device array (no workspace).
+cudaError_t launch_topk512_noalloc(const TopkArgs &a, cudaStream_t s);
 
 struct AttnArgs {
     const void *q;

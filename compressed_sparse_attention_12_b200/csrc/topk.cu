@@ -299,4 +299,31 @@ cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ no-allocation variant
+//
+// For callers that cannot provide a workspace: the candidates live in this
+// file-scope device array (held by every GPU that loads the library until the
+// process exits).  Host code may not use the array's name as a device
+// address, so its address is looked up once per device with that device
+// current and cached.  Nothing in the array needs to start at zero: stage 1
+// writes every entry stage 2 reads.  Concurrent calls share it and race.
+static __device__ __align__(256) uint8_t g_topk_scratch[CSA_TOPK_NOALLOC_MAX_BYTES];
+
+cudaError_t launch_topk512_noalloc(const TopkArgs &a, cudaStream_t s) {
+    static void *scratch_addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!scratch_addr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_topk_scratch);
+        if (e != cudaSuccess) return e;
+        scratch_addr[dev] = ptr;
+    }
+    TopkArgs b = a;
+    b.workspace = scratch_addr[dev];
+    return launch_topk512(b, s);
+}
+
 }  // namespace csa

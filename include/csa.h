@@ -227,6 +227,37 @@ csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stri
                                         size_t workspace_bytes, int32_t *status, void *stream);
 
 /*
+ * csa_topk512_page_transform_noalloc -- the same selection and page transform
+ * as csa_topk512_page_transform, for callers that cannot hand the library a
+ * workspace or call the device allocator when they make the call: plugin and
+ * operator interfaces that pass only input and output buffers, or hot paths
+ * that must never reach cudaMalloc.  The pages have no counterpart of this
+ * entry point; it exists for those callers only.
+ *
+ * Scratch lives in one file-scope device array of CSA_TOPK_NOALLOC_MAX_BYTES
+ * bytes inside libcsa.so: every GPU that loads the library holds that memory
+ * until the process exits.  The first call on a device (with that device
+ * current) looks up the array's device address once; make that first call
+ * before any stream capture.  Calls return CSA_ERR_WORKSPACE without launching
+ * when csa_topk512_workspace_size(num_q, max_c4_len) exceeds the maximum.
+ * Every call shares the one array (its contents persist between calls and
+ * nothing in it needs to start at zero), so calls that overlap on the GPU --
+ * on different streams, or from several threads -- race and must be ordered
+ * by the caller.  Never calls cudaMalloc, cudaFree or any allocating routine.
+ * Arguments are those of csa_topk512_page_transform without the workspace.
+ */
+enum { CSA_TOPK_NOALLOC_MAX_BYTES = 16 << 20 };
+csa_status_t csa_topk512_page_transform_noalloc(const float *logits, int64_t logits_stride,
+                                                int32_t num_q, const int32_t *c4_seq_lens,
+                                                int32_t bs, const int32_t *cu_q,
+                                                const int32_t *q_pos, const int32_t *page_table,
+                                                int32_t page_table_stride, int64_t num_slots,
+                                                int32_t c4_page_size, int32_t max_c4_len,
+                                                int32_t *c4_sparse_page_indices,
+                                                int32_t *raw_indices, int32_t *status,
+                                                void *stream);
+
+/*
  * csa_sparse_mqa_decode / csa_sparse_mqa_prefill -- step 4, sparse attention
  * over the selected compressed rows joined with the sliding window of raw
  * rows under ONE softmax ([T] §1; [H] "Compressed Sparse Attention（CSA）").
