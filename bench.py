@@ -40,8 +40,8 @@ UNIT = "query-tok/s"
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="decode_128k")
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -111,7 +111,7 @@ class Clocks:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -142,6 +142,27 @@ class Clocks:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def rank_workload(name, rank):
+    """Each rank times its own batch: same shapes, seed offset by the rank
+    (requests are independent, so the path shards with no data exchange)."""
+    from compressed_sparse_attention_12_b200 import synth
+    w = synth.workload(name)
+    w.seed += 1000 * rank
+    return w
+
+
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of per-rank timings (seconds) over the process group;
+    identity on one rank."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
 
 
 def cpu_baseline(w, data, pt, budget_s=20.0):
@@ -222,8 +243,7 @@ def main():
         dist.barrier()
     csa.lib()
 
-    w = synth.workload(args.workload)
-    w.seed += 1000 * rank                      # each rank its own batch
+    w = rank_workload(args.workload, rank)
     data = synth.draw(w, dev)
     batch = pipeline.CsaBatch(w, data, device=dev)
     if args.profile:
@@ -299,10 +319,7 @@ def main():
     batch.check_status()
     t_step = sum(step_ms) / len(step_ms) / 1e3
     t_idx = sum(idx_ms) / len(idx_ms) / 1e3
-    if world > 1:
-        t = torch.tensor([t_step, t_idx], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_step, t_idx = t.tolist()
+    t_step, t_idx = max_over_ranks([t_step, t_idx], world, dev)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -330,10 +347,7 @@ def main():
                 if i >= args.warmup:
                     e2e_ms.append(e0.elapsed_time(e1))
         t_e2e = sum(e2e_ms) / len(e2e_ms) / 1e3
-        if world > 1:
-            t = torch.tensor([t_e2e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            t_e2e = t.item()
+        t_e2e = max_over_ranks([t_e2e], world, dev)[0]
         e2e = {"value": world * w.num_q / t_e2e, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": t_e2e * 1e3}
 

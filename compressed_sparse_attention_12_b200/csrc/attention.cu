@@ -46,9 +46,9 @@ struct AtSmem {
     float rscale[2][kAtRows][4];            // per-row scales of the 4 latent blocks
     float red_max[4][kAtHeads];
     float red_sum[4][kAtHeads];
-    int32_t slot[2][kAtRows];               // >= 0: row slot; -1: masked
-    int32_t is_raw[2][kAtRows];
-    int16_t tiles[kAtMaxTiles];             // non-empty tiles of this split
+    int32_t slot[kAtMaxTiles * kAtRows];    // row slots of the split's tiles (-1: masked)
+    int8_t is_raw[kAtMaxTiles * kAtRows];
+    int16_t tiles[kAtMaxTiles];             // non-empty tiles of this split (local index)
     int32_t n_tiles;
 };
 static_assert(2 * kTileBytes <= kRegionBytes, "region holds two bf16 tiles");
@@ -135,58 +135,51 @@ __device__ __forceinline__ int32_t row_slot(const AttnArgs &a, const AtQuery &qq
     return (int32_t)s;
 }
 
-// Fills the slot table of stage `st` for tile `tile` (threads 0..31).
-__device__ __forceinline__ void fill_slots(const AttnArgs &a, const AtQuery &qq, int t, int tile,
-                                           int st, AtSmem &sm) {
-    if (threadIdx.x < kAtRows) {
-        int32_t raw;
-        const int32_t slot = row_slot(a, qq, t, tile * kAtRows + threadIdx.x, &raw);
-        sm.slot[st][threadIdx.x] = slot;
-        sm.is_raw[st][threadIdx.x] = raw;
-    }
-}
-
 __device__ __forceinline__ __nv_bfloat16 *tile_ptr(int fmt, int st, AtSmem &sm) {
     return reinterpret_cast<__nv_bfloat16 *>(
         sm.region + (fmt == CSA_FMT_FP8 ? 2 * kStageBytes : st * kTileBytes));
 }
 
-// Issues the cp.async gathers of stage `st` (slots already filled and visible).
-__device__ __forceinline__ void issue_loads(const AttnArgs &a, int st, AtSmem &sm) {
+// Issues the cp.async gathers of local tile `lt` into stage `st`.
+__device__ __forceinline__ void issue_loads(const AttnArgs &a, int lt, int st, AtSmem &sm) {
     const uint8_t *c4 = reinterpret_cast<const uint8_t *>(a.c4_cache);
     const uint8_t *rc = reinterpret_cast<const uint8_t *>(a.raw_cache);
+    const int32_t *slots = sm.slot + lt * kAtRows;
+    const int8_t *raws = sm.is_raw + lt * kAtRows;
     if (a.kv_fmt == CSA_FMT_BF16) {
         __nv_bfloat16 *tile = tile_ptr(CSA_FMT_BF16, st, sm);
         for (int u = threadIdx.x; u < kAtRows * 72; u += kAtThreads) {
             const int r = u / 72, c = u % 72;
             __nv_bfloat16 *dst = tile + r * kAtStride + c * 8;
-            const int32_t slot = sm.slot[st][r];
+            const int32_t slot = slots[r];
             if (slot < 0)
                 *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
             else
-                cp_async16(dst, (sm.is_raw[st][r] ? rc : c4) + (int64_t)slot * kBf16RowBytes + c * 16);
+                cp_async16(dst, (raws[r] ? rc : c4) + (int64_t)slot * kBf16RowBytes + c * 16);
         }
     } else {
         uint8_t *stage = sm.region + st * kStageBytes;
         for (int u = threadIdx.x; u < kAtRows * 41; u += kAtThreads) {
             const int r = u / 41, c = u % 41;
-            const int32_t slot = sm.slot[st][r];
+            const int32_t slot = slots[r];
             if (slot >= 0)
                 cp_async16(stage + r * kFp8RowBytes + c * 16,
-                           (sm.is_raw[st][r] ? rc : c4) + (int64_t)slot * kFp8RowBytes + c * 16);
+                           (raws[r] ? rc : c4) + (int64_t)slot * kFp8RowBytes + c * 16);
         }
     }
     cp_async_commit();
 }
 
-// FP8: expands staging `st` into the bf16 tile (exact codes) and the row scales.
-__device__ __forceinline__ void expand_fp8(int st, AtSmem &sm) {
+// FP8: expands staging `st` (local tile `lt`) into the bf16 tile (exact codes)
+// and the row scales.
+__device__ __forceinline__ void expand_fp8(int lt, int st, AtSmem &sm) {
     const uint8_t *stage = sm.region + st * kStageBytes;
     __nv_bfloat16 *tile = tile_ptr(CSA_FMT_FP8, st, sm);
+    const int32_t *slots = sm.slot + lt * kAtRows;
     if (threadIdx.x < kAtRows) {
         const int r = threadIdx.x;
         float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (sm.slot[st][r] >= 0) sc = *reinterpret_cast<const float4 *>(stage + r * kFp8RowBytes + 512);
+        if (slots[r] >= 0) sc = *reinterpret_cast<const float4 *>(stage + r * kFp8RowBytes + 512);
         sm.rscale[st][r][0] = sc.x;
         sm.rscale[st][r][1] = sc.y;
         sm.rscale[st][r][2] = sc.z;
@@ -196,7 +189,7 @@ __device__ __forceinline__ void expand_fp8(int st, AtSmem &sm) {
         const int r = u / 40, c = u % 40;
         __nv_bfloat16 *dst = tile + r * kAtStride + (c < 32 ? c * 16 : 512 + (c - 32) * 8);
         const uint8_t *row = stage + r * kFp8RowBytes;
-        const bool valid = sm.slot[st][r] >= 0;
+        const bool valid = slots[r] >= 0;
         if (c < 32) {
             uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
             if (valid) {
@@ -235,26 +228,15 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
     const int tile0 = sp * tiles_per_split;
     const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
 
-    // non-empty tiles of this split (compressed tiles whose entries are all -1 are skipped)
-    if (tid == 0) sm.n_tiles = 0;
-    __syncthreads();
-    for (int tile = tile0 + warp; tile < tile1; tile += 4) {
-        const int r = tile * kAtRows + lane;
-        bool any = r >= kTopK ? (r - kTopK) < qq.nw : a.idx[(int64_t)t * kTopK + r] >= 0;
-        any = __any_sync(0xffffffffu, any);
-        if (lane == 0) sm.tiles[tile - tile0] = any ? 1 : 0;
+    // row slots of every tile of this split, resolved once; tiles whose rows are
+    // all masked (padding of short requests) are skipped
+    const int n_local = max(0, tile1 - tile0);
+    for (int u = tid; u < n_local * kAtRows; u += kAtThreads) {
+        int32_t raw;
+        const int32_t slot = row_slot(a, qq, t, tile0 * kAtRows + u, &raw);
+        sm.slot[u] = slot;
+        sm.is_raw[u] = (int8_t)raw;
     }
-    __syncthreads();
-    if (tid == 0) {
-        int n = 0;
-        for (int tile = tile0; tile < tile1; tile++)
-            if (sm.tiles[tile - tile0]) sm.tiles[n++] = (int16_t)tile;
-        sm.n_tiles = n;
-    }
-    __syncthreads();
-    const int nt = sm.n_tiles;
-
-    // prologue: Q (heads 16g..16g+15) and the first two tiles
     {
         const __nv_bfloat16 *qsrc = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                                     ((int64_t)t * a.heads + g * kAtHeads) * kKvDim;
@@ -263,12 +245,22 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             cp_async16(sm.q + h * kAtStride + c * 8, qsrc + h * kKvDim + c * 8);
         }
     }
-    for (int j = 0; j < 2; j++) {
-        if (j < nt) fill_slots(a, qq, t, sm.tiles[j], j, sm);
+    __syncthreads();
+    for (int lt = warp; lt < n_local; lt += 4) {
+        const bool any = __any_sync(0xffffffffu, sm.slot[lt * kAtRows + lane] >= 0);
+        if (lane == 0) sm.tiles[lt] = any ? 1 : 0;
     }
     __syncthreads();
+    if (tid == 0) {
+        int n = 0;
+        for (int lt = 0; lt < n_local; lt++)
+            if (sm.tiles[lt]) sm.tiles[n++] = (int16_t)lt;
+        sm.n_tiles = n;
+    }
+    __syncthreads();
+    const int nt = sm.n_tiles;
     for (int j = 0; j < 2; j++) {
-        if (j < nt) issue_loads(a, j, sm);
+        if (j < nt) issue_loads(a, sm.tiles[j], j, sm);
         else cp_async_commit();
     }
 
@@ -285,10 +277,12 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
         const int st = j & 1;
         if (j + 1 < nt) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
+        const int lt = sm.tiles[j];
+        const int32_t *slots = sm.slot + lt * kAtRows;
         if (fp8) {
-            expand_fp8(st, sm);
+            expand_fp8(lt, st, sm);
         } else if (tid < kAtRows) {
-            const float one = sm.slot[st][tid] >= 0 ? 1.0f : 0.0f;
+            const float one = slots[tid] >= 0 ? 1.0f : 0.0f;
             sm.rscale[st][tid][0] = sm.rscale[st][tid][1] = one;
             sm.rscale[st][tid][2] = sm.rscale[st][tid][3] = one;
         }
@@ -302,22 +296,22 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
                                 (uint32_t)((warp * 8 + (lane & 7)) * kAtStride + (lane >> 3) * 8) * 2;
 #pragma unroll 1
         for (int blk = 0; blk < 5; blk++) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
             const int k0 = blk * 8, nk = blk < 4 ? 8 : 4;
-#pragma unroll 2
+#pragma unroll 4
             for (int kk = k0; kk < k0 + nk; kk += 2) {
                 uint32_t a0[4], a1[4], bf[4];
                 ldsm_x4(a0, q_base + kk * 32);
                 ldsm_x4(a1, q_base + (kk + 1) * 32);
                 ldsm_x4(bf, k_base + kk * 32);
-                mma16816(acc, a0, bf[0], bf[1]);
-                mma16816(acc, a1, bf[2], bf[3]);
+                mma16816(acc0, a0, bf[0], bf[1]);
+                mma16816(acc1, a1, bf[2], bf[3]);
             }
 #pragma unroll
             for (int jj = 0; jj < 4; jj++) {
                 const int row = warp * 8 + 2 * tq + (jj & 1);
                 const float sc = blk < 4 ? sm.rscale[st][row][blk] : 1.0f;
-                s[jj] = fmaf(acc[jj], sc, s[jj]);
+                s[jj] = fmaf(acc0[jj] + acc1[jj], sc, s[jj]);
             }
         }
         // scale, mask, per-head tile max
@@ -325,7 +319,7 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
 #pragma unroll
         for (int jj = 0; jj < 4; jj++) {
             const int row = warp * 8 + 2 * tq + (jj & 1);
-            const float v = sm.slot[st][row] >= 0 ? s[jj] * scale2 : -INFINITY;
+            const float v = slots[row] >= 0 ? s[jj] * scale2 : -INFINITY;
             s[jj] = v;
             tmax[jj >> 1] = fmaxf(tmax[jj >> 1], v);
         }
@@ -424,13 +418,8 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
             }
         }
         __syncthreads();   // stage `st` and the tile are free again
-        if (j + 2 < nt) {
-            fill_slots(a, qq, t, sm.tiles[j + 2], st, sm);
-            __syncthreads();
-            issue_loads(a, st, sm);
-        } else {
-            cp_async_commit();
-        }
+        if (j + 2 < nt) issue_loads(a, sm.tiles[j + 2], st, sm);
+        else cp_async_commit();
     }
 
     const int h0 = g * kAtHeads;
@@ -516,8 +505,10 @@ static int at_tiles(int window) { return (kTopK + window + kAtRows - 1) / kAtRow
 
 static int at_splits(int num_q, int heads, int window, bool decode) {
     if (!decode) return 1;
+    // split each query's rows so that the grid stays within one wave
+    // (2 CTAs per SM on 148 SMs)
     const int ctas = num_q * (heads / kAtHeads);
-    int sp = (2 * 148 * 2 + ctas - 1) / ctas;
+    int sp = (2 * 148) / ctas;
     sp = sp < 1 ? 1 : sp;
     const int nt = at_tiles(window);
     sp = sp > 5 ? 5 : sp;

@@ -191,18 +191,18 @@ __device__ __forceinline__ float pool4(const float (&x)[4], const float (&z)[4])
     return __fdiv_rn(num, den);
 }
 
-// Locate block `blk` of request b; returns the compressed slot or -1.
-__device__ __forceinline__ int64_t compress_target(int b, int blk, const int32_t *cu_x,
-                                                   const int32_t *start_pos, int max_rows,
-                                                   const int32_t *page_table, int pt_stride,
-                                                   int64_t num_slots, int32_t *status,
-                                                   int64_t *row0, bool leader) {
+// First input row of block `blk` of request b (or -1 when there is no such
+// complete block, or the request is malformed); `j` gets the block's
+// compressed index.
+__device__ __forceinline__ int64_t compress_row(int b, int blk, const int32_t *cu_x,
+                                                const int32_t *start_pos, int max_rows,
+                                                int32_t *status, bool leader, int32_t *j) {
     const int32_t x0 = cu_x[b], n = cu_x[b + 1] - x0;
+    const int32_t sp = start_pos[b];
     if (n < 4) {                      // no complete block: nothing to compress
         if (n < 0 && leader && blk == 0) report(status, CSA_ERR_BOUNDS);
         return -1;
     }
-    const int32_t sp = start_pos[b];
     if (sp < 0 || (sp & 3) != 0) {
         if (leader && blk == 0) report(status, CSA_ERR_BOUNDS);
         return -1;
@@ -210,7 +210,14 @@ __device__ __forceinline__ int64_t compress_target(int b, int blk, const int32_t
     if (n > max_rows && leader && blk == 0) report(status, CSA_ERR_BOUNDS);
     const int nblk = min(n, max_rows) / 4;
     if (blk >= nblk) return -1;
-    const int32_t j = sp / 4 + blk;
+    *j = sp / 4 + blk;
+    return (int64_t)x0 + 4 * blk;
+}
+
+// Compressed slot of compressed index j of request b, or -1 (reported).
+__device__ __forceinline__ int64_t compress_slot(int b, int32_t j, const int32_t *page_table,
+                                                 int pt_stride, int64_t num_slots,
+                                                 int32_t *status, bool leader) {
     if (j / kC4Page >= pt_stride) {
         if (leader) report(status, CSA_ERR_BOUNDS);
         return -1;
@@ -221,7 +228,6 @@ __device__ __forceinline__ int64_t compress_target(int b, int blk, const int32_t
         if (leader) report(status, CSA_ERR_BOUNDS);
         return -1;
     }
-    *row0 = (int64_t)x0 + 4 * blk;
     return slot;
 }
 
@@ -232,21 +238,26 @@ compress_kv_kernel(const float *__restrict__ x, const float *__restrict__ gate,
                    const int32_t *start_pos, int max_rows, const int32_t *page_table,
                    int pt_stride, int fmt, uint8_t *out, int64_t num_slots, int32_t *status) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int64_t row0 = 0;
-    const int64_t slot = compress_target(blockIdx.y, blockIdx.x, cu_x, start_pos, max_rows,
-                                         page_table, pt_stride, num_slots, status, &row0,
-                                         threadIdx.x == 0);
-    if (slot < 0) return;
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    int32_t j = 0;
+    const int64_t row0 = compress_row(blockIdx.y, blockIdx.x, cu_x, start_pos, max_rows, status,
+                                      threadIdx.x == 0, &j);
+    if (row0 < 0) return;
+    // the input rows are fetched before the page-table lookup resolves
+    float4 xv[4], gv[4], bv[4];
     if (kv_active(warp, lane)) {
         const int c = kv_channel(warp, lane);
-        float4 xv[4], gv[4], bv[4];
 #pragma unroll
         for (int i = 0; i < 4; i++) {
             xv[i] = *reinterpret_cast<const float4 *>(x + (row0 + i) * kKvDim + c);
             gv[i] = *reinterpret_cast<const float4 *>(gate + (row0 + i) * kKvDim + c);
             bv[i] = *reinterpret_cast<const float4 *>(bias + i * kKvDim + c);
         }
+    }
+    const int64_t slot = compress_slot(blockIdx.y, j, page_table, pt_stride, num_slots, status,
+                                       threadIdx.x == 0);
+    if (slot < 0) return;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (kv_active(warp, lane)) {
         float xs[4], zs[4];
 #define CSA_POOL_LANE(F)                                                              \
         for (int i = 0; i < 4; i++) { xs[i] = xv[i].F; zs[i] = gv[i].F + bv[i].F; } \
@@ -273,22 +284,26 @@ compress_index_kernel(const float *__restrict__ x, const float *__restrict__ gat
     constexpr int D = 32 * E;
     const int lane = threadIdx.x & 31;
     const int blk = blockIdx.x * 8 + (threadIdx.x >> 5);
-    int64_t row0 = 0;
-    const int64_t slot = compress_target(blockIdx.y, blk, cu_x, start_pos, max_rows, page_table,
-                                         pt_stride, num_slots, status, &row0, lane == 0);
-    if (slot < 0) return;
-    float v[E];
+    int32_t j = 0;
+    const int64_t row0 = compress_row(blockIdx.y, blk, cu_x, start_pos, max_rows, status,
+                                      lane == 0, &j);
+    if (row0 < 0) return;
+    float xs[E][4], zs[E][4];
 #pragma unroll
     for (int e = 0; e < E; e++) {
         const int c = lane * E + e;
-        float xs[4], zs[4];
 #pragma unroll
         for (int i = 0; i < 4; i++) {
-            xs[i] = x[(row0 + i) * D + c];
-            zs[i] = gate[(row0 + i) * D + c] + bias[i * D + c];
+            xs[e][i] = x[(row0 + i) * D + c];
+            zs[e][i] = gate[(row0 + i) * D + c] + bias[i * D + c];
         }
-        v[e] = pool4(xs, zs);
     }
+    const int64_t slot = compress_slot(blockIdx.y, j, page_table, pt_stride, num_slots, status,
+                                       lane == 0);
+    if (slot < 0) return;
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) v[e] = pool4(xs[e], zs[e]);
     rotate<E>(v, lane);
     quant_index_row<E>(v, lane, fmt, slot, codes, block_scales, scales);
 }

@@ -15,8 +15,11 @@
 //   warp 1  MMA issuer: Di/32-byte K-steps of tcgen05.mma into one of two
 //           TMEM accumulators, commits free the stage and hand the
 //           accumulator to the epilogue,
-//   warps 2-5 epilogue: tcgen05.ld of the key's row, ReLU, head-weighted sum
-//           per query, times the key's scale, one coalesced float store.
+//   warps 2-9 epilogue, two groups of four warps (each group covers the four
+//           TMEM lane quadrants; group 0 takes the even tiles / accumulator 0,
+//           group 1 the odd tiles / accumulator 1): tcgen05.ld of the key's
+//           row, ReLU, head-weighted sum per query, times the key's scale,
+//           one coalesced float store.
 // Formats: FP8 E4M3 (kind::f8f6f4), bf16 (kind::f16), and FP4 E2M1 with
 // unsigned-E4M3 block-16 scales (kind::mxf4nvf4 block-scaled): warp 0's other
 // lanes gather each tile's key block scales into the 128-row scale-factor
@@ -29,7 +32,7 @@
 
 namespace csa {
 
-constexpr int kTcThreads = 192;   // 6 warps
+constexpr int kTcThreads = 320;   // 10 warps: producer, MMA, two epilogue groups of 4
 constexpr int kTcTile = 128;      // keys per tile (two 64-row pages)
 
 template <int RB>
@@ -51,7 +54,7 @@ struct TcParams {
 };
 
 template <int FMT, int RB>
-__global__ void __launch_bounds__(kTcThreads)
+__global__ void __launch_bounds__(kTcThreads, 2)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                   const TcParams p) {
     using G = TcGeom<RB>;
@@ -121,7 +124,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         }
         for (int i = 0; i < 2; i++) {
             tc::mbar_init(tc::saddr(&tfull[i]), 1);
-            tc::mbar_init(tc::saddr(&tempty[i]), 4);
+            tc::mbar_init(tc::saddr(&tempty[i]), 4);     // the 4 warps of one group
         }
         tc::mbar_init(tc::saddr(drain), 1);
         *abort_flag = 0;
@@ -294,7 +297,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             tc::mbar_wait(tc::saddr(drain), 0, nullptr);
         }
     } else {
-        // ---------------- epilogue (warps 2-5 cover the four TMEM lane quadrants)
+        // ---------------- epilogue: group eg = (warp-2)/4 takes tiles i with i%2 == eg
+        const int eg = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
@@ -314,13 +318,13 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             return FMT == CSA_FMT_BF16 ? 1.0f : __ldg(a.k_scales + slot);
         };
         bool valid_next = false;
-        float kscale_next = key_scale(0, valid_next);
-        for (int i = 0; i < my_tiles; i++) {
-            const int acc = i & 1;
+        float kscale_next = eg < my_tiles ? key_scale(eg, valid_next) : 0.0f;
+        for (int i = eg; i < my_tiles; i += 2) {
+            const int acc = eg;
             const int sk = (tile_begin + i) * kTcTile + row;
             const float kscale = kscale_next;
             const bool valid = valid_next;
-            if (i + 1 < my_tiles) kscale_next = key_scale(i + 1, valid_next);
+            if (i + 2 < my_tiles) kscale_next = key_scale(i + 2, valid_next);
             if (!tc::mbar_wait(tc::saddr(&tfull[acc]), (uint32_t)((i >> 1) & 1), abort_flag)) {
                 if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
                 *abort_flag = 1;
@@ -329,16 +333,28 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             tc::fence_after_sync();
             float out[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t ta = tmem_base + lane_addr + (uint32_t)(acc * p.n);
-            for (int c0 = 0; c0 < p.n; c0 += 16) {
-                float v[16];
-                tc::tmem_ld16(ta + (uint32_t)c0, v);
-                float sacc = 0.0f;
+            for (int c0 = 0; c0 < p.n; c0 += 32) {
+                // 32 columns per TMEM round trip; sum_j w'[c+j] * ReLU(acc[c+j])
+                // over 16-column groups (a group never straddles two queries:
+                // hi_pad is a multiple of 16)
+                uint32_t v[32];
+                tc::tmem_ld32_nowait(ta + (uint32_t)c0, v);
+                tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; j++) sacc = fmaf(w_s[c0 + j], fmaxf(v[j], 0.0f), sacc);
-                const int qi = c0 / p.hi_pad;
+                for (int q16 = 0; q16 < 2; q16++) {
+                    const int c = c0 + 16 * q16;
+                    if (c < p.n) {
+                        float sacc = 0.0f;
 #pragma unroll
-                for (int x = 0; x < 4; x++)
-                    if (x == qi) out[x] += sacc;
+                        for (int j = 0; j < 16; j++)
+                            sacc = fmaf(w_s[c + j], fmaxf(__uint_as_float(v[16 * q16 + j]), 0.0f),
+                                        sacc);
+                        const int qi = c / p.hi_pad;
+#pragma unroll
+                        for (int x = 0; x < 4; x++)
+                            if (x == qi) out[x] += sacc;
+                    }
+                }
             }
             tc::fence_before_sync();
             __syncwarp();
@@ -429,12 +445,28 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
     while (cols < need) cols <<= 1;
     p.tmem_cols = cols;
     p.num_pages = (int)(a.num_slots / kC4Page);
-    p.stages = rb >= 128 ? 4 : rb == 64 ? 8 : 12;     // ~64 KB of key tiles in flight
+    // ~96 KB of key tiles in flight per CTA, two CTAs per SM
+    p.stages = rb == 256 ? 3 : rb == 128 ? 6 : rb == 64 ? 12 : 16;
     const int tiles_max = (a.max_c4_len + kTcTile - 1) / kTcTile;
     const int groups = (a.num_q + p.qg - 1) / p.qg;
-    const int ctas_per_sm = 512 / cols < 3 ? 512 / cols : 3;
-    const int target = 148 * ctas_per_sm;
-    int chunks = (target + groups - 1) / groups;
+    // one wave: at most (SMs x resident CTAs per SM) CTAs, split evenly over
+    // the query groups (a second, nearly empty wave would double the time)
+    int sms = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    p.tiles_per_cta = tiles_max;                      // upper bound for the estimate
+    // 228 KB of shared memory per SM, 1 KB of it reserved per resident CTA
+    const size_t smem_est = tc_smem_bytes(rb, fp4, p) + 1024;
+    int by_smem = (int)((228 * 1024) / smem_est);
+    int ctas_per_sm = 512 / cols;
+    if (by_smem < ctas_per_sm) ctas_per_sm = by_smem;
+    if (ctas_per_sm > 2) ctas_per_sm = 2;             // register budget: 320 threads x 102
+    if (ctas_per_sm < 1) ctas_per_sm = 1;
+    const int target = sms * ctas_per_sm;
+    int chunks = target / groups;
     if (chunks > tiles_max) chunks = tiles_max;
     if (chunks < 1) chunks = 1;
     p.tiles_per_cta = (tiles_max + chunks - 1) / chunks;

@@ -26,6 +26,7 @@ constexpr int kTkThreads = 512;
 constexpr int kTkChunk = 8192;
 constexpr int kTkWarps = kTkThreads / 32;
 constexpr int kHistBins = 4096;
+constexpr int kTk2Smem = 16384;      // stage-2 candidates staged in shared memory
 
 __device__ __forceinline__ uint32_t order_key(float f, int32_t *status) {
     uint32_t u = __float_as_uint(f);
@@ -42,7 +43,11 @@ struct TkShared {
     uint32_t warp_a[kTkWarps];
     uint32_t warp_b[kTkWarps];
     uint32_t digit, above;
+    int32_t row_b, row_nvis;
 };
+// the key buffers that follow TkShared in dynamic shared memory start on a
+// 16-byte boundary (they are read and written with 16-byte vectors)
+constexpr size_t kTkKeysOffset = (sizeof(TkShared) + 15) & ~(size_t)15;
 
 // Exclusive scan of one value per thread over the block; returns the prefix
 // and writes the block total to *total.  Uses sh.warp_a.
@@ -132,43 +137,46 @@ __device__ void radix_threshold(const uint32_t *keys, int n, int K, TkShared &sh
 
 // Walks keys[0..n) in index order and calls emit(pos, i, key) for the
 // selected ones: key > T, or key == T among the first need_eq such keys.
+// Each warp owns one contiguous segment: it counts its segment with ballots,
+// one block barrier publishes the per-warp counts, then every warp writes its
+// selected elements at their global ranks.
 template <typename Emit>
 __device__ void ordered_compact(const uint32_t *keys, int n, uint32_t T, int need_eq, int K,
                                 TkShared &sh, Emit emit) {
+    (void)K;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
-    uint32_t base_eq = 0, base_out = 0;
-    for (int r0 = 0; r0 < n && base_out < (uint32_t)K; r0 += kTkThreads) {
-        const int i = r0 + threadIdx.x;
-        const uint32_t k = i < n ? keys[i] : 0u;
-        const bool eq = i < n && k == T;
-        const bool gt = i < n && k > T;
+    const int seg = ((n + kTkWarps - 1) / kTkWarps + 31) & ~31;
+    const int beg = min(n, warp * seg), end = min(n, beg + seg);
+    uint32_t gt_w = 0, eq_w = 0;
+    for (int i = beg + lane; i < end + lane; i += 32) {   // uniform trip count per warp
+        const uint32_t k = i < end ? keys[i] : 0u;
+        gt_w += __popc(__ballot_sync(0xffffffffu, i < end && k > T));
+        eq_w += __popc(__ballot_sync(0xffffffffu, i < end && k == T));
+    }
+    if (lane == 0) {
+        sh.warp_a[warp] = eq_w;
+        sh.warp_b[warp] = gt_w;
+    }
+    __syncthreads();
+    uint32_t eq_before = 0, gt_before = 0;
+    for (int w = 0; w < warp; w++) {
+        eq_before += sh.warp_a[w];
+        gt_before += sh.warp_b[w];
+    }
+    __syncthreads();    // the counts may be reused by the caller's next phase
+    uint32_t eq_seen = eq_before;
+    uint32_t out = gt_before + min(eq_before, (uint32_t)need_eq);
+    for (int i = beg + lane; i < end + lane; i += 32) {
+        const uint32_t k = i < end ? keys[i] : 0u;
+        const bool gt = i < end && k > T;
+        const bool eq = i < end && k == T;
         const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-        if (lane == 0) sh.warp_a[warp] = __popc(beq);
-        __syncthreads();
-        uint32_t eq_before = 0, eq_total = 0;
-#pragma unroll
-        for (int w = 0; w < kTkWarps; w++) {
-            const uint32_t x = sh.warp_a[w];
-            eq_before += (w < warp) ? x : 0u;
-            eq_total += x;
-        }
-        const uint32_t eq_rank = base_eq + eq_before + __popc(beq & lt);
-        const bool take = gt || (eq && eq_rank < (uint32_t)need_eq);
+        const bool take = gt || (eq && eq_seen + __popc(beq & lt) < (uint32_t)need_eq);
         const uint32_t btk = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) sh.warp_b[warp] = __popc(btk);
-        __syncthreads();
-        uint32_t tk_before = 0, tk_total = 0;
-#pragma unroll
-        for (int w = 0; w < kTkWarps; w++) {
-            const uint32_t x = sh.warp_b[w];
-            tk_before += (w < warp) ? x : 0u;
-            tk_total += x;
-        }
-        if (take) emit((int)(base_out + tk_before + __popc(btk & lt)), i, k);
-        base_eq += eq_total;
-        base_out += tk_total;
-        __syncthreads();
+        if (take) emit((int)(out + __popc(btk & lt)), i, k);
+        eq_seen += __popc(beq);
+        out += __popc(btk);
     }
 }
 
@@ -176,25 +184,45 @@ struct RowInfo {
     int b, n_vis;
 };
 
-__device__ __forceinline__ RowInfo row_info(int t, const int32_t *cu_q, int bs,
-                                            const int32_t *q_pos, const int32_t *c4_lens,
-                                            int max_c4_len, int pt_stride, int32_t *status,
-                                            bool leader) {
-    int lo = 0, hi = bs - 1;
-    while (lo < hi) {  // last b with cu_q[b] <= t
-        const int mid = (lo + hi + 1) >> 1;
-        if (cu_q[mid] <= t) lo = mid; else hi = mid - 1;
+// Request and visible length of query row t, found by warp 0 with coalesced
+// reads of cu_q and c4_lens (one round trip for up to 32 requests) and
+// published to the block through shared memory.
+__device__ RowInfo row_info(int t, const int32_t *cu_q, int bs, const int32_t *q_pos,
+                            const int32_t *c4_lens, int max_c4_len, int pt_stride,
+                            int32_t *status, bool leader, TkShared &sh) {
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int pos = q_pos ? q_pos[t] : 0;
+        int cnt = 0, len = 0;
+        for (int base = 0; base < bs; base += 32) {
+            const int i = base + lane;
+            const bool le = i < bs && cu_q[i] <= t;
+            const int li = i < bs ? c4_lens[i] : 0;
+            const uint32_t m = __ballot_sync(0xffffffffu, le);
+            const int c = __popc(m);
+            // the last request whose start is <= t is entry cnt+c-1
+            const int src = c > 0 ? c - 1 : 0;
+            const int lsel = __shfl_sync(0xffffffffu, li, src);
+            if (c > 0) len = lsel;
+            cnt += c;
+            if (m != 0xffffffffu) break;
+        }
+        if (lane == 0) {
+            int n = len;
+            if (q_pos) n = min(n, (pos + 1) / 4);
+            const int cap = min(max_c4_len, pt_stride * kC4Page);
+            if (n > cap) {
+                if (leader) report(status, CSA_ERR_BOUNDS);
+                n = cap;
+            }
+            sh.row_b = max(cnt - 1, 0);
+            sh.row_nvis = max(n, 0);
+        }
     }
+    __syncthreads();
     RowInfo r;
-    r.b = lo;
-    int n = c4_lens[lo];
-    if (q_pos) n = min(n, (q_pos[t] + 1) / 4);
-    const int cap = min(max_c4_len, pt_stride * kC4Page);
-    if (n > cap) {
-        if (leader) report(status, CSA_ERR_BOUNDS);
-        n = cap;
-    }
-    r.n_vis = max(n, 0);
+    r.b = sh.row_b;
+    r.n_vis = sh.row_nvis;
     return r;
 }
 
@@ -205,15 +233,27 @@ topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32
                    int32_t *status) {
     extern __shared__ __align__(16) uint8_t tk_smem[];
     TkShared &sh = *reinterpret_cast<TkShared *>(tk_smem);
-    uint32_t *skeys = reinterpret_cast<uint32_t *>(tk_smem + sizeof(TkShared));
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(tk_smem + kTkKeysOffset);
     const int t = blockIdx.y, c = blockIdx.x;
     const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
-                                threadIdx.x == 0 && c == 0);
+                                c == 0, sh);
     const int lo = c * kTkChunk;
     if (lo >= ri.n_vis) return;
     const int len = min(kTkChunk, ri.n_vis - lo);
     const float *row = logits + (int64_t)t * stride + lo;
-    for (int i = threadIdx.x; i < len; i += kTkThreads) skeys[i] = order_key(row[i], status);
+    if ((reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+        const int n4 = len / 4;
+        for (int i = threadIdx.x; i < n4; i += kTkThreads) {
+            const float4 v = reinterpret_cast<const float4 *>(row)[i];
+            skeys[4 * i] = order_key(v.x, status);
+            skeys[4 * i + 1] = order_key(v.y, status);
+            skeys[4 * i + 2] = order_key(v.z, status);
+            skeys[4 * i + 3] = order_key(v.w, status);
+        }
+        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTkThreads) skeys[i] = order_key(row[i], status);
+    } else {
+        for (int i = threadIdx.x; i < len; i += kTkThreads) skeys[i] = order_key(row[i], status);
+    }
     __syncthreads();
     const int K = min(kTopK, len);
     uint32_t T = 0;
@@ -232,10 +272,12 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
                    int max_c4_len, const int32_t *page_table, int pt_stride, int64_t num_slots,
                    int max_chunks, const uint32_t *cand_key, const int32_t *cand_idx,
                    int32_t *out_phys, int32_t *out_raw, int32_t *status) {
-    __shared__ TkShared sh;
+    extern __shared__ __align__(16) uint8_t tk2_smem[];
+    TkShared &sh = *reinterpret_cast<TkShared *>(tk2_smem);
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(tk2_smem + kTkKeysOffset);
     const int t = blockIdx.x;
     const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
-                                false);
+                                false, sh);
     const int n = ri.n_vis;
     int total = 0;
     if (n > 0) {
@@ -243,8 +285,28 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
         total = (nch - 1) * kTopK + min(kTopK, n - (nch - 1) * kTkChunk);
     }
     const int K = min(kTopK, total);
-    const uint32_t *keys = cand_key + (int64_t)t * max_chunks * kTopK;
+    const uint32_t *gkeys = cand_key + (int64_t)t * max_chunks * kTopK;
     const int32_t *idx = cand_idx + (int64_t)t * max_chunks * kTopK;
+    // candidates (keys and indices) up to kTk2Smem keys are staged in shared memory; longer rows
+    // are selected straight from the workspace (L2)
+    const uint32_t *keys = gkeys;
+    int32_t *sidx = reinterpret_cast<int32_t *>(skeys + kTk2Smem);
+    if (total <= kTk2Smem) {
+        for (int i = threadIdx.x * 4; i < total; i += kTkThreads * 4) {
+            if (i + 4 <= total) {
+                *reinterpret_cast<uint4 *>(skeys + i) = *reinterpret_cast<const uint4 *>(gkeys + i);
+                *reinterpret_cast<int4 *>(sidx + i) = *reinterpret_cast<const int4 *>(idx + i);
+            } else {
+                for (int j = i; j < total; j++) {
+                    skeys[j] = gkeys[j];
+                    sidx[j] = idx[j];
+                }
+            }
+        }
+        __syncthreads();
+        keys = skeys;
+        idx = sidx;
+    }
     const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
     uint32_t T = 0;
     int need_eq = total;
@@ -282,7 +344,7 @@ cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
     const int mc = topk_max_chunks(a.max_c4_len);
     uint32_t *ck = (uint32_t *)a.workspace;
     int32_t *ci = (int32_t *)((uint8_t *)a.workspace + (size_t)a.num_q * mc * kTopK * 4);
-    const size_t smem1 = sizeof(TkShared) + kTkChunk * sizeof(uint32_t);
+    const size_t smem1 = kTkKeysOffset + kTkChunk * sizeof(uint32_t);
     static int done[64] = {0};
     cudaError_t e0 = ensure_max_smem((const void *)topk_stage1_kernel, (int)smem1, done);
     if (e0 != cudaSuccess) return e0;
@@ -292,7 +354,11 @@ cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
                                                  ck, ci, a.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    topk_stage2_kernel<<<a.num_q, kTkThreads, 0, s>>>(a.c4_seq_lens, a.bs, a.cu_q, a.q_pos,
+    const size_t smem2 = kTkKeysOffset + kTk2Smem * (sizeof(uint32_t) + sizeof(int32_t));
+    static int done2[64] = {0};
+    e = ensure_max_smem((const void *)topk_stage2_kernel, (int)smem2, done2);
+    if (e != cudaSuccess) return e;
+    topk_stage2_kernel<<<a.num_q, kTkThreads, smem2, s>>>(a.c4_seq_lens, a.bs, a.cu_q, a.q_pos,
                                                       a.max_c4_len, a.page_table, a.pt_stride,
                                                       a.num_slots, mc, ck, ci, a.out_phys,
                                                       a.out_raw, a.status);
