@@ -44,6 +44,8 @@ struct AtSmem {
     alignas(16) uint8_t region[kRegionBytes];
     float p[kAtHeads * kAtPStride];         // probabilities of the tile, float32
     float rscale[2][kAtRows][4];            // per-row scales of the 4 latent blocks
+    float rope_mul[2][kAtRows];             // fp16 path: power-of-two scale of the RoPE part
+    float qmul[kAtHeads];                   // fp16 path: power-of-two scale of each query head
     float red_max[4][kAtHeads];
     float red_sum[4][kAtHeads];
     int32_t slot[kAtMaxTiles * kAtRows];    // row slots of the split's tiles (-1: masked)
@@ -209,6 +211,361 @@ __device__ __forceinline__ void expand_fp8(int lt, int st, AtSmem &sm) {
             *reinterpret_cast<uint4 *>(dst) =
                 valid ? *reinterpret_cast<const uint4 *>(row + 528 + (c - 32) * 16)
                       : make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Power of two 2^(top - e) for amax = f * 2^e with f in [0.5, 1), so that
+// amax times it lies in [2^(top-1), 2^top); 1 for amax == 0.  Exponents are
+// clamped to the normal float range.
+__device__ __forceinline__ float fit_pow2(float amax, int top) {
+    if (!(amax > 0.0f)) return 1.0f;
+    const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 126;
+    const int k = max(-126, min(126, top - e));
+    return __uint_as_float((uint32_t)(k + 127) << 23);
+}
+
+// FP8 -> fp16 expansion of staging `st` (local tile `lt`): E4M3 codes exactly
+// (one conversion per two codes); RoPE values times a per-row power of two
+// that brings the row's largest magnitude into [2^13, 2^14), which converts
+// exactly every bf16 value above 2^-30 of that maximum; block scales kept aside.
+__device__ __forceinline__ void expand_fp8_f16(int lt, int st, AtSmem &sm) {
+    const uint8_t *stage = sm.region + st * kStageBytes;
+    __half *tile = reinterpret_cast<__half *>(tile_ptr(CSA_FMT_FP8, st, sm));
+    const int32_t *slots = sm.slot + lt * kAtRows;
+    // RoPE: 8 threads per row, 8 values (16 bytes) each
+#pragma unroll
+    for (int it = 0; it < kAtRows * 8 / kAtThreads; it++) {
+        const int u = threadIdx.x + it * kAtThreads;
+        const int r = u >> 3, c = u & 7;
+        const bool valid = slots[r] >= 0;
+        const uint8_t *row = stage + r * kFp8RowBytes;
+        const uint4 w4 = valid ? *reinterpret_cast<const uint4 *>(row + 528 + c * 16)
+                               : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+        float v[8];
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            amax = fmaxf(amax, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        const float m = fit_pow2(amax, 14);
+        uint4 o;
+        o.x = pack_f16(v[0] * m, v[1] * m);
+        o.y = pack_f16(v[2] * m, v[3] * m);
+        o.z = pack_f16(v[4] * m, v[5] * m);
+        o.w = pack_f16(v[6] * m, v[7] * m);
+        *reinterpret_cast<uint4 *>(tile + r * kAtStride + 512 + c * 8) = o;
+        if (c == 0) {
+            const float4 sc = valid ? *reinterpret_cast<const float4 *>(row + 512)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            sm.rscale[st][r][0] = sc.x;
+            sm.rscale[st][r][1] = sc.y;
+            sm.rscale[st][r][2] = sc.z;
+            sm.rscale[st][r][3] = sc.w;
+            sm.rope_mul[st][r] = valid ? 1.0f / m : 0.0f;
+        }
+    }
+    for (int u = threadIdx.x; u < kAtRows * 32; u += kAtThreads) {
+        const int r = u / 32, c = u % 32;
+        __half *dst = tile + r * kAtStride + c * 16;
+        uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        if (slots[r] >= 0) {
+            const uint4 u4 = *reinterpret_cast<const uint4 *>(stage + r * kFp8RowBytes + c * 16);
+            const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                uint32_t lo, hi;
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"((uint16_t)(w[j] & 0xFFFF)));
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"((uint16_t)(w[j] >> 16)));
+                o[2 * j] = lo;
+                o[2 * j + 1] = hi;
+            }
+        }
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+// FP8 KV on fp16 tensor cores.  One CTA: query t, head group g (16 heads),
+// split sp.  Scores: fp16 query (scaled per head by a power of two into fp16
+// range) times exact E4M3 codes, per-block partial sums scaled by the row
+// scales in float32.  P V: the probabilities times the value block's row
+// scale, normalised per tile by a power of two, in fp16 (11 significant bits).
+__global__ void __launch_bounds__(kAtThreads, 2)
+sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part_o,
+                      float *part_ml) {
+    extern __shared__ __align__(16) uint8_t at_smem_raw[];
+    AtSmem &sm = *reinterpret_cast<AtSmem *>(at_smem_raw);
+    const int t = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    const AtQuery qq = at_query(a, t);
+    const int n_rows = kTopK + qq.nw;
+    const int tile0 = sp * tiles_per_split;
+    const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
+
+    const int n_local = max(0, tile1 - tile0);
+    for (int u = tid; u < n_local * kAtRows; u += kAtThreads) {
+        int32_t raw;
+        const int32_t slot = row_slot(a, qq, t, tile0 * kAtRows + u, &raw);
+        sm.slot[u] = slot;
+        sm.is_raw[u] = (int8_t)raw;
+    }
+    {
+        const __nv_bfloat16 *qsrc = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                    ((int64_t)t * a.heads + g * kAtHeads) * kKvDim;
+        for (int u = tid; u < kAtHeads * 72; u += kAtThreads) {
+            const int h = u / 72, c = u % 72;
+            cp_async16(sm.q + h * kAtStride + c * 8, qsrc + h * kKvDim + c * 8);
+        }
+        cp_async_commit();
+    }
+    __syncthreads();
+    for (int lt = warp; lt < n_local; lt += 4) {
+        const bool any = __any_sync(0xffffffffu, sm.slot[lt * kAtRows + lane] >= 0);
+        if (lane == 0) sm.tiles[lt] = any ? 1 : 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int n = 0;
+        for (int lt = 0; lt < n_local; lt++)
+            if (sm.tiles[lt]) sm.tiles[n++] = (int16_t)lt;
+        sm.n_tiles = n;
+    }
+    __syncthreads();
+    const int nt = sm.n_tiles;
+    for (int j = 0; j < 2; j++) {
+        if (j < nt) issue_loads(a, sm.tiles[j], j, sm);
+        else cp_async_commit();
+    }
+    // Q to fp16 in place: warp w converts heads 4w..4w+3, each times a power
+    // of two that brings its largest magnitude into [2^13, 2^14), so every
+    // bf16 value above 2^-30 of that maximum converts exactly
+    cp_async_wait<2>();
+    __syncthreads();
+    {
+        uint16_t *qh = reinterpret_cast<uint16_t *>(sm.q);
+        for (int h = warp * 4; h < warp * 4 + 4; h++) {
+            float v[18];
+            float amax = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 18; k++) {
+                v[k] = bf16_bits_to_f32(qh[h * kAtStride + lane + 32 * k]);
+                amax = fmaxf(amax, fabsf(v[k]));
+            }
+            amax = warp_max(amax);
+            const float m = fit_pow2(amax, 14);
+#pragma unroll
+            for (int k = 0; k < 18; k++) {
+                const __half hv = __float2half_rn(v[k] * m);
+                qh[h * kAtStride + lane + 32 * k] = *reinterpret_cast<const uint16_t *>(&hv);
+            }
+            if (lane == 0) sm.qmul[h] = 1.0f / m;
+        }
+    }
+    __syncthreads();
+
+    float qscale[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) qscale[h] = a.sm_scale * kLog2e * sm.qmul[gq + 8 * h];
+    float o[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    float pw = 1.0f;     // O holds (true partial output) * pw
+    const uint32_t q_base = smem_u32(sm.q) +
+                            (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
+                                       (lane >> 4) * 8) * 2;
+
+    for (int j = 0; j < nt; j++) {
+        const int st = j & 1;
+        if (j + 1 < nt) cp_async_wait<1>(); else cp_async_wait<0>();
+        __syncthreads();
+        const int lt = sm.tiles[j];
+        const int32_t *slots = sm.slot + lt * kAtRows;
+        expand_fp8_f16(lt, st, sm);
+        __syncthreads();
+        const __half *tile = reinterpret_cast<const __half *>(tile_ptr(CSA_FMT_FP8, st, sm));
+
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t k_base = smem_u32(tile) +
+                                (uint32_t)((warp * 8 + (lane & 7)) * kAtStride + (lane >> 3) * 8) * 2;
+#pragma unroll 1
+        for (int blk = 0; blk < 5; blk++) {
+            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+            const int k0 = blk * 8, nk = blk < 4 ? 8 : 4;
+#pragma unroll 4
+            for (int kk = k0; kk < k0 + nk; kk += 2) {
+                uint32_t a0[4], a1[4], bf[4];
+                ldsm_x4(a0, q_base + kk * 32);
+                ldsm_x4(a1, q_base + (kk + 1) * 32);
+                ldsm_x4(bf, k_base + kk * 32);
+                mma16816_f16(acc0, a0, bf[0], bf[1]);
+                mma16816_f16(acc1, a1, bf[2], bf[3]);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; jj++) {
+                const int row = warp * 8 + 2 * tq + (jj & 1);
+                const float sc = blk < 4 ? sm.rscale[st][row][blk] : sm.rope_mul[st][row];
+                s[jj] = fmaf(acc0[jj] + acc1[jj], sc, s[jj]);
+            }
+        }
+        float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) {
+            const int row = warp * 8 + 2 * tq + (jj & 1);
+            const float v = slots[row] >= 0 ? s[jj] * qscale[jj >> 1] : -INFINITY;
+            s[jj] = v;
+            tmax[jj >> 1] = fmaxf(tmax[jj >> 1], v);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 1));
+            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
+        }
+        if (tq == 0) {
+            sm.red_max[warp][gq] = tmax[0];
+            sm.red_max[warp][gq + 8] = tmax[1];
+        }
+        __syncthreads();
+        float m_new[2], alpha[2];
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int hh = gq + 8 * h;
+            const float mx = fmaxf(fmaxf(sm.red_max[0][hh], sm.red_max[1][hh]),
+                                   fmaxf(sm.red_max[2][hh], sm.red_max[3][hh]));
+            m_new[h] = fmaxf(m_run[h], mx);
+            alpha[h] = m_new[h] == -INFINITY ? 1.0f : exp2f(m_run[h] - m_new[h]);
+        }
+        float psum[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int jj = 0; jj < 4; jj++) {
+            const int h = jj >> 1;
+            const float pv = m_new[h] == -INFINITY ? 0.0f : exp2f(s[jj] - m_new[h]);
+            s[jj] = pv;
+            psum[h] += pv;
+        }
+        {
+            const int col = warp * 8 + 2 * tq;
+            *reinterpret_cast<float2 *>(sm.p + gq * kAtPStride + col) = make_float2(s[0], s[1]);
+            *reinterpret_cast<float2 *>(sm.p + (gq + 8) * kAtPStride + col) = make_float2(s[2], s[3]);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 1);
+            psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 2);
+        }
+        if (tq == 0) {
+            sm.red_sum[warp][gq] = psum[0];
+            sm.red_sum[warp][gq + 8] = psum[1];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int hh = gq + 8 * h;
+            const float ts = sm.red_sum[0][hh] + sm.red_sum[1][hh] + sm.red_sum[2][hh] +
+                             sm.red_sum[3][hh];
+            l_run[h] = l_run[h] * alpha[h] + ts;
+            m_run[h] = m_new[h];
+        }
+        // power-of-two normalisation of this tile's block-w row scales
+        const float smax = warp_max(sm.rscale[st][lane][warp]);
+        const float pw_new = smax > 0.0f ? fit_pow2(smax, 0) : pw;
+        const float rs = pw_new / pw;
+        pw = pw_new;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            o[i][0] *= alpha[0] * rs;
+            o[i][1] *= alpha[0] * rs;
+            o[i][2] *= alpha[1] * rs;
+            o[i][3] *= alpha[1] * rs;
+        }
+        const uint32_t v_base = smem_u32(tile) +
+                                (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
+                                           warp * 128 + (lane >> 4) * 8) * 2;
+#pragma unroll
+        for (int ks = 0; ks < kAtRows / 16; ks++) {
+            const int r0k = ks * 16 + 2 * tq;
+            const float2 p00 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k);
+            const float2 p10 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k);
+            const float2 p01 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k + 8);
+            const float2 p11 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k + 8);
+            const float c0 = sm.rscale[st][r0k][warp] * pw, c1 = sm.rscale[st][r0k + 1][warp] * pw;
+            const float c8 = sm.rscale[st][r0k + 8][warp] * pw, c9 = sm.rscale[st][r0k + 9][warp] * pw;
+            uint32_t af[4];
+            af[0] = pack_f16(p00.x * c0, p00.y * c1);
+            af[1] = pack_f16(p10.x * c0, p10.y * c1);
+            af[2] = pack_f16(p01.x * c8, p01.y * c9);
+            af[3] = pack_f16(p11.x * c8, p11.y * c9);
+#pragma unroll
+            for (int np = 0; np < 8; np++) {
+                uint32_t bf[4];
+                ldsm_x4_t(bf, v_base + (uint32_t)(ks * 16 * kAtStride + np * 16) * 2);
+                mma16816_f16(o[2 * np], af, bf[0], bf[1]);
+                mma16816_f16(o[2 * np + 1], af, bf[2], bf[3]);
+            }
+        }
+        __syncthreads();   // stage `st` and the tile are free again
+        if (j + 2 < nt) issue_loads(a, sm.tiles[j + 2], st, sm);
+        else cp_async_commit();
+    }
+
+    const float unpw = 1.0f / pw;
+    const int h0 = g * kAtHeads;
+    if (splits == 1) {
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int hh = gq + 8 * h;
+            const float inv = l_run[h] > 0.0f ? unpw / l_run[h] : 0.0f;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +
+                                  ((int64_t)t * a.heads + h0 + hh) * kLatent;
+#pragma unroll
+            for (int n8 = 0; n8 < 16; n8++) {
+                const int col = warp * 128 + n8 * 8 + 2 * tq;
+                *reinterpret_cast<uint32_t *>(orow + col) =
+                    pack_bf16(o[n8][2 * h] * inv, o[n8][2 * h + 1] * inv);
+            }
+            if (a.lse && warp == 0 && tq == 0)
+                a.lse[(int64_t)t * a.heads + h0 + hh] =
+                    l_run[h] > 0.0f ? (m_run[h] + log2f(l_run[h])) * 0.6931471805599453f
+                                    : -INFINITY;
+        }
+    } else {
+        const int64_t pbase = (((int64_t)t * gridDim.y + g) * splits + sp) * kAtHeads;
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const int hh = gq + 8 * h;
+            float *prow = part_o + (pbase + hh) * kLatent;
+#pragma unroll
+            for (int n8 = 0; n8 < 16; n8++) {
+                const int col = warp * 128 + n8 * 8 + 2 * tq;
+                *reinterpret_cast<float2 *>(prow + col) =
+                    make_float2(o[n8][2 * h] * unpw, o[n8][2 * h + 1] * unpw);
+            }
+            if (warp == 0 && tq == 0) {
+                part_ml[(pbase + hh) * 2] = m_run[h];
+                part_ml[(pbase + hh) * 2 + 1] = l_run[h];
+            }
         }
     }
 }
@@ -533,11 +890,19 @@ cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s) {
         pml = po + (size_t)a.num_q * a.heads * sp * kLatent;
     }
     const size_t smem = sizeof(AtSmem);
-    static int done[64] = {0};
-    cudaError_t e = ensure_max_smem((const void *)sparse_mqa_kernel, (int)smem, done);
-    if (e != cudaSuccess) return e;
     dim3 grid(a.num_q, groups, sp);
-    sparse_mqa_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
+    cudaError_t e;
+    if (a.kv_fmt == CSA_FMT_FP8) {
+        static int done[64] = {0};
+        e = ensure_max_smem((const void *)sparse_mqa_f16_kernel, (int)smem, done);
+        if (e != cudaSuccess) return e;
+        sparse_mqa_f16_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
+    } else {
+        static int done[64] = {0};
+        e = ensure_max_smem((const void *)sparse_mqa_kernel, (int)smem, done);
+        if (e != cudaSuccess) return e;
+        sparse_mqa_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess || sp == 1) return e;
     sparse_mqa_combine_kernel<<<a.num_q * a.heads, 128, 0, s>>>(a, sp, po, pml);
