@@ -36,16 +36,13 @@ constexpr int kAtMaxTiles = (kTopK + 1024 + kAtRows - 1) / kAtRows;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTileBytes = kAtRows * kAtStride * 2;             // one bf16 tile
 constexpr int kStageBytes = kAtRows * kFp8RowBytes;             // one FP8 staging buffer
-constexpr int kRegionBytes = 2 * kStageBytes + kTileBytes;      // >= 2 bf16 tiles
+constexpr int kRegionBytes = 2 * kStageBytes + kTileBytes;      // FP8: 2 stagings + fp16 tile
 
-struct AtSmem {
+struct AtSmem {                              // BF16 KV kernel
     __nv_bfloat16 q[kAtHeads * kAtStride];
-    // FP8: [staging 0 | staging 1 | tile];  BF16: [tile 0 | tile 1]
-    alignas(16) uint8_t region[kRegionBytes];
+    alignas(16) uint8_t region[2 * kTileBytes];   // [tile 0 | tile 1]
     float p[kAtHeads * kAtPStride];         // probabilities of the tile, float32
-    float rscale[2][kAtRows][4];            // per-row scales of the 4 latent blocks
-    float rope_mul[2][kAtRows];             // fp16 path: power-of-two scale of the RoPE part
-    float qmul[kAtHeads];                   // fp16 path: power-of-two scale of each query head
+    float rscale[2][kAtRows][4];            // 1 for live rows, 0 for masked ones
     float red_max[4][kAtHeads];
     float red_sum[4][kAtHeads];
     int32_t slot[kAtMaxTiles * kAtRows];    // row slots of the split's tiles (-1: masked)
@@ -53,7 +50,6 @@ struct AtSmem {
     int16_t tiles[kAtMaxTiles];             // non-empty tiles of this split (local index)
     int32_t n_tiles;
 };
-static_assert(2 * kTileBytes <= kRegionBytes, "region holds two bf16 tiles");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -137,82 +133,27 @@ __device__ __forceinline__ int32_t row_slot(const AttnArgs &a, const AtQuery &qq
     return (int32_t)s;
 }
 
-__device__ __forceinline__ __nv_bfloat16 *tile_ptr(int fmt, int st, AtSmem &sm) {
-    return reinterpret_cast<__nv_bfloat16 *>(
-        sm.region + (fmt == CSA_FMT_FP8 ? 2 * kStageBytes : st * kTileBytes));
+__device__ __forceinline__ __nv_bfloat16 *tile_ptr(int st, AtSmem &sm) {
+    return reinterpret_cast<__nv_bfloat16 *>(sm.region + st * kTileBytes);
 }
 
-// Issues the cp.async gathers of local tile `lt` into stage `st`.
+// Issues the cp.async gathers of the bf16 rows of local tile `lt` into tile `st`.
 __device__ __forceinline__ void issue_loads(const AttnArgs &a, int lt, int st, AtSmem &sm) {
     const uint8_t *c4 = reinterpret_cast<const uint8_t *>(a.c4_cache);
     const uint8_t *rc = reinterpret_cast<const uint8_t *>(a.raw_cache);
     const int32_t *slots = sm.slot + lt * kAtRows;
     const int8_t *raws = sm.is_raw + lt * kAtRows;
-    if (a.kv_fmt == CSA_FMT_BF16) {
-        __nv_bfloat16 *tile = tile_ptr(CSA_FMT_BF16, st, sm);
-        for (int u = threadIdx.x; u < kAtRows * 72; u += kAtThreads) {
-            const int r = u / 72, c = u % 72;
-            __nv_bfloat16 *dst = tile + r * kAtStride + c * 8;
-            const int32_t slot = slots[r];
-            if (slot < 0)
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
-            else
-                cp_async16(dst, (raws[r] ? rc : c4) + (int64_t)slot * kBf16RowBytes + c * 16);
-        }
-    } else {
-        uint8_t *stage = sm.region + st * kStageBytes;
-        for (int u = threadIdx.x; u < kAtRows * 41; u += kAtThreads) {
-            const int r = u / 41, c = u % 41;
-            const int32_t slot = slots[r];
-            if (slot >= 0)
-                cp_async16(stage + r * kFp8RowBytes + c * 16,
-                           (raws[r] ? rc : c4) + (int64_t)slot * kFp8RowBytes + c * 16);
-        }
+    __nv_bfloat16 *tile = tile_ptr(st, sm);
+    for (int u = threadIdx.x; u < kAtRows * 72; u += kAtThreads) {
+        const int r = u / 72, c = u % 72;
+        __nv_bfloat16 *dst = tile + r * kAtStride + c * 8;
+        const int32_t slot = slots[r];
+        if (slot < 0)
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
+        else
+            cp_async16(dst, (raws[r] ? rc : c4) + (int64_t)slot * kBf16RowBytes + c * 16);
     }
     cp_async_commit();
-}
-
-// FP8: expands staging `st` (local tile `lt`) into the bf16 tile (exact codes)
-// and the row scales.
-__device__ __forceinline__ void expand_fp8(int lt, int st, AtSmem &sm) {
-    const uint8_t *stage = sm.region + st * kStageBytes;
-    __nv_bfloat16 *tile = tile_ptr(CSA_FMT_FP8, st, sm);
-    const int32_t *slots = sm.slot + lt * kAtRows;
-    if (threadIdx.x < kAtRows) {
-        const int r = threadIdx.x;
-        float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (slots[r] >= 0) sc = *reinterpret_cast<const float4 *>(stage + r * kFp8RowBytes + 512);
-        sm.rscale[st][r][0] = sc.x;
-        sm.rscale[st][r][1] = sc.y;
-        sm.rscale[st][r][2] = sc.z;
-        sm.rscale[st][r][3] = sc.w;
-    }
-    for (int u = threadIdx.x; u < kAtRows * 40; u += kAtThreads) {
-        const int r = u / 40, c = u % 40;
-        __nv_bfloat16 *dst = tile + r * kAtStride + (c < 32 ? c * 16 : 512 + (c - 32) * 8);
-        const uint8_t *row = stage + r * kFp8RowBytes;
-        const bool valid = slots[r] >= 0;
-        if (c < 32) {
-            uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            if (valid) {
-                const uint4 u4 = *reinterpret_cast<const uint4 *>(row + c * 16);
-                const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const float2 lo = e4m3x2_to_f32x2((uint16_t)(w[j] & 0xFFFF));
-                    const float2 hi = e4m3x2_to_f32x2((uint16_t)(w[j] >> 16));
-                    o[2 * j] = pack_bf16(lo.x, lo.y);
-                    o[2 * j + 1] = pack_bf16(hi.x, hi.y);
-                }
-            }
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
-        } else {
-            *reinterpret_cast<uint4 *>(dst) =
-                valid ? *reinterpret_cast<const uint4 *>(row + 528 + (c - 32) * 16)
-                      : make_uint4(0, 0, 0, 0);
-        }
-    }
 }
 
 __device__ __forceinline__ void mma16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
@@ -239,18 +180,58 @@ __device__ __forceinline__ float fit_pow2(float amax, int top) {
     return __uint_as_float((uint32_t)(k + 127) << 23);
 }
 
+// ------------------------------------------------------------------ FP8 KV
+// The FP8 kernel keeps G groups of 16 heads in one CTA (4 warps per group):
+// every gathered tile is loaded and expanded once for all of them.
+
+template <int G>
+struct AtSmem8 {
+    __nv_bfloat16 q[G * kAtHeads * kAtStride];   // bf16 as loaded, then fp16 in place
+    alignas(16) uint8_t region[kRegionBytes];     // [staging 0 | staging 1 | fp16 tile]
+    float p[G][kAtHeads * kAtPStride];            // probabilities of the tile, per group
+    float rscale[2][kAtRows][4];                  // per-row scales of the 4 latent blocks
+    float rope_mul[2][kAtRows];                   // power-of-two scale of each row's RoPE part
+    float qmul[G * kAtHeads];                     // power-of-two scale of each query head
+    float red_max[G][4][kAtHeads];
+    float red_sum[G][4][kAtHeads];
+    int32_t slot[kAtMaxTiles * kAtRows];          // row slots of the split's tiles (-1: masked)
+    int8_t is_raw[kAtMaxTiles * kAtRows];
+    int16_t tiles[kAtMaxTiles];                   // non-empty tiles of this split (local index)
+    int32_t n_tiles;
+};
+
+// Issues the cp.async gathers of the packed FP8 rows of local tile `lt` into
+// staging buffer `st`.
+template <int G>
+__device__ __forceinline__ void issue_loads8(const AttnArgs &a, int lt, int st, AtSmem8<G> &sm) {
+    constexpr int kThr = kAtThreads * G;
+    const uint8_t *c4 = reinterpret_cast<const uint8_t *>(a.c4_cache);
+    const uint8_t *rc = reinterpret_cast<const uint8_t *>(a.raw_cache);
+    const int32_t *slots = sm.slot + lt * kAtRows;
+    const int8_t *raws = sm.is_raw + lt * kAtRows;
+    uint8_t *stage = sm.region + st * kStageBytes;
+    for (int u = threadIdx.x; u < kAtRows * 41; u += kThr) {
+        const int r = u / 41, c = u % 41;
+        const int32_t slot = slots[r];
+        if (slot >= 0)
+            cp_async16(stage + r * kFp8RowBytes + c * 16,
+                       (raws[r] ? rc : c4) + (int64_t)slot * kFp8RowBytes + c * 16);
+    }
+    cp_async_commit();
+}
+
 // FP8 -> fp16 expansion of staging `st` (local tile `lt`): E4M3 codes exactly
 // (one conversion per two codes); RoPE values times a per-row power of two
 // that brings the row's largest magnitude into [2^13, 2^14), which converts
 // exactly every bf16 value above 2^-30 of that maximum; block scales kept aside.
-__device__ __forceinline__ void expand_fp8_f16(int lt, int st, AtSmem &sm) {
+template <int G>
+__device__ __forceinline__ void expand8(int lt, int st, AtSmem8<G> &sm) {
+    constexpr int kThr = kAtThreads * G;
     const uint8_t *stage = sm.region + st * kStageBytes;
-    __half *tile = reinterpret_cast<__half *>(tile_ptr(CSA_FMT_FP8, st, sm));
+    __half *tile = reinterpret_cast<__half *>(sm.region + 2 * kStageBytes);
     const int32_t *slots = sm.slot + lt * kAtRows;
-    // RoPE: 8 threads per row, 8 values (16 bytes) each
-#pragma unroll
-    for (int it = 0; it < kAtRows * 8 / kAtThreads; it++) {
-        const int u = threadIdx.x + it * kAtThreads;
+    // RoPE: 8 threads per row, 8 values (16 bytes) each; whole warps take part
+    for (int u = threadIdx.x; u < kAtRows * 8; u += kThr) {
         const int r = u >> 3, c = u & 7;
         const bool valid = slots[r] >= 0;
         const uint8_t *row = stage + r * kFp8RowBytes;
@@ -285,7 +266,7 @@ __device__ __forceinline__ void expand_fp8_f16(int lt, int st, AtSmem &sm) {
             sm.rope_mul[st][r] = valid ? 1.0f / m : 0.0f;
         }
     }
-    for (int u = threadIdx.x; u < kAtRows * 32; u += kAtThreads) {
+    for (int u = threadIdx.x; u < kAtRows * 32; u += kThr) {
         const int r = u / 32, c = u % 32;
         __half *dst = tile + r * kAtStride + c * 16;
         uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -306,26 +287,36 @@ __device__ __forceinline__ void expand_fp8_f16(int lt, int st, AtSmem &sm) {
     }
 }
 
-// FP8 KV on fp16 tensor cores.  One CTA: query t, head group g (16 heads),
-// split sp.  Scores: fp16 query (scaled per head by a power of two into fp16
-// range) times exact E4M3 codes, per-block partial sums scaled by the row
+__device__ __forceinline__ void group_sync(int grp) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(kAtThreads) : "memory");
+}
+
+// FP8 KV on fp16 tensor cores.  One CTA: query t, head groups
+// blockIdx.y*G .. +G-1 (16 heads each), split sp of the row list.  Warp w
+// works for head group w/4: rows 8(w%4).. of each tile in Q K^T, latent
+// columns 128(w%4).. in P V.  Scores: fp16 query (scaled per head by a power
+// of two) times exact E4M3 codes, per-block partial sums scaled by the row
 // scales in float32.  P V: the probabilities times the value block's row
 // scale, normalised per tile by a power of two, in fp16 (11 significant bits).
-__global__ void __launch_bounds__(kAtThreads, 2)
-sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part_o,
+template <int G>
+__global__ void __launch_bounds__(kAtThreads * G, G == 1 ? 2 : 1)
+sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part_o,
                       float *part_ml) {
+    constexpr int kThr = kAtThreads * G;
     extern __shared__ __align__(16) uint8_t at_smem_raw[];
-    AtSmem &sm = *reinterpret_cast<AtSmem *>(at_smem_raw);
-    const int t = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
+    AtSmem8<G> &sm = *reinterpret_cast<AtSmem8<G> *>(at_smem_raw);
+    const int t = blockIdx.x, sp = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = warp >> 2, wq = warp & 3;
     const int gq = lane >> 2, tq = lane & 3;
+    const int hg = blockIdx.y * G + grp;          // global 16-head group of this warp
     const AtQuery qq = at_query(a, t);
     const int n_rows = kTopK + qq.nw;
     const int tile0 = sp * tiles_per_split;
     const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
 
     const int n_local = max(0, tile1 - tile0);
-    for (int u = tid; u < n_local * kAtRows; u += kAtThreads) {
+    for (int u = tid; u < n_local * kAtRows; u += kThr) {
         int32_t raw;
         const int32_t slot = row_slot(a, qq, t, tile0 * kAtRows + u, &raw);
         sm.slot[u] = slot;
@@ -333,15 +324,15 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
     }
     {
         const __nv_bfloat16 *qsrc = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
-                                    ((int64_t)t * a.heads + g * kAtHeads) * kKvDim;
-        for (int u = tid; u < kAtHeads * 72; u += kAtThreads) {
+                                    ((int64_t)t * a.heads + blockIdx.y * G * kAtHeads) * kKvDim;
+        for (int u = tid; u < G * kAtHeads * 72; u += kThr) {
             const int h = u / 72, c = u % 72;
             cp_async16(sm.q + h * kAtStride + c * 8, qsrc + h * kKvDim + c * 8);
         }
         cp_async_commit();
     }
     __syncthreads();
-    for (int lt = warp; lt < n_local; lt += 4) {
+    for (int lt = warp; lt < n_local; lt += 4 * G) {
         const bool any = __any_sync(0xffffffffu, sm.slot[lt * kAtRows + lane] >= 0);
         if (lane == 0) sm.tiles[lt] = any ? 1 : 0;
     }
@@ -355,7 +346,7 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
     __syncthreads();
     const int nt = sm.n_tiles;
     for (int j = 0; j < 2; j++) {
-        if (j < nt) issue_loads(a, sm.tiles[j], j, sm);
+        if (j < nt) issue_loads8(a, sm.tiles[j], j, sm);
         else cp_async_commit();
     }
     // Q to fp16 in place: warp w converts heads 4w..4w+3, each times a power
@@ -387,15 +378,23 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
 
     float qscale[2];
 #pragma unroll
-    for (int h = 0; h < 2; h++) qscale[h] = a.sm_scale * kLog2e * sm.qmul[gq + 8 * h];
+    for (int h = 0; h < 2; h++)
+        qscale[h] = a.sm_scale * kLog2e * sm.qmul[grp * kAtHeads + gq + 8 * h];
     float o[16][4];
 #pragma unroll
     for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
     float pw = 1.0f;     // O holds (true partial output) * pw
-    const uint32_t q_base = smem_u32(sm.q) +
-                            (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
-                                       (lane >> 4) * 8) * 2;
+    float *p_s = sm.p[grp];
+    const uint32_t q_base =
+        smem_u32(sm.q) + (uint32_t)((grp * kAtHeads + (lane & 7) + ((lane >> 3) & 1) * 8) *
+                                        kAtStride + (lane >> 4) * 8) * 2;
+    const __half *tile = reinterpret_cast<const __half *>(sm.region + 2 * kStageBytes);
+    const uint32_t k_base =
+        smem_u32(tile) + (uint32_t)((wq * 8 + (lane & 7)) * kAtStride + (lane >> 3) * 8) * 2;
+    const uint32_t v_base =
+        smem_u32(tile) + (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride + wq * 128 +
+                                    (lane >> 4) * 8) * 2;
 
     for (int j = 0; j < nt; j++) {
         const int st = j & 1;
@@ -403,13 +402,10 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
         __syncthreads();
         const int lt = sm.tiles[j];
         const int32_t *slots = sm.slot + lt * kAtRows;
-        expand_fp8_f16(lt, st, sm);
+        expand8(lt, st, sm);
         __syncthreads();
-        const __half *tile = reinterpret_cast<const __half *>(tile_ptr(CSA_FMT_FP8, st, sm));
 
         float s[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t k_base = smem_u32(tile) +
-                                (uint32_t)((warp * 8 + (lane & 7)) * kAtStride + (lane >> 3) * 8) * 2;
 #pragma unroll 1
         for (int blk = 0; blk < 5; blk++) {
             float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -425,7 +421,7 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             }
 #pragma unroll
             for (int jj = 0; jj < 4; jj++) {
-                const int row = warp * 8 + 2 * tq + (jj & 1);
+                const int row = wq * 8 + 2 * tq + (jj & 1);
                 const float sc = blk < 4 ? sm.rscale[st][row][blk] : sm.rope_mul[st][row];
                 s[jj] = fmaf(acc0[jj] + acc1[jj], sc, s[jj]);
             }
@@ -433,7 +429,7 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
         float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
         for (int jj = 0; jj < 4; jj++) {
-            const int row = warp * 8 + 2 * tq + (jj & 1);
+            const int row = wq * 8 + 2 * tq + (jj & 1);
             const float v = slots[row] >= 0 ? s[jj] * qscale[jj >> 1] : -INFINITY;
             s[jj] = v;
             tmax[jj >> 1] = fmaxf(tmax[jj >> 1], v);
@@ -444,16 +440,16 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
         }
         if (tq == 0) {
-            sm.red_max[warp][gq] = tmax[0];
-            sm.red_max[warp][gq + 8] = tmax[1];
+            sm.red_max[grp][wq][gq] = tmax[0];
+            sm.red_max[grp][wq][gq + 8] = tmax[1];
         }
-        __syncthreads();
+        group_sync(grp);
         float m_new[2], alpha[2];
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             const int hh = gq + 8 * h;
-            const float mx = fmaxf(fmaxf(sm.red_max[0][hh], sm.red_max[1][hh]),
-                                   fmaxf(sm.red_max[2][hh], sm.red_max[3][hh]));
+            const float mx = fmaxf(fmaxf(sm.red_max[grp][0][hh], sm.red_max[grp][1][hh]),
+                                   fmaxf(sm.red_max[grp][2][hh], sm.red_max[grp][3][hh]));
             m_new[h] = fmaxf(m_run[h], mx);
             alpha[h] = m_new[h] == -INFINITY ? 1.0f : exp2f(m_run[h] - m_new[h]);
         }
@@ -466,9 +462,9 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             psum[h] += pv;
         }
         {
-            const int col = warp * 8 + 2 * tq;
-            *reinterpret_cast<float2 *>(sm.p + gq * kAtPStride + col) = make_float2(s[0], s[1]);
-            *reinterpret_cast<float2 *>(sm.p + (gq + 8) * kAtPStride + col) = make_float2(s[2], s[3]);
+            const int col = wq * 8 + 2 * tq;
+            *reinterpret_cast<float2 *>(p_s + gq * kAtPStride + col) = make_float2(s[0], s[1]);
+            *reinterpret_cast<float2 *>(p_s + (gq + 8) * kAtPStride + col) = make_float2(s[2], s[3]);
         }
 #pragma unroll
         for (int h = 0; h < 2; h++) {
@@ -476,20 +472,20 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 2);
         }
         if (tq == 0) {
-            sm.red_sum[warp][gq] = psum[0];
-            sm.red_sum[warp][gq + 8] = psum[1];
+            sm.red_sum[grp][wq][gq] = psum[0];
+            sm.red_sum[grp][wq][gq + 8] = psum[1];
         }
-        __syncthreads();
+        group_sync(grp);
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             const int hh = gq + 8 * h;
-            const float ts = sm.red_sum[0][hh] + sm.red_sum[1][hh] + sm.red_sum[2][hh] +
-                             sm.red_sum[3][hh];
+            const float ts = sm.red_sum[grp][0][hh] + sm.red_sum[grp][1][hh] +
+                             sm.red_sum[grp][2][hh] + sm.red_sum[grp][3][hh];
             l_run[h] = l_run[h] * alpha[h] + ts;
             m_run[h] = m_new[h];
         }
-        // power-of-two normalisation of this tile's block-w row scales
-        const float smax = warp_max(sm.rscale[st][lane][warp]);
+        // power-of-two normalisation of this tile's block-wq row scales
+        const float smax = warp_max(sm.rscale[st][lane][wq]);
         const float pw_new = smax > 0.0f ? fit_pow2(smax, 0) : pw;
         const float rs = pw_new / pw;
         pw = pw_new;
@@ -500,18 +496,16 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             o[i][2] *= alpha[1] * rs;
             o[i][3] *= alpha[1] * rs;
         }
-        const uint32_t v_base = smem_u32(tile) +
-                                (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride +
-                                           warp * 128 + (lane >> 4) * 8) * 2;
 #pragma unroll
         for (int ks = 0; ks < kAtRows / 16; ks++) {
             const int r0k = ks * 16 + 2 * tq;
-            const float2 p00 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k);
-            const float2 p10 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k);
-            const float2 p01 = *reinterpret_cast<const float2 *>(sm.p + gq * kAtPStride + r0k + 8);
-            const float2 p11 = *reinterpret_cast<const float2 *>(sm.p + (gq + 8) * kAtPStride + r0k + 8);
-            const float c0 = sm.rscale[st][r0k][warp] * pw, c1 = sm.rscale[st][r0k + 1][warp] * pw;
-            const float c8 = sm.rscale[st][r0k + 8][warp] * pw, c9 = sm.rscale[st][r0k + 9][warp] * pw;
+            const float2 p00 = *reinterpret_cast<const float2 *>(p_s + gq * kAtPStride + r0k);
+            const float2 p10 = *reinterpret_cast<const float2 *>(p_s + (gq + 8) * kAtPStride + r0k);
+            const float2 p01 = *reinterpret_cast<const float2 *>(p_s + gq * kAtPStride + r0k + 8);
+            const float2 p11 =
+                *reinterpret_cast<const float2 *>(p_s + (gq + 8) * kAtPStride + r0k + 8);
+            const float c0 = sm.rscale[st][r0k][wq] * pw, c1 = sm.rscale[st][r0k + 1][wq] * pw;
+            const float c8 = sm.rscale[st][r0k + 8][wq] * pw, c9 = sm.rscale[st][r0k + 9][wq] * pw;
             uint32_t af[4];
             af[0] = pack_f16(p00.x * c0, p00.y * c1);
             af[1] = pack_f16(p10.x * c0, p10.y * c1);
@@ -526,12 +520,12 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             }
         }
         __syncthreads();   // stage `st` and the tile are free again
-        if (j + 2 < nt) issue_loads(a, sm.tiles[j + 2], st, sm);
+        if (j + 2 < nt) issue_loads8(a, sm.tiles[j + 2], st, sm);
         else cp_async_commit();
     }
 
     const float unpw = 1.0f / pw;
-    const int h0 = g * kAtHeads;
+    const int h0 = hg * kAtHeads;
     if (splits == 1) {
 #pragma unroll
         for (int h = 0; h < 2; h++) {
@@ -541,28 +535,29 @@ sparse_mqa_f16_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
                                   ((int64_t)t * a.heads + h0 + hh) * kLatent;
 #pragma unroll
             for (int n8 = 0; n8 < 16; n8++) {
-                const int col = warp * 128 + n8 * 8 + 2 * tq;
+                const int col = wq * 128 + n8 * 8 + 2 * tq;
                 *reinterpret_cast<uint32_t *>(orow + col) =
                     pack_bf16(o[n8][2 * h] * inv, o[n8][2 * h + 1] * inv);
             }
-            if (a.lse && warp == 0 && tq == 0)
+            if (a.lse && wq == 0 && tq == 0)
                 a.lse[(int64_t)t * a.heads + h0 + hh] =
                     l_run[h] > 0.0f ? (m_run[h] + log2f(l_run[h])) * 0.6931471805599453f
                                     : -INFINITY;
         }
     } else {
-        const int64_t pbase = (((int64_t)t * gridDim.y + g) * splits + sp) * kAtHeads;
+        const int64_t pbase =
+            (((int64_t)t * (a.heads / kAtHeads) + hg) * splits + sp) * kAtHeads;
 #pragma unroll
         for (int h = 0; h < 2; h++) {
             const int hh = gq + 8 * h;
             float *prow = part_o + (pbase + hh) * kLatent;
 #pragma unroll
             for (int n8 = 0; n8 < 16; n8++) {
-                const int col = warp * 128 + n8 * 8 + 2 * tq;
+                const int col = wq * 128 + n8 * 8 + 2 * tq;
                 *reinterpret_cast<float2 *>(prow + col) =
                     make_float2(o[n8][2 * h] * unpw, o[n8][2 * h + 1] * unpw);
             }
-            if (warp == 0 && tq == 0) {
+            if (wq == 0 && tq == 0) {
                 part_ml[(pbase + hh) * 2] = m_run[h];
                 part_ml[(pbase + hh) * 2 + 1] = l_run[h];
             }
@@ -579,7 +574,6 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
     const int t = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
-    const bool fp8 = a.kv_fmt == CSA_FMT_FP8;
     const AtQuery qq = at_query(a, t);
     const int n_rows = kTopK + qq.nw;
     const int tile0 = sp * tiles_per_split;
@@ -636,15 +630,13 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
         __syncthreads();
         const int lt = sm.tiles[j];
         const int32_t *slots = sm.slot + lt * kAtRows;
-        if (fp8) {
-            expand_fp8(lt, st, sm);
-        } else if (tid < kAtRows) {
+        if (tid < kAtRows) {
             const float one = slots[tid] >= 0 ? 1.0f : 0.0f;
             sm.rscale[st][tid][0] = sm.rscale[st][tid][1] = one;
             sm.rscale[st][tid][2] = sm.rscale[st][tid][3] = one;
         }
         __syncthreads();
-        const __nv_bfloat16 *tile = tile_ptr(a.kv_fmt, st, sm);
+        const __nv_bfloat16 *tile = tile_ptr(st, sm);
 
         // S = Q K^T: warp w covers rows 8w..8w+7.  Each 128-channel latent block
         // accumulates separately and is folded in with its row scale.
@@ -860,50 +852,69 @@ sparse_mqa_combine_kernel(const AttnArgs a, int splits, const float *part_o,
 
 static int at_tiles(int window) { return (kTopK + window + kAtRows - 1) / kAtRows; }
 
-static int at_splits(int num_q, int heads, int window, bool decode) {
+// Head groups (of 16) per CTA: the FP8 kernel takes 64 heads at a time when
+// the head count allows, the BF16 kernel one group.
+static int at_groups(int heads, int kv_fmt) {
+    return kv_fmt == CSA_FMT_FP8 && heads % (4 * kAtHeads) == 0 ? 4 : 1;
+}
+
+static int at_splits(int num_q, int heads, int window, bool decode, int groups) {
     if (!decode) return 1;
-    // split each query's rows so that the grid stays within one wave
-    // (2 CTAs per SM on 148 SMs)
-    const int ctas = num_q * (heads / kAtHeads);
-    int sp = (2 * 148) / ctas;
+    // split each query's rows so that the grid fills one wave of the 148 SMs
+    // (two CTAs per SM with one head group, one CTA with four)
+    const int per_sm = groups == 1 ? 2 : 1;
+    const int ctas = num_q * (heads / (kAtHeads * groups));
+    int sp = (per_sm * 148) / ctas;
     sp = sp < 1 ? 1 : sp;
     const int nt = at_tiles(window);
-    sp = sp > 5 ? 5 : sp;
+    sp = sp > 16 ? 16 : sp;
     return sp > nt ? nt : sp;
 }
 
 size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode) {
-    const int sp = at_splits(num_q, heads, window, decode);
+    // the larger of the two formats' needs
+    int sp = at_splits(num_q, heads, window, decode, at_groups(heads, CSA_FMT_BF16));
+    const int sp8 = at_splits(num_q, heads, window, decode, at_groups(heads, CSA_FMT_FP8));
+    sp = sp8 > sp ? sp8 : sp;
     if (sp == 1) return 0;
     return (size_t)num_q * heads * sp * (kLatent + 2) * sizeof(float);
 }
 
+template <int G>
+static cudaError_t launch_fp8(const AttnArgs &a, dim3 grid, int sp, int tps, float *po,
+                              float *pml, cudaStream_t s) {
+    static int done[64] = {0};
+    const size_t smem = sizeof(AtSmem8<G>);
+    cudaError_t e = ensure_max_smem((const void *)sparse_mqa_fp8_kernel<G>, (int)smem, done);
+    if (e != cudaSuccess) return e;
+    sparse_mqa_fp8_kernel<G><<<grid, kAtThreads * G, smem, s>>>(a, sp, tps, po, pml);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s) {
     if (a.num_q == 0) return cudaSuccess;
-    const int sp = at_splits(a.num_q, a.heads, a.window, decode);
+    const int groups = at_groups(a.heads, a.kv_fmt);
+    const int sp = at_splits(a.num_q, a.heads, a.window, decode, groups);
     const int nt = at_tiles(a.window);
     const int tps = (nt + sp - 1) / sp;
-    const int groups = a.heads / kAtHeads;
     float *po = nullptr, *pml = nullptr;
     if (sp > 1) {
         po = (float *)a.workspace;
         pml = po + (size_t)a.num_q * a.heads * sp * kLatent;
     }
-    const size_t smem = sizeof(AtSmem);
-    dim3 grid(a.num_q, groups, sp);
+    dim3 grid(a.num_q, a.heads / (kAtHeads * groups), sp);
     cudaError_t e;
     if (a.kv_fmt == CSA_FMT_FP8) {
-        static int done[64] = {0};
-        e = ensure_max_smem((const void *)sparse_mqa_f16_kernel, (int)smem, done);
-        if (e != cudaSuccess) return e;
-        sparse_mqa_f16_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
+        e = groups == 4 ? launch_fp8<4>(a, grid, sp, tps, po, pml, s)
+                        : launch_fp8<1>(a, grid, sp, tps, po, pml, s);
     } else {
         static int done[64] = {0};
+        const size_t smem = sizeof(AtSmem);
         e = ensure_max_smem((const void *)sparse_mqa_kernel, (int)smem, done);
         if (e != cudaSuccess) return e;
         sparse_mqa_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
+        e = cudaGetLastError();
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess || sp == 1) return e;
     sparse_mqa_combine_kernel<<<a.num_q * a.heads, 128, 0, s>>>(a, sp, po, pml);
     return cudaGetLastError();

@@ -159,7 +159,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         if constexpr (kFp4) {
             // scale-factor layout of 128 rows: row n = m0 + 32*m1 keeps its four
             // block scales of K-step ks at byte ks*512 + m0*16 + m1*4
-            constexpr int nsf = RB / 4;      // block scales per row (Di/16)
+            constexpr int nsf = RB / 8;      // block scales per row (Di/16; a row is Di/2 bytes)
             for (int u = threadIdx.x; u < 128 * G::kKSteps; u += kTcThreads) {
                 const int n = u % 128, ks = u / 128;
                 const int qi = n / p.hi_pad, h = n % p.hi_pad;
@@ -210,7 +210,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             }
             if constexpr (kFp4) {
                 // key m = lane + 32*m1 of the tile; its block scales for K-step ks
-                constexpr int nsf = RB / 4;
+                constexpr int nsf = RB / 8;      // Di/16 block scales per key
                 uint32_t wv[G::kKSteps][4];
 #pragma unroll
                 for (int m1 = 0; m1 < 4; m1++) {
@@ -423,9 +423,14 @@ static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p) {
 
 bool indexer_tc_supported(const IndexerArgs &a) {
     const bool fmt_ok = (a.dim == 64 || a.dim == 128) &&
-                        (a.fmt == CSA_FMT_FP8 || a.fmt == CSA_FMT_BF16);
-    return fmt_ok && a.heads <= 128 && (a.num_slots % kC4Page) == 0 && a.num_slots >= kC4Page &&
-           (reinterpret_cast<uintptr_t>(a.k_codes) % 16) == 0 && encode_fn() != nullptr;
+                        (a.fmt == CSA_FMT_FP8 || a.fmt == CSA_FMT_BF16 || a.fmt == CSA_FMT_FP4);
+    // FP4 block scales are gathered four at a time (32-bit loads)
+    const bool sf_ok = a.fmt != CSA_FMT_FP4 ||
+                       ((reinterpret_cast<uintptr_t>(a.k_block_scales) % 4) == 0 &&
+                        (reinterpret_cast<uintptr_t>(a.q_block_scales) % 4) == 0);
+    return fmt_ok && sf_ok && a.heads <= 128 && (a.num_slots % kC4Page) == 0 &&
+           a.num_slots >= kC4Page && (reinterpret_cast<uintptr_t>(a.k_codes) % 16) == 0 &&
+           encode_fn() != nullptr;
 }
 
 cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
