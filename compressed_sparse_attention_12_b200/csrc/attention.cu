@@ -302,6 +302,7 @@ template <int G>
 __global__ void __launch_bounds__(kAtThreads * G, G == 1 ? 2 : 1)
 sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part_o,
                       float *part_ml) {
+    pdl_begin();
     constexpr int kThr = kAtThreads * G;
     extern __shared__ __align__(16) uint8_t at_smem_raw[];
     AtSmem8<G> &sm = *reinterpret_cast<AtSmem8<G> *>(at_smem_raw);
@@ -569,6 +570,7 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
 __global__ void __launch_bounds__(kAtThreads, 2)
 sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part_o,
                   float *part_ml) {
+    pdl_begin();
     extern __shared__ __align__(16) uint8_t at_smem_raw[];
     AtSmem &sm = *reinterpret_cast<AtSmem *>(at_smem_raw);
     const int t = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
@@ -811,33 +813,52 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
 
 // Merge the splits of one (query, head): grid num_q * heads, 128 threads,
 // four output columns per thread.
+// Merges the split partials of one (query, head): every split's (max, sum)
+// and 4-column slice are loaded before any is used (one memory round trip).
+constexpr int kAtMaxSplits = 16;
+
+template <int MAXSP>
 __global__ void __launch_bounds__(128)
 sparse_mqa_combine_kernel(const AttnArgs a, int splits, const float *part_o,
                           const float *part_ml) {
+    pdl_begin();
     const int t = blockIdx.x / a.heads, head = blockIdx.x % a.heads;
     const int g = head / kAtHeads, hh = head % kAtHeads;
     const int groups = a.heads / kAtHeads;
     const int64_t base = ((int64_t)t * groups + g) * splits;
-    float M = -INFINITY;
-    for (int sp = 0; sp < splits; sp++) {
-        const int64_t r = (base + sp) * kAtHeads + hh;
-        if (part_ml[r * 2 + 1] > 0.0f) M = fmaxf(M, part_ml[r * 2]);
+    const int c = threadIdx.x * 4;
+    float m[MAXSP], l[MAXSP];
+    float4 v[MAXSP];
+#pragma unroll
+    for (int sp = 0; sp < MAXSP; sp++) {
+        if (sp < splits) {
+            const int64_t r = (base + sp) * kAtHeads + hh;
+            const float2 ml = *reinterpret_cast<const float2 *>(part_ml + r * 2);
+            m[sp] = ml.x;
+            l[sp] = ml.y;
+            v[sp] = *reinterpret_cast<const float4 *>(part_o + r * kLatent + c);
+        } else {
+            m[sp] = -INFINITY;
+            l[sp] = 0.0f;
+            v[sp] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < MAXSP; sp++)
+        if (l[sp] > 0.0f) M = fmaxf(M, m[sp]);
     float L = 0.0f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int c = threadIdx.x * 4;
     if (M != -INFINITY) {
-        for (int sp = 0; sp < splits; sp++) {
-            const int64_t r = (base + sp) * kAtHeads + hh;
-            const float l = part_ml[r * 2 + 1];
-            if (!(l > 0.0f)) continue;
-            const float w = exp2f(part_ml[r * 2] - M);
-            L += l * w;
-            const float4 v = *reinterpret_cast<const float4 *>(part_o + r * kLatent + c);
-            acc.x += v.x * w;
-            acc.y += v.y * w;
-            acc.z += v.z * w;
-            acc.w += v.w * w;
+#pragma unroll
+        for (int sp = 0; sp < MAXSP; sp++) {
+            if (!(l[sp] > 0.0f)) continue;
+            const float w = exp2f(m[sp] - M);
+            L += l[sp] * w;
+            acc.x += v[sp].x * w;
+            acc.y += v[sp].y * w;
+            acc.z += v[sp].z * w;
+            acc.w += v[sp].w * w;
         }
     }
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
@@ -867,7 +888,7 @@ static int at_splits(int num_q, int heads, int window, bool decode, int groups) 
     int sp = (per_sm * 148) / ctas;
     sp = sp < 1 ? 1 : sp;
     const int nt = at_tiles(window);
-    sp = sp > 16 ? 16 : sp;
+    sp = sp > kAtMaxSplits ? kAtMaxSplits : sp;
     return sp > nt ? nt : sp;
 }
 
@@ -887,7 +908,7 @@ static cudaError_t launch_fp8(const AttnArgs &a, dim3 grid, int sp, int tps, flo
     const size_t smem = sizeof(AtSmem8<G>);
     cudaError_t e = ensure_max_smem((const void *)sparse_mqa_fp8_kernel<G>, (int)smem, done);
     if (e != cudaSuccess) return e;
-    sparse_mqa_fp8_kernel<G><<<grid, kAtThreads * G, smem, s>>>(a, sp, tps, po, pml);
+    launch_k(sparse_mqa_fp8_kernel<G>, grid, kAtThreads * G, smem, s, a, sp, tps, po, pml);
     return cudaGetLastError();
 }
 
@@ -912,11 +933,13 @@ cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s) {
         const size_t smem = sizeof(AtSmem);
         e = ensure_max_smem((const void *)sparse_mqa_kernel, (int)smem, done);
         if (e != cudaSuccess) return e;
-        sparse_mqa_kernel<<<grid, kAtThreads, smem, s>>>(a, sp, tps, po, pml);
+        launch_k(sparse_mqa_kernel, grid, kAtThreads, smem, s, a, sp, tps, po, pml);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess || sp == 1) return e;
-    sparse_mqa_combine_kernel<<<a.num_q * a.heads, 128, 0, s>>>(a, sp, po, pml);
+    if (sp <= 4) launch_k(sparse_mqa_combine_kernel<4>, a.num_q * a.heads, 128, 0, s, a, sp, po, pml);
+    else if (sp <= 8) launch_k(sparse_mqa_combine_kernel<8>, a.num_q * a.heads, 128, 0, s, a, sp, po, pml);
+    else launch_k(sparse_mqa_combine_kernel<16>, a.num_q * a.heads, 128, 0, s, a, sp, po, pml);
     return cudaGetLastError();
 }
 

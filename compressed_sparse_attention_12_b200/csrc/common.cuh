@@ -24,6 +24,17 @@ constexpr int kFp8RowBytes = 656;
 constexpr int kBf16RowBytes = 1152;
 
 // First recorded device-side problem wins; later ones are dropped.
+// Programmatic dependent launch.  Every kernel starts with this: it lets the
+// next kernel on the stream be scheduled at once (its blocks become resident
+// as resources free up and wait here in turn), then waits until the kernels
+// this one depends on have completed and their writes are visible.  Nothing
+// global is read before the wait.  Both instructions are no-ops when the
+// kernel was launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void report(int32_t *status, int32_t code) {
     if (status) atomicCAS(status, 0, code);
 }

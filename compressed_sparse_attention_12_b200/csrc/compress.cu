@@ -59,6 +59,7 @@ __device__ __forceinline__ bool kv_active(int warp, int lane) { return warp < 4 
 __global__ void __launch_bounds__(kKvRowThreads)
 kv_store_kernel(const float *__restrict__ rows, int64_t n, const int32_t *__restrict__ slots,
                 int fmt, uint8_t *__restrict__ cache, int64_t num_slots, int32_t *status) {
+    pdl_begin();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_bytes = fmt == CSA_FMT_FP8 ? kFp8RowBytes : kBf16RowBytes;
     for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
@@ -148,6 +149,7 @@ hadamard_quant_kernel(const T *__restrict__ x, int64_t rows, int fmt,
                       const int32_t *__restrict__ row_map, int64_t num_out_rows,
                       uint8_t *codes, uint8_t *block_scales, float *scales,
                       const float *__restrict__ w_in, float *w_out, int32_t *status) {
+    pdl_begin();
     constexpr int D = 32 * E;
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -237,6 +239,7 @@ compress_kv_kernel(const float *__restrict__ x, const float *__restrict__ gate,
                    const float *__restrict__ bias, const int32_t *cu_x,
                    const int32_t *start_pos, int max_rows, const int32_t *page_table,
                    int pt_stride, int fmt, uint8_t *out, int64_t num_slots, int32_t *status) {
+    pdl_begin();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t j = 0;
     const int64_t row0 = compress_row(blockIdx.y, blockIdx.x, cu_x, start_pos, max_rows, status,
@@ -281,6 +284,7 @@ compress_index_kernel(const float *__restrict__ x, const float *__restrict__ gat
                       const int32_t *start_pos, int max_rows, const int32_t *page_table,
                       int pt_stride, int fmt, uint8_t *codes, uint8_t *block_scales,
                       float *scales, int64_t num_slots, int32_t *status) {
+    pdl_begin();
     constexpr int D = 32 * E;
     const int lane = threadIdx.x & 31;
     const int blk = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -314,7 +318,7 @@ cudaError_t launch_kv_store(const float *rows, int64_t n, const int32_t *slots, 
                             void *cache, int64_t num_slots, int32_t *status, cudaStream_t s) {
     if (n == 0) return cudaSuccess;
     const int grid = (int)(n < 65535 * 8 ? n : 65535 * 8);
-    kv_store_kernel<<<grid, kKvRowThreads, 0, s>>>(rows, n, slots, fmt, (uint8_t *)cache,
+    launch_k(kv_store_kernel, grid, kKvRowThreads, 0, s, rows, n, slots, fmt, (uint8_t *)cache,
                                                    num_slots, status);
     return cudaGetLastError();
 }
@@ -327,7 +331,7 @@ cudaError_t launch_hadamard_quant(const void *x, int x_dtype, int64_t rows, int 
     const unsigned grid = (unsigned)((rows + 7) / 8);
     uint8_t *c = (uint8_t *)codes;
 #define CSA_HQ(E, T)                                                                        \
-    hadamard_quant_kernel<E, T><<<grid, 256, 0, s>>>((const T *)x, rows, fmt, row_map,      \
+    launch_k(hadamard_quant_kernel<E, T>, grid, 256, 0, s, (const T *)x, rows, fmt, row_map,      \
                                                      num_out_rows, c, block_scales, scales, \
                                                      w_in, w_out, status)
     if (dim == 64 && x_dtype == CSA_FMT_BF16) CSA_HQ(2, uint16_t);
@@ -349,7 +353,7 @@ cudaError_t launch_c4_compress(const float *x, const float *gate, const float *b
     if (out_kind == CSA_OUT_KV_BF16 || out_kind == CSA_OUT_KV_FP8) {
         const int fmt = out_kind == CSA_OUT_KV_FP8 ? CSA_FMT_FP8 : CSA_FMT_BF16;
         dim3 grid(max_blocks, bs);
-        compress_kv_kernel<<<grid, kKvRowThreads, 0, s>>>(x, gate, bias, cu_x, start_pos,
+        launch_k(compress_kv_kernel, grid, kKvRowThreads, 0, s, x, gate, bias, cu_x, start_pos,
                                                           max_rows, page_table, pt_stride, fmt,
                                                           (uint8_t *)out, num_slots, status);
     } else {
@@ -358,11 +362,11 @@ cudaError_t launch_c4_compress(const float *x, const float *gate, const float *b
                                                         : CSA_FMT_BF16;
         dim3 grid((max_blocks + 7) / 8, bs);
         if (dim == 64)
-            compress_index_kernel<2><<<grid, 256, 0, s>>>(
+            launch_k(compress_index_kernel<2>, grid, 256, 0, s, 
                 x, gate, bias, cu_x, start_pos, max_rows, page_table, pt_stride, fmt,
                 (uint8_t *)out, out_block_scales, out_scales, num_slots, status);
         else
-            compress_index_kernel<4><<<grid, 256, 0, s>>>(
+            launch_k(compress_index_kernel<4>, grid, 256, 0, s, 
                 x, gate, bias, cu_x, start_pos, max_rows, page_table, pt_stride, fmt,
                 (uint8_t *)out, out_block_scales, out_scales, num_slots, status);
     }

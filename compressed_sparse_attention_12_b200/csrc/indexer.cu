@@ -77,6 +77,7 @@ __device__ __forceinline__ void load_key(const uint8_t *codes_row, const uint8_t
 template <int FMT, int DIM>
 __global__ void __launch_bounds__(kIdxThreads)
 indexer_simple_kernel(const IndexerArgs a) {
+    pdl_begin();
     extern __shared__ float q_smem[];  // [heads][DIM] then w'[heads]
     constexpr int CB = FMT == CSA_FMT_BF16 ? 2 * DIM : FMT == CSA_FMT_FP8 ? DIM : DIM / 2;
     const int t = blockIdx.y;
@@ -141,7 +142,7 @@ cudaError_t launch_indexer(const IndexerArgs &a, cudaStream_t s) {
         cudaError_t e = ensure_max_smem((const void *)indexer_simple_kernel<F, D>,       \
                                         128 * (D + 1) * 4, done);                        \
         if (e != cudaSuccess) return e;                                                  \
-        indexer_simple_kernel<F, D><<<grid, kIdxThreads, smem, s>>>(a);                  \
+        launch_k(indexer_simple_kernel<F, D>, grid, kIdxThreads, smem, s, a);                  \
     } while (0)
     if (a.fmt == CSA_FMT_BF16 && a.dim == 64) CSA_IDX(CSA_FMT_BF16, 64);
     else if (a.fmt == CSA_FMT_BF16) CSA_IDX(CSA_FMT_BF16, 128);

@@ -57,6 +57,7 @@ template <int FMT, int RB>
 __global__ void __launch_bounds__(kTcThreads, 2)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                   const TcParams p) {
+    pdl_begin();
     using G = TcGeom<RB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned carve-up: stages | q tile | w' | nv | barriers
@@ -486,7 +487,7 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
         static int done[64] = {0};                                                          \
         cudaError_t e = ensure_max_smem((const void *)indexer_tc_kernel<F, R>, 200 * 1024, done); \
         if (e != cudaSuccess) return e;                                                     \
-        indexer_tc_kernel<F, R><<<grid, kTcThreads, smem, s>>>(a, map, p);                  \
+        launch_k(indexer_tc_kernel<F, R>, grid, kTcThreads, smem, s, a, map, p);                  \
     } while (0)
     if (a.fmt == CSA_FMT_FP8 && rb == 128) CSA_TC(CSA_FMT_FP8, 128);
     else if (a.fmt == CSA_FMT_FP8) CSA_TC(CSA_FMT_FP8, 64);

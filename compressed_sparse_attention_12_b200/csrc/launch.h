@@ -7,6 +7,26 @@
 
 namespace csa {
 
+// Launches `kernel` on stream s with programmatic stream serialization, so it
+// may be scheduled while the previous kernel on the stream is finishing; the
+// kernel itself waits for its predecessors (pdl_begin) before reading global
+// memory.  Captured into CUDA graphs as a programmatic edge.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // Raises a kernel's dynamic shared-memory limit once per device (the call is
 // not a stream operation, so it is kept out of CUDA-graph captures after the
 // first eager launch).  `done` is a per-kernel table indexed by device.

@@ -73,55 +73,78 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total,
     return before + incl - v;
 }
 
-// Finds the K-th largest key T among keys[0..n) (K <= n) and how many keys
-// equal to T belong to the top K (need_eq >= 1).  keys may point to shared
-// or global memory.
-__device__ void radix_threshold(const uint32_t *keys, int n, int K, TkShared &sh,
-                                uint32_t *T_out, int *need_eq_out) {
-    const int shifts[3] = {20, 8, 0};
-    const int widths[3] = {12, 12, 8};
-    uint32_t prefix = 0;
+// Block-wide min and max of one value pair per thread (uses sh.warp_a/b).
+__device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, TkShared &sh) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+        sh.warp_a[warp] = lo;
+        sh.warp_b[warp] = hi;
+    }
+    __syncthreads();
+    lo = 0xffffffffu;
+    hi = 0u;
+#pragma unroll
+    for (int w = 0; w < kTkWarps; w++) {
+        lo = min(lo, sh.warp_a[w]);
+        hi = max(hi, sh.warp_b[w]);
+    }
+    __syncthreads();
+}
+
+// Finds the K-th largest key T among the keys[0..n) that are >= kmin (K <= their
+// count; kmax is their maximum) and how many keys equal to T belong to the top K
+// (need_eq >= 1).  The radix digits are taken from d = key - kmin, 12 bits at a
+// time from the highest set bit of kmax - kmin down, so that keys sharing sign
+// and exponent (the usual case for one row of logits) already spread over the
+// bins of the first pass; two passes resolve a range of up to 24 bits.  keys may
+// point to shared or global memory.
+__device__ void radix_threshold(const uint32_t *keys, int n, int K, uint32_t kmin, uint32_t kmax,
+                                TkShared &sh, uint32_t *T_out, int *need_eq_out) {
+    const uint32_t range = kmax - kmin;
+    const int B = range == 0 ? 0 : 32 - __clz(range);
+    uint32_t prefix = 0;            // resolved high bits of d
     int remaining = K;
 #pragma unroll 1
-    for (int p = 0; p < 3; p++) {
-        const int shift = shifts[p], bits = widths[p];
-        const uint32_t nb = 1u << bits;
-        const uint64_t hi_mask64 = ~((1ull << (shift + bits)) - 1ull);
-        const uint32_t hi_mask = (uint32_t)hi_mask64;
+    for (int done = 0; done < B;) {
+        const int width = min(12, B - done);
+        const int shift = B - done - width;
+        const int hi = shift + width;            // bits at and above hi are resolved
+        const uint32_t nb = 1u << width;
         for (uint32_t i = threadIdx.x; i < nb; i += kTkThreads) sh.hist[i] = 0;
         __syncthreads();
         for (int i = threadIdx.x; i < n; i += kTkThreads) {
             const uint32_t k = keys[i];
-            if ((k & hi_mask) == (prefix & hi_mask))
-                atomicAdd(&sh.hist[(k >> shift) & (nb - 1)], 1u);
+            const uint32_t d = k - kmin;
+            const bool match = k >= kmin && (hi >= 32 || ((d ^ prefix) >> hi) == 0);
+            if (match) atomicAdd(&sh.hist[(d >> shift) & (nb - 1)], 1u);
         }
         __syncthreads();
-        // Suffix scan from the top bin: thread i owns bins nb-1-8i .. nb-8-8i.
-        const int per = (int)nb / kTkThreads;  // 8 (4096 bins) or 0 (256 bins)
-        uint32_t mine = 0;
+        // Suffix scan from the top bin: thread i owns bins nb-1-per*i .. nb-per*(i+1).
+        const int per = nb > (uint32_t)kTkThreads ? (int)nb / kTkThreads : 1;   // 1..8
         uint32_t c[8];
-        if (per == 8) {
+        uint32_t mine = 0;
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                c[j] = sh.hist[nb - 1 - (threadIdx.x * 8 + j)];
-                mine += c[j];
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; j++) c[j] = 0;
-            if (threadIdx.x < nb) c[0] = sh.hist[nb - 1 - threadIdx.x];
-            mine = c[0];
+        for (int j = 0; j < 8; j++) {
+            const int bin = (int)nb - 1 - ((int)threadIdx.x * per + j);
+            c[j] = (j < per && bin >= 0) ? sh.hist[bin] : 0u;
+            mine += c[j];
         }
         uint32_t total;
         const uint32_t excl = block_excl_scan(mine, &total, sh);
         if (excl < (uint32_t)remaining && (uint32_t)remaining <= excl + mine) {
             uint32_t acc = excl;
-            const int cnt = per == 8 ? 8 : 1;
-            for (int j = 0; j < cnt; j++) {
-                if (acc + c[j] >= (uint32_t)remaining) {
-                    sh.digit = per == 8 ? nb - 1 - (threadIdx.x * 8 + j) : nb - 1 - threadIdx.x;
+            bool found = false;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                if (!found && j < per && acc + c[j] >= (uint32_t)remaining) {
+                    found = true;
+                    sh.digit = nb - 1 - (threadIdx.x * per + j);
                     sh.above = acc;
-                    break;
                 }
                 acc += c[j];
             }
@@ -129,21 +152,22 @@ __device__ void radix_threshold(const uint32_t *keys, int n, int K, TkShared &sh
         __syncthreads();
         prefix |= sh.digit << shift;
         remaining -= (int)sh.above;
+        done += width;
         __syncthreads();
     }
-    *T_out = prefix;
+    *T_out = kmin + prefix;
     *need_eq_out = remaining;
 }
 
 // Walks keys[0..n) in index order and calls emit(pos, i, key) for the
 // selected ones: key > T, or key == T among the first need_eq such keys.
+// Returns how many were selected.
 // Each warp owns one contiguous segment: it counts its segment with ballots,
 // one block barrier publishes the per-warp counts, then every warp writes its
 // selected elements at their global ranks.
 template <typename Emit>
-__device__ void ordered_compact(const uint32_t *keys, int n, uint32_t T, int need_eq, int K,
-                                TkShared &sh, Emit emit) {
-    (void)K;
+__device__ int ordered_compact(const uint32_t *keys, int n, uint32_t T, int need_eq,
+                               TkShared &sh, Emit emit) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = (1u << lane) - 1u;
     const int seg = ((n + kTkWarps - 1) / kTkWarps + 31) & ~31;
@@ -159,10 +183,12 @@ __device__ void ordered_compact(const uint32_t *keys, int n, uint32_t T, int nee
         sh.warp_b[warp] = gt_w;
     }
     __syncthreads();
-    uint32_t eq_before = 0, gt_before = 0;
-    for (int w = 0; w < warp; w++) {
-        eq_before += sh.warp_a[w];
-        gt_before += sh.warp_b[w];
+    uint32_t eq_before = 0, gt_before = 0, eq_all = 0, gt_all = 0;
+    for (int w = 0; w < kTkWarps; w++) {
+        eq_before += w < warp ? sh.warp_a[w] : 0u;
+        gt_before += w < warp ? sh.warp_b[w] : 0u;
+        eq_all += sh.warp_a[w];
+        gt_all += sh.warp_b[w];
     }
     __syncthreads();    // the counts may be reused by the caller's next phase
     uint32_t eq_seen = eq_before;
@@ -178,6 +204,7 @@ __device__ void ordered_compact(const uint32_t *keys, int n, uint32_t T, int nee
         eq_seen += __popc(beq);
         out += __popc(btk);
     }
+    return (int)(gt_all + min(eq_all, (uint32_t)need_eq));
 }
 
 struct RowInfo {
@@ -226,11 +253,15 @@ __device__ RowInfo row_info(int t, const int32_t *cu_q, int bs, const int32_t *q
     return r;
 }
 
+// Stage 1: one CTA per (query row, 8192-logit chunk).  Writes the chunk's
+// top-512 (or all of it when shorter) in index order, plus the chunk's
+// 512th-largest key (0 when it holds fewer) and its largest key.
 __global__ void __launch_bounds__(kTkThreads)
 topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens,
                    int bs, const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
                    int pt_stride, int max_chunks, uint32_t *cand_key, int32_t *cand_idx,
-                   int32_t *status) {
+                   uint2 *chunk_info, int32_t *status) {
+    pdl_begin();
     extern __shared__ __align__(16) uint8_t tk_smem[];
     TkShared &sh = *reinterpret_cast<TkShared *>(tk_smem);
     uint32_t *skeys = reinterpret_cast<uint32_t *>(tk_smem + kTkKeysOffset);
@@ -241,79 +272,138 @@ topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32
     if (lo >= ri.n_vis) return;
     const int len = min(kTkChunk, ri.n_vis - lo);
     const float *row = logits + (int64_t)t * stride + lo;
+    uint32_t kmax = 0u;
+    bool has = false;
+    auto put = [&](int i, float f) {
+        const uint32_t k = order_key(f, status);
+        skeys[i] = k;
+        kmax = max(kmax, k);
+        has = true;
+    };
     if ((reinterpret_cast<uintptr_t>(row) & 15) == 0) {
         const int n4 = len / 4;
         for (int i = threadIdx.x; i < n4; i += kTkThreads) {
             const float4 v = reinterpret_cast<const float4 *>(row)[i];
-            skeys[4 * i] = order_key(v.x, status);
-            skeys[4 * i + 1] = order_key(v.y, status);
-            skeys[4 * i + 2] = order_key(v.z, status);
-            skeys[4 * i + 3] = order_key(v.w, status);
+            put(4 * i, v.x);
+            put(4 * i + 1, v.y);
+            put(4 * i + 2, v.z);
+            put(4 * i + 3, v.w);
         }
-        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTkThreads) skeys[i] = order_key(row[i], status);
+        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTkThreads) put(i, row[i]);
     } else {
-        for (int i = threadIdx.x; i < len; i += kTkThreads) skeys[i] = order_key(row[i], status);
+        for (int i = threadIdx.x; i < len; i += kTkThreads) put(i, row[i]);
     }
-    __syncthreads();
+    // The keys each thread loaded form one group.  When all 512 groups are
+    // non-empty the smallest group maximum is a lower bound of the 512th-largest
+    // key (the 512 group maxima are distinct keys >= it); otherwise the bound
+    // is 0.
+    uint32_t lbound = has ? kmax : 0u;
+    block_minmax(lbound, kmax, sh);     // its barrier also publishes skeys
     const int K = min(kTopK, len);
     uint32_t T = 0;
     int need_eq = len;
-    if (len > kTopK) radix_threshold(skeys, len, K, sh, &T, &need_eq);
+    if (len > kTopK) radix_threshold(skeys, len, K, lbound, kmax, sh, &T, &need_eq);
+    if (threadIdx.x == 0)
+        chunk_info[(int64_t)t * max_chunks + c] = make_uint2(len > kTopK ? T : 0u, kmax);
     uint32_t *ok = cand_key + ((int64_t)t * max_chunks + c) * kTopK;
     int32_t *oi = cand_idx + ((int64_t)t * max_chunks + c) * kTopK;
-    ordered_compact(skeys, len, T, need_eq, K, sh, [&](int pos, int i, uint32_t k) {
+    ordered_compact(skeys, len, T, need_eq, sh, [&](int pos, int i, uint32_t k) {
         ok[pos] = k;
         oi[pos] = lo + i;
     });
 }
 
+// Stage 2: one CTA per query row.  The row's top-512 are all >= L, the largest
+// of the chunks' 512th keys (that chunk alone holds 512 keys >= L), so the
+// candidates below L are dropped first (in index order, into shared memory),
+// the threshold is found among the survivors, and the selection is written in
+// ascending index order, mapped through the page table, then padded with -1.
+// Rows with more than 16384 candidates select straight from the workspace.
 __global__ void __launch_bounds__(kTkThreads)
 topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const int32_t *q_pos,
                    int max_c4_len, const int32_t *page_table, int pt_stride, int64_t num_slots,
                    int max_chunks, const uint32_t *cand_key, const int32_t *cand_idx,
-                   int32_t *out_phys, int32_t *out_raw, int32_t *status) {
+                   const uint2 *chunk_info, int32_t *out_phys, int32_t *out_raw,
+                   int32_t *status) {
+    pdl_begin();
     extern __shared__ __align__(16) uint8_t tk2_smem[];
     TkShared &sh = *reinterpret_cast<TkShared *>(tk2_smem);
     uint32_t *skeys = reinterpret_cast<uint32_t *>(tk2_smem + kTkKeysOffset);
+    int32_t *sidx = reinterpret_cast<int32_t *>(skeys + kTk2Smem);
     const int t = blockIdx.x;
     const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
                                 false, sh);
     const int n = ri.n_vis;
-    int total = 0;
+    int total = 0, nch = 0;
     if (n > 0) {
-        const int nch = (n + kTkChunk - 1) / kTkChunk;
+        nch = (n + kTkChunk - 1) / kTkChunk;
         total = (nch - 1) * kTopK + min(kTopK, n - (nch - 1) * kTkChunk);
     }
     const int K = min(kTopK, total);
-    const uint32_t *gkeys = cand_key + (int64_t)t * max_chunks * kTopK;
+    const uint32_t *keys = cand_key + (int64_t)t * max_chunks * kTopK;
     const int32_t *idx = cand_idx + (int64_t)t * max_chunks * kTopK;
-    // candidates (keys and indices) up to kTk2Smem keys are staged in shared memory; longer rows
-    // are selected straight from the workspace (L2)
-    const uint32_t *keys = gkeys;
-    int32_t *sidx = reinterpret_cast<int32_t *>(skeys + kTk2Smem);
-    if (total <= kTk2Smem) {
-        for (int i = threadIdx.x * 4; i < total; i += kTkThreads * 4) {
-            if (i + 4 <= total) {
-                *reinterpret_cast<uint4 *>(skeys + i) = *reinterpret_cast<const uint4 *>(gkeys + i);
-                *reinterpret_cast<int4 *>(sidx + i) = *reinterpret_cast<const int4 *>(idx + i);
-            } else {
-                for (int j = i; j < total; j++) {
-                    skeys[j] = gkeys[j];
-                    sidx[j] = idx[j];
-                }
-            }
-        }
-        __syncthreads();
-        keys = skeys;
-        idx = sidx;
-    }
-    const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
     uint32_t T = 0;
     int need_eq = total;
-    if (total > kTopK) radix_threshold(keys, total, K, sh, &T, &need_eq);
+    int m = total;
+    if (total > kTopK) {
+        uint32_t L = 0, kmax = 0;
+        for (int c = threadIdx.x; c < nch; c += kTkThreads) {
+            const uint2 ci = chunk_info[(int64_t)t * max_chunks + c];
+            L = max(L, ci.x);
+            kmax = max(kmax, ci.y);
+        }
+        uint32_t lneg = ~L;
+        block_minmax(lneg, kmax, sh);     // min of ~L is ~(max of L)
+        L = ~lneg;
+        if (total <= kTk2Smem) {
+            // Thread i holds candidates [32i, 32i+32): all loads in flight at
+            // once, then the survivors (keys >= L) are compacted in order into
+            // shared memory with one block scan.
+            constexpr int kPer = kTk2Smem / kTkThreads;    // 32
+            static_assert(kPer % 4 == 0, "16-byte loads");
+            const int i0 = threadIdx.x * kPer;
+            uint32_t kk[kPer];
+            int32_t ii[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; j += 4) {
+                const int i = i0 + j;
+                if (i + 4 <= total) {
+                    const uint4 k4 = *reinterpret_cast<const uint4 *>(keys + i);
+                    const int4 x4 = *reinterpret_cast<const int4 *>(idx + i);
+                    kk[j] = k4.x; kk[j + 1] = k4.y; kk[j + 2] = k4.z; kk[j + 3] = k4.w;
+                    ii[j] = x4.x; ii[j + 1] = x4.y; ii[j + 2] = x4.z; ii[j + 3] = x4.w;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        kk[j + q] = i + q < total ? keys[i + q] : 0u;
+                        ii[j + q] = i + q < total ? idx[i + q] : 0;
+                    }
+                }
+            }
+            uint32_t mine = 0;
+#pragma unroll
+            for (int j = 0; j < kPer; j++) mine += (i0 + j < total && kk[j] >= L) ? 1u : 0u;
+            uint32_t surv;
+            uint32_t pos = block_excl_scan(mine, &surv, sh);
+#pragma unroll
+            for (int j = 0; j < kPer; j++) {
+                if (i0 + j < total && kk[j] >= L) {
+                    skeys[pos] = kk[j];
+                    sidx[pos] = ii[j];
+                    pos++;
+                }
+            }
+            __syncthreads();
+            keys = skeys;
+            idx = sidx;
+            m = (int)surv;
+        }
+        radix_threshold(keys, m, K, L, kmax, sh, &T, &need_eq);
+    }
+    const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
     int32_t *op = out_phys + (int64_t)t * kTopK;
     int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
-    ordered_compact(keys, total, T, need_eq, K, sh, [&](int pos, int i, uint32_t) {
+    ordered_compact(keys, m, T, need_eq, sh, [&](int pos, int i, uint32_t) {
         const int32_t s = idx[i];
         const int32_t page = pt_row[s / kC4Page];
         const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
@@ -335,8 +425,11 @@ static int topk_max_chunks(int max_c4_len) {
     return max_c4_len <= 0 ? 1 : (max_c4_len + kTkChunk - 1) / kTkChunk;
 }
 
+// Workspace: candidate keys, candidate indices (num_q x chunks x 512 each),
+// then one (512th key, largest key) pair per chunk.
 size_t topk_workspace_bytes(int num_q, int max_c4_len) {
-    return (size_t)num_q * topk_max_chunks(max_c4_len) * kTopK * 8;
+    const size_t chunks = (size_t)num_q * topk_max_chunks(max_c4_len);
+    return chunks * kTopK * 8 + chunks * sizeof(uint2);
 }
 
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
@@ -344,24 +437,25 @@ cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
     const int mc = topk_max_chunks(a.max_c4_len);
     uint32_t *ck = (uint32_t *)a.workspace;
     int32_t *ci = (int32_t *)((uint8_t *)a.workspace + (size_t)a.num_q * mc * kTopK * 4);
+    uint2 *info = (uint2 *)((uint8_t *)a.workspace + (size_t)a.num_q * mc * kTopK * 8);
     const size_t smem1 = kTkKeysOffset + kTkChunk * sizeof(uint32_t);
     static int done[64] = {0};
     cudaError_t e0 = ensure_max_smem((const void *)topk_stage1_kernel, (int)smem1, done);
     if (e0 != cudaSuccess) return e0;
     dim3 g1(mc, a.num_q);
-    topk_stage1_kernel<<<g1, kTkThreads, smem1, s>>>(a.logits, a.logits_stride, a.c4_seq_lens, a.bs,
+    launch_k(topk_stage1_kernel, g1, kTkThreads, smem1, s, a.logits, a.logits_stride, a.c4_seq_lens, a.bs,
                                                  a.cu_q, a.q_pos, a.max_c4_len, a.pt_stride, mc,
-                                                 ck, ci, a.status);
+                                                 ck, ci, info, a.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem2 = kTkKeysOffset + kTk2Smem * (sizeof(uint32_t) + sizeof(int32_t));
     static int done2[64] = {0};
     e = ensure_max_smem((const void *)topk_stage2_kernel, (int)smem2, done2);
     if (e != cudaSuccess) return e;
-    topk_stage2_kernel<<<a.num_q, kTkThreads, smem2, s>>>(a.c4_seq_lens, a.bs, a.cu_q, a.q_pos,
+    launch_k(topk_stage2_kernel, a.num_q, kTkThreads, smem2, s, a.c4_seq_lens, a.bs, a.cu_q, a.q_pos,
                                                       a.max_c4_len, a.page_table, a.pt_stride,
-                                                      a.num_slots, mc, ck, ci, a.out_phys,
-                                                      a.out_raw, a.status);
+                                                      a.num_slots, mc, ck, ci, info,
+                                                      a.out_phys, a.out_raw, a.status);
     return cudaGetLastError();
 }
 

@@ -48,10 +48,11 @@ def test_status_strings_and_constants(L):
 def test_workspace_sizes(L):
     from compressed_sparse_attention_12_b200 import csa
     assert csa.csa_topk512_workspace_size(0, 100) == 0
-    # one chunk of 8192 candidates per row, (key, index) pairs of 512
-    assert csa.csa_topk512_workspace_size(3, 8192) == 3 * 1 * 512 * 8
-    assert csa.csa_topk512_workspace_size(3, 8193) == 3 * 2 * 512 * 8
-    assert csa.csa_topk512_workspace_size(8, 262144) == 8 * 32 * 512 * 8
+    # per row and 8192-logit chunk: 512 (key, index) candidate pairs and one
+    # (512th key, largest key) pair
+    assert csa.csa_topk512_workspace_size(3, 8192) == 3 * 1 * (512 * 8 + 8)
+    assert csa.csa_topk512_workspace_size(3, 8193) == 3 * 2 * (512 * 8 + 8)
+    assert csa.csa_topk512_workspace_size(8, 262144) == 8 * 32 * (512 * 8 + 8)
     assert csa.csa_sparse_mqa_workspace_size(4096, 64, 128, 0) == 0
     assert csa.csa_sparse_mqa_workspace_size(32, 64, 128, 1) > 0
 
