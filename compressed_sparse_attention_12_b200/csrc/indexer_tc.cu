@@ -51,7 +51,10 @@ struct TcParams {
     int tiles_per_cta;
     int stages;
     int num_pages;
+    int nacc;          // TMEM accumulators in flight (power of two, >= 2)
 };
+
+constexpr int kKsRing = 8;     // key-scale tiles in flight per epilogue group
 
 template <int FMT, int RB>
 __global__ void __launch_bounds__(kTcThreads, 2)
@@ -72,10 +75,13 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     int *nv_s = reinterpret_cast<int *>(w_s + 256);
     uint64_t *bars = reinterpret_cast<uint64_t *>(nv_s + 16);
     uint64_t *full = bars, *empty = bars + p.stages, *tfull = bars + 2 * p.stages;
-    uint64_t *tempty = tfull + 2, *drain = tempty + 2;
+    uint64_t *tempty = tfull + p.nacc, *drain = tempty + p.nacc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *pg_s = const_cast<int *>(abort_flag) + 4;     // page ids of this CTA's tiles (-1: none)
+    // per epilogue group, kKsRing tiles of key scales in flight (cp.async ring)
+    float *ks_ring = reinterpret_cast<float *>(
+        (reinterpret_cast<uintptr_t>(pg_s + 2 * p.tiles_per_cta) + 15) & ~(uintptr_t)15);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -119,11 +125,12 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     if (warp == 0) tc::tmem_alloc(tc::saddr(tmem_slot), (uint32_t)p.tmem_cols);
     if (threadIdx.x == 32) {
         for (int s = 0; s < p.stages; s++) {
-            // FP4: the TMA transaction and the block-scale gather both arrive
-            tc::mbar_init(tc::saddr(&full[s]), kFp4 ? 2 : 1);
+            // one arrival (the producer's expect_tx); FP4 block-scale copies
+            // add and complete their own pending arrivals
+            tc::mbar_init(tc::saddr(&full[s]), 1);
             tc::mbar_init(tc::saddr(&empty[s]), 1);
         }
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < p.nacc; i++) {
             tc::mbar_init(tc::saddr(&tfull[i]), 1);
             tc::mbar_init(tc::saddr(&tempty[i]), 4);     // the 4 warps of one group
         }
@@ -195,6 +202,33 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             const int tile = tile_begin + i;
+            if constexpr (kFp4) {
+                // key m = lane + 32*m1 of the tile: its block scales of K-step ks go
+                // to byte (s*ksteps + ks)*512 + lane*16 + m1*4 by 4-byte cp.async;
+                // each lane's copies hold the stage's phase open until they land
+                // (the non-noinc arrive adds one pending arrival first)
+                constexpr int nsf = RB / 8;      // Di/16 block scales per key
+#pragma unroll
+                for (int m1 = 0; m1 < 4; m1++) {
+                    const int m = lane + 32 * m1;
+                    const int sk = tile * kTcTile + m;
+                    int64_t slot = -1;
+                    if (sk < nv_max) {
+                        const int32_t page = pg_s[i * 2 + (m >> 6)];
+                        if (page >= 0 && page < p.num_pages) slot = (int64_t)page * kC4Page + (m & 63);
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < G::kKSteps; ks++) {
+                        uint8_t *dst = sfa_buf + (s * G::kKSteps + ks) * 512 + lane * 16 + m1 * 4;
+                        if (slot >= 0)
+                            tc::cp_async4(tc::saddr(dst), a.k_block_scales + slot * nsf + ks * 4);
+                        else
+                            *reinterpret_cast<uint32_t *>(dst) = 0u;
+                    }
+                }
+                tc::cp_async_mbar_arrive(tc::saddr(&full[s]));
+                __syncwarp();
+            }
             if (lane == 0) {
                 tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
 #pragma unroll
@@ -209,33 +243,6 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                                         tc::saddr(&full[s]));
                 }
             }
-            if constexpr (kFp4) {
-                // key m = lane + 32*m1 of the tile; its block scales for K-step ks
-                constexpr int nsf = RB / 8;      // Di/16 block scales per key
-                uint32_t wv[G::kKSteps][4];
-#pragma unroll
-                for (int m1 = 0; m1 < 4; m1++) {
-                    const int m = lane + 32 * m1;
-                    const int sk = tile * kTcTile + m;
-                    int64_t slot = -1;
-                    if (sk < nv_max) {
-                        const int32_t page = pg_s[i * 2 + (m >> 6)];
-                        if (page >= 0 && page < p.num_pages) slot = (int64_t)page * kC4Page + (m & 63);
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < G::kKSteps; ks++)
-                        wv[ks][m1] = slot >= 0 ? *reinterpret_cast<const uint32_t *>(
-                                                     a.k_block_scales + slot * nsf + ks * 4)
-                                               : 0u;
-                }
-#pragma unroll
-                for (int ks = 0; ks < G::kKSteps; ks++)
-                    *reinterpret_cast<uint4 *>(sfa_buf + (s * G::kKSteps + ks) * 512 + lane * 16) =
-                        make_uint4(wv[ks][0], wv[ks][1], wv[ks][2], wv[ks][3]);
-                tc::fence_proxy_async();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(tc::saddr(&full[s]));
-            }
             issued++;
         }
         // before leaving, every load issued must have landed
@@ -248,10 +255,11 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             const uint32_t idesc = FMT == CSA_FMT_FP8  ? tc::idesc_m128(0, 0, p.n)
                                    : FMT == CSA_FMT_BF16 ? tc::idesc_m128(1, 1, p.n)
                                                          : tc::idesc_mxf4_m128(p.n);
-            // TMEM columns: [0, 2n) accumulators, then two sets of key block
-            // scales (4 columns per K-step), then the query block scales
-            const uint32_t sfa_col = (uint32_t)(2 * p.n);
-            const uint32_t sfb_col = sfa_col + 8u * G::kKSteps;
+            // TMEM columns: [0, nacc*n) accumulators, then one set of key block
+            // scales per accumulator (4 columns per K-step), then the query
+            // block scales
+            const uint32_t sfa_col = (uint32_t)(p.nacc * p.n);
+            const uint32_t sfb_col = sfa_col + (uint32_t)(p.nacc * 4 * G::kKSteps);
             if constexpr (kFp4) {
 #pragma unroll
                 for (int ks = 0; ks < G::kKSteps; ks++)
@@ -260,15 +268,16 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             }
             for (int i = 0; i < my_tiles; i++) {
                 const int s = i % p.stages;
-                const int acc = i & 1;
+                const int acc = i & (p.nacc - 1);
                 if (!tc::mbar_wait(tc::saddr(&full[s]), (uint32_t)((i / p.stages) & 1), abort_flag) ||
-                    !tc::mbar_wait(tc::saddr(&tempty[acc]), (uint32_t)(((i >> 1) & 1) ^ 1),
+                    !tc::mbar_wait(tc::saddr(&tempty[acc]), (uint32_t)(((i / p.nacc) & 1) ^ 1),
                                    abort_flag)) {
                     if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
                     *abort_flag = 1;
                     break;
                 }
                 tc::fence_after_sync();
+                if constexpr (kFp4) tc::fence_proxy_async();   // cp.async-written scales -> tcgen05.cp
                 const uint32_t d = tmem_base + (uint32_t)(acc * p.n);
                 const uint32_t sa = tc::saddr(stage_buf + s * G::kStageBytes);
                 const uint32_t sb = tc::saddr(q_buf);
@@ -304,29 +313,47 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float *lg = a.logits;
-        // key scale of this thread's row, fetched one tile ahead of its use
-        auto key_scale = [&](int i, bool &valid) -> float {
+        // Key scale of this thread's row for the group's j-th tile (i = eg + 2j):
+        // a per-thread ring of kKsRing cp.async copies keeps the loads of the
+        // next tiles in flight while this one is reduced.
+        auto key_slot = [&](int i, bool &valid) -> int64_t {
             const int sk = (tile_begin + i) * kTcTile + row;
             valid = false;
-            if (sk >= nv_max) return 0.0f;
+            if (i >= my_tiles || sk >= nv_max) return -1;
             const int32_t page = pg_s[i * 2 + (row >> 6)];
             const int64_t slot = (int64_t)page * kC4Page + (row & 63);
             valid = page >= 0 && page < p.num_pages && slot < a.num_slots;
-            if (!valid) {
-                report(a.status, CSA_ERR_BOUNDS);
-                return 0.0f;
-            }
-            return FMT == CSA_FMT_BF16 ? 1.0f : __ldg(a.k_scales + slot);
+            return valid ? slot : -1;
         };
-        bool valid_next = false;
-        float kscale_next = eg < my_tiles ? key_scale(eg, valid_next) : 0.0f;
+        float *my_ring = ks_ring + eg * kKsRing * kTcTile + row;
+        auto ring_issue = [&](int j) {
+            if constexpr (FMT != CSA_FMT_BF16) {
+                bool v;
+                const int64_t slot = key_slot(eg + 2 * j, v);
+                if (slot >= 0) tc::cp_async4(tc::saddr(my_ring + (j % kKsRing) * kTcTile),
+                                             a.k_scales + slot);
+                tc::cp_async_commit();
+            }
+        };
+        // tiles j .. j+kKsRing-2 are in flight when tile j is consumed; the copy for
+        // tile j+kKsRing-1 then goes to the slot read one tile earlier
+#pragma unroll 1
+        for (int j = 0; j < kKsRing - 1; j++) ring_issue(j);
         for (int i = eg; i < my_tiles; i += 2) {
-            const int acc = eg;
+            const int acc = i & (p.nacc - 1);     // same parity as i: this group's
+            const int j = (i - eg) >> 1;
             const int sk = (tile_begin + i) * kTcTile + row;
-            const float kscale = kscale_next;
-            const bool valid = valid_next;
-            if (i + 2 < my_tiles) kscale_next = key_scale(i + 2, valid_next);
-            if (!tc::mbar_wait(tc::saddr(&tfull[acc]), (uint32_t)((i >> 1) & 1), abort_flag)) {
+            bool valid;
+            const int64_t slot_i = key_slot(i, valid);
+            (void)slot_i;
+            if (!valid && sk < nv_max) report(a.status, CSA_ERR_BOUNDS);
+            float kscale = 1.0f;
+            if constexpr (FMT != CSA_FMT_BF16) {
+                tc::cp_async_wait<kKsRing - 2>();
+                kscale = valid ? my_ring[(j % kKsRing) * kTcTile] : 0.0f;
+                ring_issue(j + kKsRing - 1);
+            }
+            if (!tc::mbar_wait(tc::saddr(&tfull[acc]), (uint32_t)((i / p.nacc) & 1), abort_flag)) {
                 if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
                 *abort_flag = 1;
                 break;
@@ -367,6 +394,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                         lg[(int64_t)(t0 + x) * a.logits_stride + sk] = out[x] * kscale;
             }
         }
+        tc::cp_async_wait<0>();     // no copy into the ring outlives the loop
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -418,8 +446,8 @@ static bool make_key_map(CUtensorMap *m, const void *codes, int64_t num_slots, i
 static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p) {
     const size_t ks = rb / 32;
     return 1024 + (size_t)p.stages * kTcTile * rb + (((size_t)p.n * rb + 1023) & ~(size_t)1023) +
-           (fp4 ? (p.stages + 1) * ks * 512 : 0) + 256 * 4 + 16 * 4 + (2 * p.stages + 5) * 8 + 32 +
-           (size_t)2 * p.tiles_per_cta * 4;
+           (fp4 ? (p.stages + 1) * ks * 512 : 0) + 256 * 4 + 16 * 4 + (2 * p.stages + 2 * p.nacc + 1) * 8 + 32 +
+           (size_t)2 * p.tiles_per_cta * 4 + 16 + (size_t)2 * kKsRing * kTcTile * 4;
 }
 
 bool indexer_tc_supported(const IndexerArgs &a) {
@@ -446,13 +474,19 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
     if (p.qg > 4) p.qg = 4;
     if (fp4 && p.qg * p.hi_pad > 64) p.qg = p.hi_pad >= 64 ? 1 : 64 / p.hi_pad;
     p.n = p.qg * p.hi_pad;
+    // as many accumulators in flight (up to 8) as keep the CTA within 256 TMEM
+    // columns (two CTAs per SM): the MMA of tile i waits for the epilogue of
+    // tile i - nacc, so a deeper ring hides the hand-off latency of small tiles
+    auto tmem_need = [&](int nacc) { return nacc * p.n + (fp4 ? (nacc * 4 + 4) * (rb / 32) : 0); };
+    p.nacc = 2;
+    while (p.nacc < 8 && tmem_need(2 * p.nacc) <= 256) p.nacc *= 2;
     int cols = 32;
-    const int need = 2 * p.n + (fp4 ? 12 * (rb / 32) : 0);
+    const int need = tmem_need(p.nacc);
     while (cols < need) cols <<= 1;
     p.tmem_cols = cols;
     p.num_pages = (int)(a.num_slots / kC4Page);
-    // ~96 KB of key tiles in flight per CTA, two CTAs per SM
-    p.stages = rb == 256 ? 3 : rb == 128 ? 6 : rb == 64 ? 12 : 16;
+    // 64-80 KB of key tiles in flight per CTA, two CTAs per SM
+    p.stages = rb == 256 ? 3 : rb == 128 ? 5 : rb == 64 ? 8 : 16;
     const int tiles_max = (a.max_c4_len + kTcTile - 1) / kTcTile;
     const int groups = (a.num_q + p.qg - 1) / p.qg;
     // one wave: at most (SMs x resident CTAs per SM) CTAs, split evenly over
