@@ -53,6 +53,38 @@ def parse():
     return p.parse_args()
 
 
+INDEXER_SOURCES = ("indexer_tc.cu", "tc.cuh", "common.cuh", "launch.h")
+
+
+def indexer_source_hash() -> str:
+    """sha256 over the indexer kernel's sources, to tie an ncu capture to them."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in INDEXER_SOURCES:
+        with open(os.path.join(ROOT, "compressed_sparse_attention_12_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(w):
+    """DRAM bytes (read + write) per indexer launch from the committed ncu
+    summary of this workload, or None when there is none or the indexer's
+    sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", f"indexer_tc_{w.name.replace('_', '')}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as fh:
+        for line in fh:
+            if ":" in line and line.split(":", 1)[0].strip() in ("traffic_bytes_per_launch",
+                                                                  "source_sha256"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != indexer_source_hash() or "traffic_bytes_per_launch" not in vals:
+        return None
+    return int(vals["traffic_bytes_per_launch"])
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -361,18 +393,20 @@ def main():
     if rank == 0:
         hbm, src = peaks()
         ib = indexer_alg_bytes(w)
+        traffic = profiled_traffic(w)
         achieved = ib / t_idx / 1e9
         sb = step_alg_bytes(w)
         out = {"metric": METRIC, "value": world * w.num_q / t_step, "unit": UNIT, "n_gpus": world,
                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-               "dtype": f"{w.idx_fmt} indexer, bf16 attention", "data": "synthetic",
+               "dtype": f"{w.idx_fmt} indexer, {'f16' if w.kv_fmt == 'fp8' else 'bf16'} attention",
+               "data": "synthetic",
                "config": workload_config(w),
                "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
                        "frac_of_8tbs": sb / t_step / 8e12, "frac_of_peak": sb / t_step / 1e9 / hbm},
                "roofline": {"kernel": "indexer_logits", "bound": "hbm", "achieved": achieved,
                             "peak": hbm, "peak_source": src, "unit": "GB/s",
-                            "frac": achieved / hbm, "traffic": None,
+                            "frac": achieved / hbm, "traffic": traffic,
                             "alg_bytes_per_launch": ib, "launch_ms": t_idx * 1e3},
                "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": ck}
         if not args.no_cpu_baseline and not args.profile and world == 1:
