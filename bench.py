@@ -79,7 +79,7 @@ def profiled_traffic(w):
             if ":" in line and line.split(":", 1)[0].strip() in ("traffic_bytes_per_launch",
                                                                   "source_sha256"):
                 k, v = line.split(":", 1)
-                vals[k.strip()] = v.strip().strip("`")
+                vals[k.strip()] = v.split()[0].strip("`") if v.split() else ""
     if vals.get("source_sha256") != indexer_source_hash() or "traffic_bytes_per_launch" not in vals:
         return None
     return int(vals["traffic_bytes_per_launch"])
