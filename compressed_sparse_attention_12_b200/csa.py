@@ -53,6 +53,15 @@ _SIGS = {
     "csa_topk512_page_transform_noalloc": (ctypes.c_int, [_P, _I64, _I32, _P, _I32, _P, _P, _P,
                                                          _I32, _I64, _I32, _I32, _P, _P, _P,
                                                          _P]),
+    "csa_indexer_topk512_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32]),
+    "csa_indexer_topk512": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _I64,
+                                           _P, _I32, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P,
+                                           _P, _P, _SZ, _P, _P]),
+    "csa_indexer_select": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _I64,
+                                          _P, _I32, _P, _I32, _P, _P, _I32, _P, _I64, _P, _SZ,
+                                          _P, _P]),
+    "csa_topk512_merge": (ctypes.c_int, [_I32, _I32, _I32, _I32, _P, _I32, _P, _P, _P, _I32,
+                                         _I64, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
     "csa_sparse_mqa_decode": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _P,
                                              _I32, _P, _I32, _P, _P, _I32, _F, _P, _P, _P, _SZ,
@@ -181,6 +190,55 @@ def csa_topk512_page_transform_noalloc(logits, c4_seq_lens, cu_q, q_pos, page_ta
         _ptr(logits), logits.shape[1], num_q, _ptr(c4_seq_lens), c4_seq_lens.shape[0], _ptr(cu_q),
         _ptr(q_pos), _ptr(page_table), page_table.shape[1], int(num_slots), int(c4_page_size),
         int(max_c4_len), _ptr(out_indices), _ptr(raw_indices), _ptr(status), _stream(stream)))
+
+
+def csa_indexer_topk512_workspace_size(num_q, bs, idx_heads, idx_dim, fmt, max_c4_len) -> int:
+    return lib().csa_indexer_topk512_workspace_size(num_q, bs, idx_heads, idx_dim, fmt,
+                                                    max_c4_len)
+
+
+def csa_indexer_topk512(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, fmt, k_codes,
+                        k_block_scales, k_scales, page_table, c4_seq_lens, cu_q, q_pos,
+                        max_c4_len, logits, out_indices, raw_indices=None, workspace=None,
+                        num_slots=None, c4_page_size=C4_PAGE_SIZE, status=None, stream=None):
+    """Indexer logits + top-512 page transform in one call (see include/csa.h)."""
+    num_q = q_weights.shape[0]
+    bs = c4_seq_lens.shape[0]
+    if workspace is None:
+        n = csa_indexer_topk512_workspace_size(num_q, bs, idx_heads, idx_dim, fmt, max_c4_len)
+        workspace = torch.empty(max(1, n), dtype=torch.uint8, device=logits.device)
+    _check("csa_indexer_topk512", lib().csa_indexer_topk512(
+        _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
+        _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
+        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        page_table.shape[1], _ptr(c4_seq_lens), bs, _ptr(cu_q), _ptr(q_pos), int(max_c4_len),
+        int(c4_page_size), _ptr(logits), logits.shape[1], _ptr(out_indices), _ptr(raw_indices),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
+
+
+def csa_indexer_select(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, fmt, k_codes,
+                       k_block_scales, k_scales, page_table, c4_seq_lens, cu_q, q_pos,
+                       max_c4_len, logits, workspace, num_slots=None, status=None, stream=None):
+    """First half of csa_indexer_topk512: logits + per-chunk candidates."""
+    num_q = q_weights.shape[0]
+    _check("csa_indexer_select", lib().csa_indexer_select(
+        _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
+        _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
+        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        page_table.shape[1], _ptr(c4_seq_lens), c4_seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos),
+        int(max_c4_len), _ptr(logits), logits.shape[1], _ptr(workspace), workspace.numel(),
+        _ptr(status), _stream(stream)))
+
+
+def csa_topk512_merge(num_q, idx_heads, idx_dim, fmt, c4_seq_lens, cu_q, q_pos, page_table,
+                      num_slots, max_c4_len, out_indices, workspace, raw_indices=None,
+                      c4_page_size=C4_PAGE_SIZE, status=None, stream=None):
+    """Second half of csa_indexer_topk512: row merge + page transform."""
+    _check("csa_topk512_merge", lib().csa_topk512_merge(
+        int(num_q), idx_heads, idx_dim, fmt, _ptr(c4_seq_lens), c4_seq_lens.shape[0], _ptr(cu_q),
+        _ptr(q_pos), _ptr(page_table), page_table.shape[1], int(num_slots), int(c4_page_size),
+        int(max_c4_len), _ptr(out_indices), _ptr(raw_indices), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)))
 
 
 def csa_sparse_mqa_workspace_size(num_q, heads, window, decode) -> int:

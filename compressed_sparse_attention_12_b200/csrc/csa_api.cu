@@ -158,6 +158,132 @@ csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stri
     return cuda_status(csa::launch_topk512(a, as_stream(stream)));
 }
 
+size_t csa_indexer_topk512_workspace_size(int32_t num_q, int32_t bs, int32_t idx_heads,
+                                          int32_t idx_dim, int32_t fmt, int32_t max_c4_len) {
+    if (num_q <= 0 || bs <= 0 || max_c4_len <= 0) return 0;
+    size_t need = csa::topk_workspace_bytes(num_q, max_c4_len);
+    if ((idx_dim == 64 || idx_dim == 128) && index_fmt_ok(fmt) && idx_heads >= 1 &&
+        idx_heads <= 128) {
+        csa::IndexerArgs a{};
+        a.num_q = num_q;
+        a.heads = idx_heads;
+        a.dim = idx_dim;
+        a.fmt = fmt;
+        a.bs = bs;
+        a.max_c4_len = max_c4_len;
+        a.num_slots = 64;
+        const size_t f = csa::indexer_topk_fused_bytes(a);
+        if (f > need) need = f;
+    }
+    return need;
+}
+
+csa_status_t csa_indexer_topk512(const void *q_codes, const uint8_t *q_block_scales,
+                                 const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                 int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                 const uint8_t *k_block_scales, const float *k_scales,
+                                 int64_t num_slots, const int32_t *page_table,
+                                 int32_t page_table_stride, const int32_t *c4_seq_lens, int32_t bs,
+                                 const int32_t *cu_q, const int32_t *q_pos, int32_t max_c4_len,
+                                 int32_t c4_page_size, float *logits, int64_t logits_stride,
+                                 int32_t *c4_sparse_page_indices, int32_t *raw_indices,
+                                 void *workspace, size_t workspace_bytes, int32_t *status,
+                                 void *stream) {
+    if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (c4_page_size != CSA_C4_PAGE_SIZE) return CSA_ERR_INVALID;
+    if (!index_fmt_ok(fmt)) return CSA_ERR_UNSUPPORTED;
+    if (idx_dim != 64 && idx_dim != 128) return CSA_ERR_UNSUPPORTED;
+    if (idx_heads < 1 || idx_heads > 128) return CSA_ERR_UNSUPPORTED;
+    if (num_q == 0) return CSA_OK;
+    if (bs < 1 || !c4_seq_lens || !cu_q || !page_table || !c4_sparse_page_indices)
+        return CSA_ERR_INVALID;
+    if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
+    csa::TopkArgs t{logits, logits_stride, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,
+                    page_table_stride, num_slots, max_c4_len, c4_sparse_page_indices,
+                    raw_indices, workspace, status};
+    cudaStream_t s = as_stream(stream);
+    if (max_c4_len == 0) return cuda_status(csa::launch_topk512(t, s));   // -1 padding only
+    if (!q_codes || !q_weights || !logits || logits_stride < max_c4_len) return CSA_ERR_INVALID;
+    if (fmt == CSA_FMT_FP4 && !q_block_scales) return CSA_ERR_INVALID;
+    if (!index_arrays_ok(fmt, k_codes, k_block_scales, k_scales)) return CSA_ERR_INVALID;
+    if (!workspace || workspace_bytes < csa_indexer_topk512_workspace_size(
+                                            num_q, bs, idx_heads, idx_dim, fmt, max_c4_len))
+        return CSA_ERR_WORKSPACE;
+    csa::IndexerArgs a{q_codes, q_block_scales, q_weights, num_q, idx_heads, idx_dim, fmt,
+                       k_codes, k_block_scales, k_scales, num_slots, page_table,
+                       page_table_stride, c4_seq_lens, bs, cu_q, q_pos, max_c4_len, logits,
+                       logits_stride, status};
+    if (csa::indexer_topk_fuses(a)) return cuda_status(csa::launch_indexer_topk_fused(a, t, s));
+    cudaError_t e = csa::launch_indexer(a, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    return cuda_status(csa::launch_topk512(t, s));
+}
+
+csa_status_t csa_indexer_select(const void *q_codes, const uint8_t *q_block_scales,
+                                const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                const uint8_t *k_block_scales, const float *k_scales,
+                                int64_t num_slots, const int32_t *page_table,
+                                int32_t page_table_stride, const int32_t *c4_seq_lens, int32_t bs,
+                                const int32_t *cu_q, const int32_t *q_pos, int32_t max_c4_len,
+                                float *logits, int64_t logits_stride, void *workspace,
+                                size_t workspace_bytes, int32_t *status, void *stream) {
+    if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (!index_fmt_ok(fmt)) return CSA_ERR_UNSUPPORTED;
+    if (idx_dim != 64 && idx_dim != 128) return CSA_ERR_UNSUPPORTED;
+    if (idx_heads < 1 || idx_heads > 128) return CSA_ERR_UNSUPPORTED;
+    if (num_q == 0 || max_c4_len == 0) return CSA_OK;
+    if (bs < 1 || !q_codes || !q_weights || !page_table || !c4_seq_lens || !cu_q || !logits ||
+        logits_stride < max_c4_len)
+        return CSA_ERR_INVALID;
+    if (fmt == CSA_FMT_FP4 && !q_block_scales) return CSA_ERR_INVALID;
+    if (!index_arrays_ok(fmt, k_codes, k_block_scales, k_scales)) return CSA_ERR_INVALID;
+    if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < csa_indexer_topk512_workspace_size(
+                                            num_q, bs, idx_heads, idx_dim, fmt, max_c4_len))
+        return CSA_ERR_WORKSPACE;
+    csa::IndexerArgs a{q_codes, q_block_scales, q_weights, num_q, idx_heads, idx_dim, fmt,
+                       k_codes, k_block_scales, k_scales, num_slots, page_table,
+                       page_table_stride, c4_seq_lens, bs, cu_q, q_pos, max_c4_len, logits,
+                       logits_stride, status};
+    if (!csa::indexer_topk_fuses(a)) return CSA_ERR_UNSUPPORTED;
+    return cuda_status(csa::launch_indexer_select(a, workspace, as_stream(stream)));
+}
+
+csa_status_t csa_topk512_merge(int32_t num_q, int32_t idx_heads, int32_t idx_dim, int32_t fmt,
+                               const int32_t *c4_seq_lens, int32_t bs, const int32_t *cu_q,
+                               const int32_t *q_pos, const int32_t *page_table,
+                               int32_t page_table_stride, int64_t num_slots,
+                               int32_t c4_page_size, int32_t max_c4_len,
+                               int32_t *c4_sparse_page_indices, int32_t *raw_indices,
+                               const void *workspace, size_t workspace_bytes, int32_t *status,
+                               void *stream) {
+    if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
+    if (c4_page_size != CSA_C4_PAGE_SIZE) return CSA_ERR_INVALID;
+    if (!index_fmt_ok(fmt)) return CSA_ERR_UNSUPPORTED;
+    if (idx_dim != 64 && idx_dim != 128) return CSA_ERR_UNSUPPORTED;
+    if (idx_heads < 1 || idx_heads > 128) return CSA_ERR_UNSUPPORTED;
+    if (num_q == 0) return CSA_OK;
+    if (bs < 1 || !c4_seq_lens || !cu_q || !page_table || !c4_sparse_page_indices)
+        return CSA_ERR_INVALID;
+    if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
+    if (max_c4_len > 0 && (!workspace || workspace_bytes < csa_indexer_topk512_workspace_size(
+                                             num_q, bs, idx_heads, idx_dim, fmt, max_c4_len)))
+        return CSA_ERR_WORKSPACE;
+    csa::IndexerArgs shape{};
+    shape.num_q = num_q;
+    shape.heads = idx_heads;
+    shape.dim = idx_dim;
+    shape.fmt = fmt;
+    shape.bs = bs;
+    shape.max_c4_len = max_c4_len;
+    shape.num_slots = num_slots;
+    csa::TopkArgs t{nullptr, 0, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,
+                    page_table_stride, num_slots, max_c4_len, c4_sparse_page_indices,
+                    raw_indices, const_cast<void *>(workspace), status};
+    return cuda_status(csa::launch_topk_merge(shape, t, as_stream(stream)));
+}
+
 csa_status_t csa_topk512_page_transform_noalloc(const float *logits, int64_t logits_stride,
                                                 int32_t num_q, const int32_t *c4_seq_lens,
                                                 int32_t bs, const int32_t *cu_q,

@@ -29,6 +29,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "tc.cuh"
+#include "topk.cuh"
 
 namespace csa {
 
@@ -54,12 +55,22 @@ struct TcParams {
     int nacc;          // TMEM accumulators in flight (power of two, >= 2)
 };
 
+// Where a fused launch leaves each CTA's chunk selection (all null: logits only).
+// Row t, chunk c (= blockIdx.x, tiles_per_cta*128 keys) owns 512 slots at
+// (t*max_chunks + c)*512 and one (512th key, largest key) pair.
+struct TcSelect {
+    uint32_t *cand_key;
+    int32_t *cand_idx;
+    uint2 *chunk_info;
+    int max_chunks;
+};
+
 constexpr int kKsRing = 8;     // key-scale tiles in flight per epilogue group
 
 template <int FMT, int RB>
 __global__ void __launch_bounds__(kTcThreads, 2)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
-                  const TcParams p) {
+                  const TcParams p, const TcSelect sel) {
     pdl_begin();
     using G = TcGeom<RB>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -403,6 +414,30 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         __syncwarp();
         tc::tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
     }
+    if (sel.cand_key == nullptr || *abort_flag) return;
+    // ---- fused top-512 of this CTA's chunk, per query row of the group: the
+    // logits just written (visible to the block after the barrier above, and
+    // still in L2) come back into the drained stage buffers; the chunk's
+    // candidates go to the workspace for the row-level merge
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(stage_buf);
+    TkSharedT<kTcThreads> &tsh = *reinterpret_cast<TkSharedT<kTcThreads> *>(
+        stage_buf + (size_t)p.tiles_per_cta * kTcTile * 4);
+    const int k0 = tile_begin * kTcTile;
+    for (int x = 0; x < nq; x++) {
+        const int len = min(tile_end * kTcTile, nv_s[x]) - k0;
+        if (len <= 0) continue;                    // uniform over the CTA
+        const float *row = a.logits + (int64_t)(t0 + x) * a.logits_stride + k0;
+        const int n4 = (reinterpret_cast<uintptr_t>(row) & 15) == 0 ? len / 4 : 0;
+        for (int i = threadIdx.x; i < n4; i += kTcThreads)
+            reinterpret_cast<uint4 *>(skeys)[i] = reinterpret_cast<const uint4 *>(row)[i];
+        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTcThreads)
+            skeys[i] = __float_as_uint(row[i]);
+        __syncthreads();
+        const int64_t c = (int64_t)(t0 + x) * sel.max_chunks + blockIdx.x;
+        select_chunk<kTcThreads>(skeys, len, k0, sel.cand_key + c * kTopK, sel.cand_idx + c * kTopK,
+                                 sel.chunk_info + c, tsh, a.status);
+        __syncthreads();
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -462,10 +497,22 @@ bool indexer_tc_supported(const IndexerArgs &a) {
            encode_fn() != nullptr;
 }
 
-cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
+// Launch shape of the tensor-core indexer.  `fuse`: each CTA also selects its
+// chunk's top-512, so a chunk (tiles_per_cta tiles) must hold 512..8192 keys
+// (fewer only when the whole row is one chunk) and its logits must fit the
+// drained stage buffers next to the selection's shared state.
+struct TcPlan {
+    TcParams p;
+    int rb, chunks;
+    size_t smem;
+};
+
+static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
+    TcPlan pl;
+    TcParams &p = pl.p;
     const bool fp4 = a.fmt == CSA_FMT_FP4;
     const int rb = a.fmt == CSA_FMT_FP8 ? a.dim : fp4 ? a.dim / 2 : 2 * a.dim;
-    TcParams p;
+    pl.rb = rb;
     p.hi_pad = (a.heads + 15) / 16 * 16;
     // queries of one request share the key tiles: group up to 4 of them
     // (N <= 128) when requests carry several query rows
@@ -497,7 +544,7 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
         if (cudaGetDevice(&dev) == cudaSuccess)
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    p.tiles_per_cta = tiles_max;                      // upper bound for the estimate
+    p.tiles_per_cta = fuse ? 64 : tiles_max;          // upper bound for the estimate
     // 228 KB of shared memory per SM, 1 KB of it reserved per resident CTA
     const size_t smem_est = tc_smem_bytes(rb, fp4, p) + 1024;
     int by_smem = (int)((228 * 1024) / smem_est);
@@ -510,18 +557,47 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
     if (chunks > tiles_max) chunks = tiles_max;
     if (chunks < 1) chunks = 1;
     p.tiles_per_cta = (tiles_max + chunks - 1) / chunks;
-    chunks = (tiles_max + p.tiles_per_cta - 1) / p.tiles_per_cta;
+    // when the query groups alone do not fill the wave, rows are split; keep
+    // the pieces at most 64 tiles so that rows of very different lengths
+    // (a ragged batch sized by its longest row) still spread over the SMs
+    if (groups < target && p.tiles_per_cta > 64) p.tiles_per_cta = 64;
+    if (fuse) {
+        // 512..8192 keys per chunk (the logits of a chunk, 32 KB at most, and
+        // the selection state fit in the >= 64 KB of stage buffers)
+        if (p.tiles_per_cta > 64) p.tiles_per_cta = 64;
+        if (p.tiles_per_cta < 4) p.tiles_per_cta = tiles_max < 4 ? tiles_max : 4;
+        if (p.tiles_per_cta < 1) p.tiles_per_cta = 1;
+    }
+    pl.chunks = (tiles_max + p.tiles_per_cta - 1) / p.tiles_per_cta;
+    if (pl.chunks < 1) pl.chunks = 1;
+    pl.smem = tc_smem_bytes(rb, fp4, p);
+    return pl;
+}
 
+// The fused launch is used where the plain launch's pieces are at most 64
+// tiles (the fused plan then only merges pieces below 4 tiles); elsewhere
+// (long rows per query group, e.g. chunked prefill) the plain indexer and the
+// two-stage top-k run.
+bool indexer_topk_fuses(const IndexerArgs &a) {
+    if (!indexer_tc_supported(a)) return false;
+    return plan_tc(a, false).p.tiles_per_cta <= 64;
+}
+
+static cudaError_t launch_tc_plan(const IndexerArgs &a, const TcPlan &pl, const TcSelect &sel,
+                                  cudaStream_t s) {
     CUtensorMap map;
-    if (!make_key_map(&map, a.k_codes, a.num_slots, rb)) return cudaErrorInvalidValue;
-    const size_t smem = tc_smem_bytes(rb, fp4, p);
-    dim3 grid(chunks, a.num_q);
+    if (!make_key_map(&map, a.k_codes, a.num_slots, pl.rb)) return cudaErrorInvalidValue;
+    const TcParams p = pl.p;
+    const size_t smem = pl.smem;
+    dim3 grid(pl.chunks, a.num_q);
+    const bool fp4 = a.fmt == CSA_FMT_FP4;
+    const int rb = pl.rb;
 #define CSA_TC(F, R)                                                                        \
     do {                                                                                    \
         static int done[64] = {0};                                                          \
         cudaError_t e = ensure_max_smem((const void *)indexer_tc_kernel<F, R>, 200 * 1024, done); \
         if (e != cudaSuccess) return e;                                                     \
-        launch_k(indexer_tc_kernel<F, R>, grid, kTcThreads, smem, s, a, map, p);                  \
+        launch_k(indexer_tc_kernel<F, R>, grid, kTcThreads, smem, s, a, map, p, sel);       \
     } while (0)
     if (a.fmt == CSA_FMT_FP8 && rb == 128) CSA_TC(CSA_FMT_FP8, 128);
     else if (a.fmt == CSA_FMT_FP8) CSA_TC(CSA_FMT_FP8, 64);
@@ -531,6 +607,46 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
     else CSA_TC(CSA_FMT_BF16, 256);
 #undef CSA_TC
     return cudaGetLastError();
+}
+
+cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s) {
+    const TcSelect none = {nullptr, nullptr, nullptr, 0};
+    return launch_tc_plan(a, plan_tc(a, false), none, s);
+}
+
+// Candidates + chunk pairs of the fused launch for this shape (the plan reads
+// only the shape fields of `a`: format, dim, heads, num_q, bs, max_c4_len).
+size_t indexer_topk_fused_bytes(const IndexerArgs &a) {
+    const TcPlan pl = plan_tc(a, true);
+    return (size_t)a.num_q * pl.chunks * (kTopK * 8 + sizeof(uint2));
+}
+
+static TcSelect select_layout(const TcPlan &pl, int num_q, void *workspace) {
+    const size_t nc = (size_t)num_q * pl.chunks;
+    TcSelect sel;
+    sel.cand_key = (uint32_t *)workspace;
+    sel.cand_idx = (int32_t *)((uint8_t *)workspace + nc * kTopK * 4);
+    sel.chunk_info = (uint2 *)((uint8_t *)workspace + nc * kTopK * 8);
+    sel.max_chunks = pl.chunks;
+    return sel;
+}
+
+cudaError_t launch_indexer_select(const IndexerArgs &a, void *workspace, cudaStream_t s) {
+    const TcPlan pl = plan_tc(a, true);
+    return launch_tc_plan(a, pl, select_layout(pl, a.num_q, workspace), s);
+}
+
+cudaError_t launch_topk_merge(const IndexerArgs &shape, const TopkArgs &t, cudaStream_t s) {
+    const TcPlan pl = plan_tc(shape, true);
+    const TcSelect sel = select_layout(pl, t.num_q, t.workspace);
+    return launch_topk_stage2(t, pl.chunks, pl.p.tiles_per_cta * kTcTile, sel.cand_key,
+                              sel.cand_idx, sel.chunk_info, s);
+}
+
+cudaError_t launch_indexer_topk_fused(const IndexerArgs &a, const TopkArgs &t, cudaStream_t s) {
+    cudaError_t e = launch_indexer_select(a, t.workspace, s);
+    if (e != cudaSuccess) return e;
+    return launch_topk_merge(a, t, s);
 }
 
 }  // namespace csa

@@ -101,6 +101,23 @@ struct TopkArgs {
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s);
 // Same, with the scratch in the library's own device array (no workspace).
 cudaError_t launch_topk512_noalloc(const TopkArgs &a, cudaStream_t s);
+// Row-level merge of per-chunk candidates (chunk_len keys per chunk, the last
+// one shorter; every chunk but a single one must hold >= 512 keys).
+cudaError_t launch_topk_stage2(const TopkArgs &a, int max_chunks, int chunk_len,
+                               const uint32_t *cand_key, const int32_t *cand_idx,
+                               const uint2 *chunk_info, cudaStream_t s);
+
+// Indexer whose CTAs also select their own chunk's top-512, then the row merge
+// (tensor-core indexer only: indexer_tc_supported).  The size query reads only
+// the shape fields of `a`.
+bool indexer_tc_supported(const IndexerArgs &a);
+bool indexer_topk_fuses(const IndexerArgs &a);
+size_t indexer_topk_fused_bytes(const IndexerArgs &a);
+cudaError_t launch_indexer_topk_fused(const IndexerArgs &a, const TopkArgs &t, cudaStream_t s);
+// The two halves of the fused launch: the selecting indexer (candidates into
+// `workspace`) and the row merge (reads the shape fields of `shape` only).
+cudaError_t launch_indexer_select(const IndexerArgs &a, void *workspace, cudaStream_t s);
+cudaError_t launch_topk_merge(const IndexerArgs &shape, const TopkArgs &t, cudaStream_t s);
 
 struct AttnArgs {
     const void *q;

@@ -8,204 +8,28 @@
 // ascending logical index and padded with -1.
 //
 // Two launches, no inter-CTA waits:
-//   stage 1: each CTA takes a chunk of 8192 logits of one query row into
-//            shared memory, finds the chunk's 512th key by a 3-pass radix
-//            select (12/12/8-bit digits, shared-memory histograms, block
-//            suffix scan), and writes the chunk's top-512 (key, index) pairs
-//            in index order to the workspace.
-//   stage 2: one CTA per query row repeats the select over the row's
-//            concatenated candidates (every element of the global top-512 is
-//            in its chunk's top-512 under the same total order) and writes
-//            physical slots page_table[s/64]*64 + s%64 and raw indices.
+//   stage 1: each CTA takes a chunk of logits of one query row into shared
+//            memory and writes the chunk's top-512 (key, index) pairs in index
+//            order plus (512th key, largest key) to the workspace
+//            (select_chunk in topk.cuh; the indexer kernel can run the same
+//            step on its own chunk instead).
+//   stage 2: one CTA per query row selects among the row's concatenated
+//            candidates (every element of the global top-512 is in its chunk's
+//            top-512 under the same total order) and writes physical slots
+//            page_table[s/64]*64 + s%64 and raw indices.
 #include "common.cuh"
 #include "launch.h"
+#include "topk.cuh"
 
 namespace csa {
 
 constexpr int kTkThreads = 512;
 constexpr int kTkChunk = 8192;
-constexpr int kTkWarps = kTkThreads / 32;
-constexpr int kHistBins = 4096;
 constexpr int kTk2Smem = 16384;      // stage-2 candidates staged in shared memory
-
-__device__ __forceinline__ uint32_t order_key(float f, int32_t *status) {
-    uint32_t u = __float_as_uint(f);
-    if (f != f) {  // NaN
-        report(status, CSA_ERR_NAN);
-        return 0u;
-    }
-    if (f == 0.0f) u = 0u;                        // -0 -> +0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-struct TkShared {
-    uint32_t hist[kHistBins];
-    uint32_t warp_a[kTkWarps];
-    uint32_t warp_b[kTkWarps];
-    uint32_t digit, above;
-    int32_t row_b, row_nvis;
-};
+using TkShared = TkSharedT<kTkThreads>;
 // the key buffers that follow TkShared in dynamic shared memory start on a
 // 16-byte boundary (they are read and written with 16-byte vectors)
 constexpr size_t kTkKeysOffset = (sizeof(TkShared) + 15) & ~(size_t)15;
-
-// Exclusive scan of one value per thread over the block; returns the prefix
-// and writes the block total to *total.  Uses sh.warp_a.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total, TkShared &sh) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) sh.warp_a[warp] = incl;
-    __syncthreads();
-    uint32_t before = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < kTkWarps; w++) {
-        const uint32_t x = sh.warp_a[w];
-        before += (w < warp) ? x : 0u;
-        tot += x;
-    }
-    __syncthreads();
-    *total = tot;
-    return before + incl - v;
-}
-
-// Block-wide min and max of one value pair per thread (uses sh.warp_a/b).
-__device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, TkShared &sh) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    }
-    if (lane == 0) {
-        sh.warp_a[warp] = lo;
-        sh.warp_b[warp] = hi;
-    }
-    __syncthreads();
-    lo = 0xffffffffu;
-    hi = 0u;
-#pragma unroll
-    for (int w = 0; w < kTkWarps; w++) {
-        lo = min(lo, sh.warp_a[w]);
-        hi = max(hi, sh.warp_b[w]);
-    }
-    __syncthreads();
-}
-
-// Finds the K-th largest key T among the keys[0..n) that are >= kmin (K <= their
-// count; kmax is their maximum) and how many keys equal to T belong to the top K
-// (need_eq >= 1).  The radix digits are taken from d = key - kmin, 12 bits at a
-// time from the highest set bit of kmax - kmin down, so that keys sharing sign
-// and exponent (the usual case for one row of logits) already spread over the
-// bins of the first pass; two passes resolve a range of up to 24 bits.  keys may
-// point to shared or global memory.
-__device__ void radix_threshold(const uint32_t *keys, int n, int K, uint32_t kmin, uint32_t kmax,
-                                TkShared &sh, uint32_t *T_out, int *need_eq_out) {
-    const uint32_t range = kmax - kmin;
-    const int B = range == 0 ? 0 : 32 - __clz(range);
-    uint32_t prefix = 0;            // resolved high bits of d
-    int remaining = K;
-#pragma unroll 1
-    for (int done = 0; done < B;) {
-        const int width = min(12, B - done);
-        const int shift = B - done - width;
-        const int hi = shift + width;            // bits at and above hi are resolved
-        const uint32_t nb = 1u << width;
-        for (uint32_t i = threadIdx.x; i < nb; i += kTkThreads) sh.hist[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kTkThreads) {
-            const uint32_t k = keys[i];
-            const uint32_t d = k - kmin;
-            const bool match = k >= kmin && (hi >= 32 || ((d ^ prefix) >> hi) == 0);
-            if (match) atomicAdd(&sh.hist[(d >> shift) & (nb - 1)], 1u);
-        }
-        __syncthreads();
-        // Suffix scan from the top bin: thread i owns bins nb-1-per*i .. nb-per*(i+1).
-        const int per = nb > (uint32_t)kTkThreads ? (int)nb / kTkThreads : 1;   // 1..8
-        uint32_t c[8];
-        uint32_t mine = 0;
-#pragma unroll
-        for (int j = 0; j < 8; j++) {
-            const int bin = (int)nb - 1 - ((int)threadIdx.x * per + j);
-            c[j] = (j < per && bin >= 0) ? sh.hist[bin] : 0u;
-            mine += c[j];
-        }
-        uint32_t total;
-        const uint32_t excl = block_excl_scan(mine, &total, sh);
-        if (excl < (uint32_t)remaining && (uint32_t)remaining <= excl + mine) {
-            uint32_t acc = excl;
-            bool found = false;
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                if (!found && j < per && acc + c[j] >= (uint32_t)remaining) {
-                    found = true;
-                    sh.digit = nb - 1 - (threadIdx.x * per + j);
-                    sh.above = acc;
-                }
-                acc += c[j];
-            }
-        }
-        __syncthreads();
-        prefix |= sh.digit << shift;
-        remaining -= (int)sh.above;
-        done += width;
-        __syncthreads();
-    }
-    *T_out = kmin + prefix;
-    *need_eq_out = remaining;
-}
-
-// Walks keys[0..n) in index order and calls emit(pos, i, key) for the
-// selected ones: key > T, or key == T among the first need_eq such keys.
-// Returns how many were selected.
-// Each warp owns one contiguous segment: it counts its segment with ballots,
-// one block barrier publishes the per-warp counts, then every warp writes its
-// selected elements at their global ranks.
-template <typename Emit>
-__device__ int ordered_compact(const uint32_t *keys, int n, uint32_t T, int need_eq,
-                               TkShared &sh, Emit emit) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = (1u << lane) - 1u;
-    const int seg = ((n + kTkWarps - 1) / kTkWarps + 31) & ~31;
-    const int beg = min(n, warp * seg), end = min(n, beg + seg);
-    uint32_t gt_w = 0, eq_w = 0;
-    for (int i = beg + lane; i < end + lane; i += 32) {   // uniform trip count per warp
-        const uint32_t k = i < end ? keys[i] : 0u;
-        gt_w += __popc(__ballot_sync(0xffffffffu, i < end && k > T));
-        eq_w += __popc(__ballot_sync(0xffffffffu, i < end && k == T));
-    }
-    if (lane == 0) {
-        sh.warp_a[warp] = eq_w;
-        sh.warp_b[warp] = gt_w;
-    }
-    __syncthreads();
-    uint32_t eq_before = 0, gt_before = 0, eq_all = 0, gt_all = 0;
-    for (int w = 0; w < kTkWarps; w++) {
-        eq_before += w < warp ? sh.warp_a[w] : 0u;
-        gt_before += w < warp ? sh.warp_b[w] : 0u;
-        eq_all += sh.warp_a[w];
-        gt_all += sh.warp_b[w];
-    }
-    __syncthreads();    // the counts may be reused by the caller's next phase
-    uint32_t eq_seen = eq_before;
-    uint32_t out = gt_before + min(eq_before, (uint32_t)need_eq);
-    for (int i = beg + lane; i < end + lane; i += 32) {
-        const uint32_t k = i < end ? keys[i] : 0u;
-        const bool gt = i < end && k > T;
-        const bool eq = i < end && k == T;
-        const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-        const bool take = gt || (eq && eq_seen + __popc(beq & lt) < (uint32_t)need_eq);
-        const uint32_t btk = __ballot_sync(0xffffffffu, take);
-        if (take) emit((int)(out + __popc(btk & lt)), i, k);
-        eq_seen += __popc(beq);
-        out += __popc(btk);
-    }
-    return (int)(gt_all + min(eq_all, (uint32_t)need_eq));
-}
 
 struct RowInfo {
     int b, n_vis;
@@ -272,45 +96,19 @@ topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32
     if (lo >= ri.n_vis) return;
     const int len = min(kTkChunk, ri.n_vis - lo);
     const float *row = logits + (int64_t)t * stride + lo;
-    uint32_t kmax = 0u;
-    bool has = false;
-    auto put = [&](int i, float f) {
-        const uint32_t k = order_key(f, status);
-        skeys[i] = k;
-        kmax = max(kmax, k);
-        has = true;
-    };
     if ((reinterpret_cast<uintptr_t>(row) & 15) == 0) {
         const int n4 = len / 4;
-        for (int i = threadIdx.x; i < n4; i += kTkThreads) {
-            const float4 v = reinterpret_cast<const float4 *>(row)[i];
-            put(4 * i, v.x);
-            put(4 * i + 1, v.y);
-            put(4 * i + 2, v.z);
-            put(4 * i + 3, v.w);
-        }
-        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTkThreads) put(i, row[i]);
+        for (int i = threadIdx.x; i < n4; i += kTkThreads)
+            reinterpret_cast<uint4 *>(skeys)[i] = reinterpret_cast<const uint4 *>(row)[i];
+        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTkThreads)
+            skeys[i] = __float_as_uint(row[i]);
     } else {
-        for (int i = threadIdx.x; i < len; i += kTkThreads) put(i, row[i]);
+        for (int i = threadIdx.x; i < len; i += kTkThreads) skeys[i] = __float_as_uint(row[i]);
     }
-    // The keys each thread loaded form one group.  When all 512 groups are
-    // non-empty the smallest group maximum is a lower bound of the 512th-largest
-    // key (the 512 group maxima are distinct keys >= it); otherwise the bound
-    // is 0.
-    uint32_t lbound = has ? kmax : 0u;
-    block_minmax(lbound, kmax, sh);     // its barrier also publishes skeys
-    const int K = min(kTopK, len);
-    uint32_t T = 0;
-    int need_eq = len;
-    if (len > kTopK) radix_threshold(skeys, len, K, lbound, kmax, sh, &T, &need_eq);
-    if (threadIdx.x == 0)
-        chunk_info[(int64_t)t * max_chunks + c] = make_uint2(len > kTopK ? T : 0u, kmax);
-    uint32_t *ok = cand_key + ((int64_t)t * max_chunks + c) * kTopK;
-    int32_t *oi = cand_idx + ((int64_t)t * max_chunks + c) * kTopK;
-    ordered_compact(skeys, len, T, need_eq, sh, [&](int pos, int i, uint32_t k) {
-        ok[pos] = k;
-        oi[pos] = lo + i;
-    });
+    __syncthreads();
+    select_chunk<kTkThreads>(skeys, len, lo, cand_key + ((int64_t)t * max_chunks + c) * kTopK,
+                             cand_idx + ((int64_t)t * max_chunks + c) * kTopK,
+                             chunk_info + (int64_t)t * max_chunks + c, sh, status);
 }
 
 // Stage 2: one CTA per query row.  The row's top-512 are all >= L, the largest
@@ -318,12 +116,12 @@ topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32
 // candidates below L are dropped first (in index order, into shared memory),
 // the threshold is found among the survivors, and the selection is written in
 // ascending index order, mapped through the page table, then padded with -1.
-// Rows with more than 16384 candidates select straight from the workspace.
 __global__ void __launch_bounds__(kTkThreads)
 topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const int32_t *q_pos,
                    int max_c4_len, const int32_t *page_table, int pt_stride, int64_t num_slots,
-                   int max_chunks, const uint32_t *cand_key, const int32_t *cand_idx,
-                   const uint2 *chunk_info, int32_t *out_phys, int32_t *out_raw,
+                   int max_chunks, int chunk_len, const uint32_t *cand_key,
+                   const int32_t *cand_idx, const uint2 *chunk_info, int32_t *out_phys,
+                   int32_t *out_raw,
                    int32_t *status) {
     pdl_begin();
     extern __shared__ __align__(16) uint8_t tk2_smem[];
@@ -336,8 +134,8 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
     const int n = ri.n_vis;
     int total = 0, nch = 0;
     if (n > 0) {
-        nch = (n + kTkChunk - 1) / kTkChunk;
-        total = (nch - 1) * kTopK + min(kTopK, n - (nch - 1) * kTkChunk);
+        nch = (n + chunk_len - 1) / chunk_len;
+        total = (nch - 1) * kTopK + min(kTopK, n - (nch - 1) * chunk_len);
     }
     const int K = min(kTopK, total);
     const uint32_t *keys = cand_key + (int64_t)t * max_chunks * kTopK;
@@ -352,16 +150,56 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
             L = max(L, ci.x);
             kmax = max(kmax, ci.y);
         }
+        // A tighter bound: the F full chunks (512 candidates each: all but the
+        // last) each hold m = ceil(512/F) keys >= their own m-th largest, so the
+        // row's 512th key is >= the smallest of those.  Warp w finds the m-th
+        // largest of chunks w, w+16, ... by a bitwise search over the key (16
+        // keys per lane, one warp sum per bit).
+        const int F = (n - (nch - 1) * chunk_len) >= kTopK ? nch : nch - 1;
+        uint32_t Lm = 0xffffffffu;
+        if (F >= 1) {
+            const int mth = (kTopK + F - 1) / F;
+            const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+            for (int c = warp; c < F; c += kTkThreads / 32) {
+                uint32_t kk[16];
+                const uint4 *src = reinterpret_cast<const uint4 *>(keys + (int64_t)c * kTopK) + lane * 4;
+#pragma unroll
+                for (int v = 0; v < 4; v++) {
+                    const uint4 x = src[v];
+                    kk[4 * v] = x.x; kk[4 * v + 1] = x.y; kk[4 * v + 2] = x.z; kk[4 * v + 3] = x.w;
+                }
+                uint32_t Tc = 0;
+#pragma unroll 1
+                for (int bit = 31; bit >= 0; bit--) {
+                    const uint32_t cand = Tc | (1u << bit);
+                    int cnt = 0;
+#pragma unroll
+                    for (int j = 0; j < 16; j++) cnt += kk[j] >= cand ? 1 : 0;
+                    if (__reduce_add_sync(0xffffffffu, (unsigned)cnt) >= (unsigned)mth) Tc = cand;
+                }
+                Lm = min(Lm, Tc);
+            }
+        } else {
+            Lm = 0;
+        }
         uint32_t lneg = ~L;
-        block_minmax(lneg, kmax, sh);     // min of ~L is ~(max of L)
+        block_minmax<kTkThreads>(lneg, kmax, sh);     // min of ~L is ~(max of L)
         L = ~lneg;
-        if (total <= kTk2Smem) {
-            // Thread i holds candidates [32i, 32i+32): all loads in flight at
-            // once, then the survivors (keys >= L) are compacted in order into
-            // shared memory with one block scan.
-            constexpr int kPer = kTk2Smem / kTkThreads;    // 32
-            static_assert(kPer % 4 == 0, "16-byte loads");
-            const int i0 = threadIdx.x * kPer;
+        uint32_t dummy = 0;
+        block_minmax<kTkThreads>(Lm, dummy, sh);
+        L = max(L, Lm);
+        // Batches of 512 x 32 candidates: thread i of a batch holds candidates
+        // [32i, 32i+32) (all loads in flight at once); the survivors (keys >= L)
+        // are appended in order to shared memory with one block scan per batch.
+        // Rows whose survivors overflow the buffer select straight from the
+        // workspace.
+        constexpr int kPer = 32;
+        constexpr int kBatch = kTkThreads * kPer;
+        uint32_t n_surv = 0;
+        bool fits = true;
+#pragma unroll 1
+        for (int b0 = 0; b0 < total; b0 += kBatch) {
+            const int i0 = b0 + threadIdx.x * kPer;
             uint32_t kk[kPer];
             int32_t ii[kPer];
 #pragma unroll
@@ -384,7 +222,11 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
 #pragma unroll
             for (int j = 0; j < kPer; j++) mine += (i0 + j < total && kk[j] >= L) ? 1u : 0u;
             uint32_t surv;
-            uint32_t pos = block_excl_scan(mine, &surv, sh);
+            uint32_t pos = n_surv + block_excl_scan<kTkThreads>(mine, &surv, sh);
+            if (n_surv + surv > (uint32_t)kTk2Smem) {      // uniform over the block
+                fits = false;
+                break;
+            }
 #pragma unroll
             for (int j = 0; j < kPer; j++) {
                 if (i0 + j < total && kk[j] >= L) {
@@ -393,17 +235,20 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
                     pos++;
                 }
             }
-            __syncthreads();
+            n_surv += surv;
+        }
+        __syncthreads();
+        if (fits) {
             keys = skeys;
             idx = sidx;
-            m = (int)surv;
+            m = (int)n_surv;
         }
-        radix_threshold(keys, m, K, L, kmax, sh, &T, &need_eq);
+        radix_threshold<kTkThreads>(keys, m, K, L, kmax, sh, &T, &need_eq);
     }
     const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
     int32_t *op = out_phys + (int64_t)t * kTopK;
     int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
-    ordered_compact(keys, m, T, need_eq, sh, [&](int pos, int i, uint32_t) {
+    ordered_compact<kTkThreads>(keys, m, T, need_eq, sh, [&](int pos, int i, uint32_t) {
         const int32_t s = idx[i];
         const int32_t page = pt_row[s / kC4Page];
         const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
@@ -448,14 +293,19 @@ cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
                                                  ck, ci, info, a.status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    return launch_topk_stage2(a, mc, kTkChunk, ck, ci, info, s);
+}
+
+cudaError_t launch_topk_stage2(const TopkArgs &a, int max_chunks, int chunk_len,
+                               const uint32_t *cand_key, const int32_t *cand_idx,
+                               const uint2 *chunk_info, cudaStream_t s) {
     const size_t smem2 = kTkKeysOffset + kTk2Smem * (sizeof(uint32_t) + sizeof(int32_t));
     static int done2[64] = {0};
-    e = ensure_max_smem((const void *)topk_stage2_kernel, (int)smem2, done2);
+    cudaError_t e = ensure_max_smem((const void *)topk_stage2_kernel, (int)smem2, done2);
     if (e != cudaSuccess) return e;
-    launch_k(topk_stage2_kernel, a.num_q, kTkThreads, smem2, s, a.c4_seq_lens, a.bs, a.cu_q, a.q_pos,
-                                                      a.max_c4_len, a.page_table, a.pt_stride,
-                                                      a.num_slots, mc, ck, ci, info,
-                                                      a.out_phys, a.out_raw, a.status);
+    launch_k(topk_stage2_kernel, a.num_q, kTkThreads, smem2, s, a.c4_seq_lens, a.bs, a.cu_q,
+             a.q_pos, a.max_c4_len, a.page_table, a.pt_stride, a.num_slots, max_chunks, chunk_len,
+             cand_key, cand_idx, chunk_info, a.out_phys, a.out_raw, a.status);
     return cudaGetLastError();
 }
 

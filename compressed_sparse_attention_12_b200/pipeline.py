@@ -115,6 +115,10 @@ class CsaBatch:
         self.raw_indices = torch.empty((nq, csa.TOPK), dtype=torch.int32, device=dev)
         self.topk_ws = torch.empty(max(1, csa.csa_topk512_workspace_size(nq, self.max_c4)),
                                    dtype=torch.uint8, device=dev)
+        self.fused_ws = torch.empty(
+            max(1, csa.csa_indexer_topk512_workspace_size(nq, w.bs, w.idx_heads, w.idx_dim,
+                                                          self.idx_fmt, self.max_c4)),
+            dtype=torch.uint8, device=dev)
         self.decode = bool((w.q_lens <= 8).all())
         self.attn_ws = torch.empty(
             max(1, csa.csa_sparse_mqa_workspace_size(nq, w.heads, w.window, self.decode)),
@@ -154,6 +158,22 @@ class CsaBatch:
                                self.page_table, self.c4_lens, self.cu_q, self.q_pos, self.max_c4,
                                self.logits, status=self.status, stream=stream)
 
+    def quantise_q(self, stream=None):
+        csa.csa_hadamard_quant(self.q_idx, self.idx_fmt, self.q_codes, self.q_bsc, self.q_scales,
+                               w_in=self.w_head, w_out=self.w_fold, status=self.status,
+                               stream=stream)
+
+    def index_select(self, stream=None):
+        """Indexer logits and top-512 in one call (the indexer CTAs select their
+        own chunks; see csa_indexer_topk512)."""
+        w = self.w
+        self.quantise_q(stream)
+        csa.csa_indexer_topk512(self.q_codes, self.q_bsc, self.w_fold, w.idx_heads, w.idx_dim,
+                                self.idx_fmt, self.k_codes, self.k_bsc, self.k_scales,
+                                self.page_table, self.c4_lens, self.cu_q, self.q_pos, self.max_c4,
+                                self.logits, self.indices, self.raw_indices, self.fused_ws,
+                                num_slots=self.c4_slots_n, status=self.status, stream=stream)
+
     def select(self, stream=None):
         csa.csa_topk512_page_transform(self.logits, self.c4_lens, self.cu_q, self.q_pos,
                                        self.page_table, self.c4_slots_n, self.max_c4,
@@ -166,9 +186,12 @@ class CsaBatch:
            self.seq_lens, self.cu_q, self.q_pos, self.w.window, self.sm_scale, self.out,
            self.lse, self.attn_ws, status=self.status, stream=stream)
 
-    def step(self, stream=None):
+    def step(self, stream=None, fused=True):
         self.compress(stream)
-        self.index(stream)
-        self.select(stream)
+        if fused:
+            self.index_select(stream)
+        else:
+            self.index(stream)
+            self.select(stream)
         self.attend(stream)
         return self.out

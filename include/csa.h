@@ -258,6 +258,70 @@ csa_status_t csa_topk512_page_transform_noalloc(const float *logits, int64_t log
                                                 void *stream);
 
 /*
+ * csa_indexer_topk512 -- steps 2 and 3 in one call: the indexer logits of
+ * csa_indexer_logits followed by the selection and page transform of
+ * csa_topk512_page_transform, with the same arguments and the same results
+ * (logits, c4_sparse_page_indices and raw_indices are those the two calls
+ * would write, bit for bit).  Where the tensor-core indexer applies (index dim
+ * 64 or 128, 16-byte aligned key codes, num_slots a positive multiple of 64),
+ * each indexer CTA selects the top-512 of its own chunk of keys right after
+ * computing them (the logits come back from L2 into the CTA's drained
+ * shared-memory stages), and one row-level merge follows: the separate
+ * chunk-selection launch and its re-read of the logits disappear.  Where rows
+ * are cut into pieces longer than 64 key tiles (many query rows per request,
+ * as in chunked prefill) the call runs the two separate steps instead.  This
+ * fusion is the design's own step beyond the pages, which keep the indexer and
+ * topk_transform_512 as separate operations ("Token 的一生" §3.2).
+ *   logits       [num_q, logits_stride] fp32, written (logits_stride >= max_c4_len)
+ *   workspace    >= csa_indexer_topk512_workspace_size(num_q, bs, idx_heads,
+ *                   idx_dim, fmt, max_c4_len) bytes (the size depends on the
+ *                   current device's SM count; query it on the device that runs)
+ * Errors as for the two separate calls.
+ */
+size_t csa_indexer_topk512_workspace_size(int32_t num_q, int32_t bs, int32_t idx_heads,
+                                          int32_t idx_dim, int32_t fmt, int32_t max_c4_len);
+csa_status_t csa_indexer_topk512(const void *q_codes, const uint8_t *q_block_scales,
+                                 const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                 int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                 const uint8_t *k_block_scales, const float *k_scales,
+                                 int64_t num_slots, const int32_t *page_table,
+                                 int32_t page_table_stride, const int32_t *c4_seq_lens, int32_t bs,
+                                 const int32_t *cu_q, const int32_t *q_pos, int32_t max_c4_len,
+                                 int32_t c4_page_size, float *logits, int64_t logits_stride,
+                                 int32_t *c4_sparse_page_indices, int32_t *raw_indices,
+                                 void *workspace, size_t workspace_bytes, int32_t *status,
+                                 void *stream);
+
+/*
+ * csa_indexer_select + csa_topk512_merge -- the two launches of
+ * csa_indexer_topk512 as separate calls (same arguments, same results), for
+ * callers that schedule or time them apart.  csa_indexer_select writes the
+ * logits and, in `workspace`, each chunk's top-512 candidates; it returns
+ * CSA_ERR_UNSUPPORTED (launching nothing) where csa_indexer_topk512 would not
+ * fuse -- use csa_indexer_logits + csa_topk512_page_transform there.
+ * csa_topk512_merge reads that workspace: it must get the same shape arguments
+ * (num_q, idx_heads, idx_dim, fmt, bs, max_c4_len), the same device and the
+ * workspace untouched in between.
+ */
+csa_status_t csa_indexer_select(const void *q_codes, const uint8_t *q_block_scales,
+                                const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                const uint8_t *k_block_scales, const float *k_scales,
+                                int64_t num_slots, const int32_t *page_table,
+                                int32_t page_table_stride, const int32_t *c4_seq_lens, int32_t bs,
+                                const int32_t *cu_q, const int32_t *q_pos, int32_t max_c4_len,
+                                float *logits, int64_t logits_stride, void *workspace,
+                                size_t workspace_bytes, int32_t *status, void *stream);
+csa_status_t csa_topk512_merge(int32_t num_q, int32_t idx_heads, int32_t idx_dim, int32_t fmt,
+                               const int32_t *c4_seq_lens, int32_t bs, const int32_t *cu_q,
+                               const int32_t *q_pos, const int32_t *page_table,
+                               int32_t page_table_stride, int64_t num_slots,
+                               int32_t c4_page_size, int32_t max_c4_len,
+                               int32_t *c4_sparse_page_indices, int32_t *raw_indices,
+                               const void *workspace, size_t workspace_bytes, int32_t *status,
+                               void *stream);
+
+/*
  * csa_sparse_mqa_decode / csa_sparse_mqa_prefill -- step 4, sparse attention
  * over the selected compressed rows joined with the sliding window of raw
  * rows under ONE softmax ([T] §1; [H] "Compressed Sparse Attention（CSA）").
