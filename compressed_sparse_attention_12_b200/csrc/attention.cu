@@ -220,8 +220,9 @@ __device__ __forceinline__ void issue_loads8(const AttnArgs &a, int lt, int st, 
     cp_async_commit();
 }
 
-// FP8 -> fp16 expansion of staging `st` (local tile `lt`): E4M3 codes exactly
-// (one conversion per two codes); RoPE values times a per-row power of two
+// FP8 -> fp16 expansion of staging `st` (local tile `lt`): E4M3 codes exactly,
+// as value x 2^-8 (a bit move, the 2^8 goes into the row scales); RoPE values
+// times a per-row power of two
 // that brings the row's largest magnitude into [2^13, 2^14), which converts
 // exactly every bf16 value above 2^-30 of that maximum; block scales kept aside.
 template <int G>
@@ -259,10 +260,11 @@ __device__ __forceinline__ void expand8(int lt, int st, AtSmem8<G> &sm) {
         if (c == 0) {
             const float4 sc = valid ? *reinterpret_cast<const float4 *>(row + 512)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-            sm.rscale[st][r][0] = sc.x;
-            sm.rscale[st][r][1] = sc.y;
-            sm.rscale[st][r][2] = sc.z;
-            sm.rscale[st][r][3] = sc.w;
+            // the tile holds code values x 2^-8 (see below): the scales take the 2^8
+            sm.rscale[st][r][0] = sc.x * 256.0f;
+            sm.rscale[st][r][1] = sc.y * 256.0f;
+            sm.rscale[st][r][2] = sc.z * 256.0f;
+            sm.rscale[st][r][3] = sc.w * 256.0f;
             sm.rope_mul[st][r] = valid ? 1.0f / m : 0.0f;
         }
     }
@@ -275,11 +277,13 @@ __device__ __forceinline__ void expand8(int lt, int st, AtSmem8<G> &sm) {
             const uint32_t w[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
             for (int j = 0; j < 4; j++) {
-                uint32_t lo, hi;
-                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"((uint16_t)(w[j] & 0xFFFF)));
-                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"((uint16_t)(w[j] >> 16)));
-                o[2 * j] = lo;
-                o[2 * j + 1] = hi;
+                // E4M3 -> fp16 by moving the sign and the 7 exponent/mantissa bits:
+                // exact, value x 2^-8 (normal and subnormal codes alike), on the
+                // integer pipes (byte permute, shift, masked merge)
+                const uint32_t tl = __byte_perm(w[j], 0u, 0x1404);
+                const uint32_t th = __byte_perm(w[j], 0u, 0x3424);
+                o[2 * j] = (tl & 0x80008000u) | ((tl >> 1) & 0x3F803F80u);
+                o[2 * j + 1] = (th & 0x80008000u) | ((th >> 1) & 0x3F803F80u);
             }
         }
         *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
