@@ -400,6 +400,36 @@ long oracle_c4_compress(const double *x, const double *gate, const double *bias,
     return nblk;
 }
 
+/* HCA compressor ([H] "Heavily Compressed Attention（HCA）"): the same
+ * softmax-gated pooling with a per-position bias over blocks of `ratio` raw
+ * rows (about 128 for HCA).  Block j pools rows ratio*j .. ratio*j+ratio-1 and
+ * is produced only once all are present, so floor(T/ratio) rows come out.
+ * Per channel c:  alpha_i = softmax_i(g[ratio*j+i][c] + bias[i][c]),
+ *                 y[j][c] = sum_i alpha_i x[ratio*j+i][c]. */
+long oracle_pool_compress(const double *x, const double *gate, const double *bias,
+                          long T, int D, int ratio, double *y)
+{
+    long nblk = T / ratio, j;
+#pragma omp parallel for schedule(static)
+    for (j = 0; j < nblk; j++) {
+        int c, i;
+        for (c = 0; c < D; c++) {
+            double m = -INFINITY, Z = 0.0, acc = 0.0;
+            for (i = 0; i < ratio; i++) {
+                double z = gate[(ratio * j + i) * (long)D + c] + bias[(long)i * D + c];
+                if (z > m) m = z;
+            }
+            for (i = 0; i < ratio; i++) {
+                double e = exp(gate[(ratio * j + i) * (long)D + c] + bias[(long)i * D + c] - m);
+                Z += e;
+                acc += e * x[(ratio * j + i) * (long)D + c];
+            }
+            y[j * D + c] = acc / Z;
+        }
+    }
+    return nblk;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Step 2: indexer scores ([T] §1, §3.1; [H] "Compressed Sparse Attention"). */
 /* ------------------------------------------------------------------------ */

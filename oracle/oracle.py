@@ -99,6 +99,8 @@ def _declare(L):
     L.oracle_kv_decode_rows.argtypes = [_P, _L, _I, _P]
     L.oracle_c4_compress.restype = _L
     L.oracle_c4_compress.argtypes = [_P, _P, _P, _L, _I, _P]
+    L.oracle_pool_compress.restype = _L
+    L.oracle_pool_compress.argtypes = [_P, _P, _P, _L, _I, _I, _P]
     L.oracle_indexer_logits.restype = None
     L.oracle_indexer_logits.argtypes = [_P, _P, _L, _I, _I, _P, _P, _P, _L]
     L.oracle_topk_transform.restype = _L
@@ -316,6 +318,52 @@ def c4_compress(x: np.ndarray, gate: np.ndarray, bias: np.ndarray) -> np.ndarray
     n = lib().oracle_c4_compress(_ptr(x), _ptr(gate), _ptr(bias), T, D, _ptr(y))
     assert n == T // 4
     return y
+
+
+HCA_RATIO = 128         # [H] HCA: "about 128x" compression
+HCA_PAGE_SIZE = PAGE_SIZE // HCA_RATIO   # compressed rows per 256-token page (reading)
+
+
+def pool_compress(x: np.ndarray, gate: np.ndarray, bias: np.ndarray, ratio: int) -> np.ndarray:
+    """Softmax-gated pooling over blocks of `ratio` raw rows with a per-position
+    bias; the C4 compressor is ratio 4, the HCA compressor ([H] HCA) ratio 128.
+    Returns [floor(T/ratio), D]."""
+    x = _c(x, np.float64)
+    gate = _c(gate, np.float64)
+    bias = _c(bias, np.float64)
+    T, D = x.shape
+    assert gate.shape == (T, D) and bias.shape == (ratio, D)
+    y = np.empty((T // ratio, D), dtype=np.float64)
+    n = lib().oracle_pool_compress(_ptr(x), _ptr(gate), _ptr(bias), T, D, int(ratio), _ptr(y))
+    assert n == T // ratio
+    return y
+
+
+def hca_compress(x: np.ndarray, gate: np.ndarray, bias: np.ndarray) -> np.ndarray:
+    """HCA compressor ([H] HCA): pool_compress with ratio 128."""
+    return pool_compress(x, gate, bias, HCA_RATIO)
+
+
+def hca_len(L: int) -> int:
+    """HCA compressed length of a request with L raw tokens: floor(L/128)."""
+    return L // HCA_RATIO
+
+
+def hca_visible(pos: int) -> int:
+    """HCA blocks visible to a query at raw position pos: floor((pos+1)/128)."""
+    return (pos + 1) // HCA_RATIO
+
+
+def hca_attention(q: np.ndarray, hca_rows: np.ndarray, window_rows: np.ndarray,
+                  sm_scale: float):
+    """HCA attention ([H] HCA: dense attention over the compressed blocks) for
+    one query: every visible compressed row joined with the raw window rows
+    under one softmax (the window is a reading: the pages describe it for CSA
+    only; window 0 gives the compressed rows alone).  Returns (out [H, 512],
+    lse [H])."""
+    rows = np.concatenate([np.asarray(hca_rows, np.float64).reshape(-1, KV_DIM),
+                           np.asarray(window_rows, np.float64).reshape(-1, KV_DIM)])
+    return sparse_attention(q, rows, sm_scale)
 
 
 def c4_len(L: int) -> int:
