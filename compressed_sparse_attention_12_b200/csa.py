@@ -23,6 +23,7 @@ CSA_OUT_KV_BF16, CSA_OUT_KV_FP8 = 0, 1
 CSA_OUT_INDEX_BF16, CSA_OUT_INDEX_FP8, CSA_OUT_INDEX_FP4 = 2, 3, 4
 TOPK, PAGE_SIZE, C4_PAGE_SIZE, KV_DIM, KV_LATENT = 512, 256, 64, 576, 512
 TOPK_NOALLOC_MAX_BYTES = 16 << 20
+HCA_RATIO, HCA_PAGE_SIZE, HCA_MAX_ROWS = 128, 2, 16 * 48 * 32
 
 FMT = {"bf16": CSA_FMT_BF16, "fp8": CSA_FMT_FP8, "fp4": CSA_FMT_FP4}
 
@@ -62,6 +63,12 @@ _SIGS = {
                                           _P, _P]),
     "csa_topk512_merge": (ctypes.c_int, [_I32, _I32, _I32, _I32, _P, _I32, _P, _P, _P, _I32,
                                          _I64, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
+    "csa_hca_compress": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _I64, _P, _I32, _P, _I32,
+                                        _I32, _P, _I64, _P, _P]),
+    "csa_hca_attention_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
+    "csa_hca_attention": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _I32, _P,
+                                         _I32, _P, _P, _I32, _I32, _F, _I32, _P, _P, _P, _SZ,
+                                         _P, _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
     "csa_sparse_mqa_decode": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _P,
                                              _I32, _P, _I32, _P, _P, _I32, _F, _P, _P, _P, _SZ,
@@ -268,3 +275,35 @@ def csa_sparse_mqa_decode(*args, **kw):
 
 def csa_sparse_mqa_prefill(*args, **kw):
     _sparse_mqa("csa_sparse_mqa_prefill", False, *args, **kw)
+
+
+def csa_hca_compress(x, gate, bias, cu_x, start_pos, max_rows_per_req, page_table, out_kind, out,
+                     num_slots=None, status=None, stream=None):
+    """HCA compressor: softmax-gated pooling of blocks of 128 raw rows (see include/csa.h)."""
+    bs = start_pos.shape[0]
+    _check("csa_hca_compress", lib().csa_hca_compress(
+        _ptr(x), _ptr(gate), _ptr(bias), x.shape[1], bs, _ptr(cu_x), x.shape[0], _ptr(start_pos),
+        int(max_rows_per_req), _ptr(page_table), page_table.shape[1], out_kind, _ptr(out),
+        out.shape[0] if num_slots is None else int(num_slots), _ptr(status), _stream(stream)))
+
+
+def csa_hca_attention_workspace_size(num_q, heads, window, decode, max_hca_len) -> int:
+    return lib().csa_hca_attention_workspace_size(num_q, heads, window, int(bool(decode)),
+                                                  max_hca_len)
+
+
+def csa_hca_attention(q, hca_cache, raw_cache, kv_fmt, page_table, seq_lens, cu_q, q_pos,
+                      max_hca_len, window, sm_scale, decode, out, lse=None, workspace=None,
+                      status=None, stream=None):
+    """Dense attention over every visible HCA row plus the raw window (include/csa.h)."""
+    num_q, heads = q.shape[0], q.shape[1]
+    if workspace is None:
+        n = csa_hca_attention_workspace_size(num_q, heads, window, decode, max_hca_len)
+        workspace = torch.empty(max(1, n), dtype=torch.uint8, device=q.device)
+    _check("csa_hca_attention", lib().csa_hca_attention(
+        _ptr(q), num_q, heads, _ptr(hca_cache), _ptr(raw_cache), kv_fmt,
+        hca_cache.shape[0] if hca_cache is not None else 0,
+        raw_cache.shape[0] if raw_cache is not None else 0, _ptr(page_table), page_table.shape[1],
+        _ptr(seq_lens), seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos), int(max_hca_len),
+        int(window), float(sm_scale), int(bool(decode)), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)))

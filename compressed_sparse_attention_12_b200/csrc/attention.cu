@@ -91,6 +91,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 struct AtQuery {
     int b, p, nw;        // request, raw position, window rows
+    int nsel;            // rows before the window (512 selected, or the HCA rows)
 };
 
 __device__ __forceinline__ AtQuery at_query(const AttnArgs &a, int t) {
@@ -103,6 +104,15 @@ __device__ __forceinline__ AtQuery at_query(const AttnArgs &a, int t) {
     q.b = lo;
     q.p = a.q_pos ? a.q_pos[t] : a.seq_lens[lo] - 1;
     q.nw = max(0, min(a.window, q.p + 1));
+    q.nsel = kTopK;
+    if (a.dense_ratio > 0) {
+        const int len = a.seq_lens[lo] / a.dense_ratio;
+        q.nsel = max(0, min(len, (q.p + 1) / a.dense_ratio));
+        if (q.nsel > a.max_sel) {
+            report(a.status, CSA_ERR_BOUNDS);
+            q.nsel = a.max_sel;
+        }
+    }
     return q;
 }
 
@@ -111,7 +121,20 @@ __device__ __forceinline__ AtQuery at_query(const AttnArgs &a, int t) {
 __device__ __forceinline__ int32_t row_slot(const AttnArgs &a, const AtQuery &qq, int t, int r,
                                             int32_t *raw) {
     *raw = 0;
-    if (r < kTopK) {
+    if (r < qq.nsel) {
+        if (a.dense_ratio > 0) {
+            // HCA: every visible compressed row, kPage / ratio of them per page
+            const int rpp = kPage / a.dense_ratio;
+            const int32_t page = r / rpp < a.pt_stride
+                                     ? a.page_table[(int64_t)qq.b * a.pt_stride + r / rpp]
+                                     : -1;
+            const int64_t slot = (int64_t)page * rpp + r % rpp;
+            if (page < 0 || slot >= a.num_c4_slots) {
+                report(a.status, CSA_ERR_BOUNDS);
+                return -1;
+            }
+            return (int32_t)slot;
+        }
         int32_t slot = a.idx[(int64_t)t * kTopK + r];
         if (slot >= a.num_c4_slots) {
             report(a.status, CSA_ERR_BOUNDS);
@@ -119,8 +142,8 @@ __device__ __forceinline__ int32_t row_slot(const AttnArgs &a, const AtQuery &qq
         }
         return slot < 0 ? -1 : slot;
     }
-    if (r - kTopK >= qq.nw) return -1;
-    const int pos = qq.p - qq.nw + 1 + (r - kTopK);
+    if (r - qq.nsel >= qq.nw) return -1;
+    const int pos = qq.p - qq.nw + 1 + (r - qq.nsel);
     const int32_t page = pos / kPage < a.pt_stride
                              ? a.page_table[(int64_t)qq.b * a.pt_stride + pos / kPage]
                              : -1;
@@ -316,7 +339,7 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
     const int gq = lane >> 2, tq = lane & 3;
     const int hg = blockIdx.y * G + grp;          // global 16-head group of this warp
     const AtQuery qq = at_query(a, t);
-    const int n_rows = kTopK + qq.nw;
+    const int n_rows = qq.nsel + qq.nw;
     const int tile0 = sp * tiles_per_split;
     const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
 
@@ -581,7 +604,7 @@ sparse_mqa_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gq = lane >> 2, tq = lane & 3;
     const AtQuery qq = at_query(a, t);
-    const int n_rows = kTopK + qq.nw;
+    const int n_rows = qq.nsel + qq.nw;
     const int tile0 = sp * tiles_per_split;
     const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
 
@@ -875,7 +898,9 @@ sparse_mqa_combine_kernel(const AttnArgs a, int splits, const float *part_o,
             L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
-static int at_tiles(int window) { return (kTopK + window + kAtRows - 1) / kAtRows; }
+static int at_tiles(int window, int max_sel = kTopK) {
+    return (max_sel + window + kAtRows - 1) / kAtRows;
+}
 
 // Head groups (of 16) per CTA: the FP8 kernel takes 64 heads at a time when
 // the head count allows, the BF16 kernel one group.
@@ -883,23 +908,27 @@ static int at_groups(int heads, int kv_fmt) {
     return kv_fmt == CSA_FMT_FP8 && heads % (4 * kAtHeads) == 0 ? 4 : 1;
 }
 
-static int at_splits(int num_q, int heads, int window, bool decode, int groups) {
-    if (!decode) return 1;
+static int at_splits(int num_q, int heads, int window, bool decode, int groups,
+                     int max_sel = kTopK) {
+    const int nt = at_tiles(window, max_sel);
+    // a split holds at most kAtMaxTiles tiles (its row slots live in shared memory)
+    const int need = (nt + kAtMaxTiles - 1) / kAtMaxTiles;
+    if (!decode) return need;
     // split each query's rows so that the grid fills one wave of the 148 SMs
     // (two CTAs per SM with one head group, one CTA with four)
     const int per_sm = groups == 1 ? 2 : 1;
     const int ctas = num_q * (heads / (kAtHeads * groups));
     int sp = (per_sm * 148) / ctas;
     sp = sp < 1 ? 1 : sp;
-    const int nt = at_tiles(window);
     sp = sp > kAtMaxSplits ? kAtMaxSplits : sp;
-    return sp > nt ? nt : sp;
+    sp = sp > nt ? nt : sp;
+    return sp < need ? need : sp;
 }
 
-size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode) {
+size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode, int max_sel) {
     // the larger of the two formats' needs
-    int sp = at_splits(num_q, heads, window, decode, at_groups(heads, CSA_FMT_BF16));
-    const int sp8 = at_splits(num_q, heads, window, decode, at_groups(heads, CSA_FMT_FP8));
+    int sp = at_splits(num_q, heads, window, decode, at_groups(heads, CSA_FMT_BF16), max_sel);
+    const int sp8 = at_splits(num_q, heads, window, decode, at_groups(heads, CSA_FMT_FP8), max_sel);
     sp = sp8 > sp ? sp8 : sp;
     if (sp == 1) return 0;
     return (size_t)num_q * heads * sp * (kLatent + 2) * sizeof(float);
@@ -919,8 +948,9 @@ static cudaError_t launch_fp8(const AttnArgs &a, dim3 grid, int sp, int tps, flo
 cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s) {
     if (a.num_q == 0) return cudaSuccess;
     const int groups = at_groups(a.heads, a.kv_fmt);
-    const int sp = at_splits(a.num_q, a.heads, a.window, decode, groups);
-    const int nt = at_tiles(a.window);
+    const int max_sel = a.dense_ratio > 0 ? a.max_sel : kTopK;
+    const int sp = at_splits(a.num_q, a.heads, a.window, decode, groups, max_sel);
+    const int nt = at_tiles(a.window, max_sel);
     const int tps = (nt + sp - 1) / sp;
     float *po = nullptr, *pml = nullptr;
     if (sp > 1) {

@@ -17,6 +17,8 @@ namespace csa {
 constexpr int kTopK = 512;
 constexpr int kPage = 256;       // raw tokens per page
 constexpr int kC4Page = 64;      // compressed rows per page
+constexpr int kHcaRatio = 128;   // HCA: raw rows per compressed row
+constexpr int kHcaPage = 2;      // HCA compressed rows per 256-token page
 constexpr int kKvDim = 576;
 constexpr int kLatent = 512;
 constexpr int kRope = 64;

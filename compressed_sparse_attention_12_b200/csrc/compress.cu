@@ -198,34 +198,37 @@ __device__ __forceinline__ float pool4(const float (&x)[4], const float (&z)[4])
 // compressed index.
 __device__ __forceinline__ int64_t compress_row(int b, int blk, const int32_t *cu_x,
                                                 const int32_t *start_pos, int max_rows,
-                                                int32_t *status, bool leader, int32_t *j) {
+                                                int32_t *status, bool leader, int32_t *j,
+                                                int ratio = 4) {
     const int32_t x0 = cu_x[b], n = cu_x[b + 1] - x0;
     const int32_t sp = start_pos[b];
-    if (n < 4) {                      // no complete block: nothing to compress
+    if (n < ratio) {                  // no complete block: nothing to compress
         if (n < 0 && leader && blk == 0) report(status, CSA_ERR_BOUNDS);
         return -1;
     }
-    if (sp < 0 || (sp & 3) != 0) {
+    if (sp < 0 || (sp % ratio) != 0) {
         if (leader && blk == 0) report(status, CSA_ERR_BOUNDS);
         return -1;
     }
     if (n > max_rows && leader && blk == 0) report(status, CSA_ERR_BOUNDS);
-    const int nblk = min(n, max_rows) / 4;
+    const int nblk = min(n, max_rows) / ratio;
     if (blk >= nblk) return -1;
-    *j = sp / 4 + blk;
-    return (int64_t)x0 + 4 * blk;
+    *j = sp / ratio + blk;
+    return (int64_t)x0 + (int64_t)ratio * blk;
 }
 
-// Compressed slot of compressed index j of request b, or -1 (reported).
+// Compressed slot of compressed index j of request b (rows_per_page compressed
+// rows per 256-token page), or -1 (reported).
 __device__ __forceinline__ int64_t compress_slot(int b, int32_t j, const int32_t *page_table,
                                                  int pt_stride, int64_t num_slots,
-                                                 int32_t *status, bool leader) {
-    if (j / kC4Page >= pt_stride) {
+                                                 int32_t *status, bool leader,
+                                                 int rows_per_page = kC4Page) {
+    if (j / rows_per_page >= pt_stride) {
         if (leader) report(status, CSA_ERR_BOUNDS);
         return -1;
     }
-    const int32_t page = page_table[(int64_t)b * pt_stride + j / kC4Page];
-    const int64_t slot = (int64_t)page * kC4Page + j % kC4Page;
+    const int32_t page = page_table[(int64_t)b * pt_stride + j / rows_per_page];
+    const int64_t slot = (int64_t)page * rows_per_page + j % rows_per_page;
     if (page < 0 || slot >= num_slots) {
         if (leader) report(status, CSA_ERR_BOUNDS);
         return -1;
@@ -271,6 +274,63 @@ compress_kv_kernel(const float *__restrict__ x, const float *__restrict__ gate,
         CSA_POOL_LANE(w)
 #undef CSA_POOL_LANE
     }
+    const int row_bytes = fmt == CSA_FMT_FP8 ? kFp8RowBytes : kBf16RowBytes;
+    write_kv_row(y, warp, lane, fmt, out + slot * row_bytes);
+}
+
+// HCA: one compressed row of 128 raw rows per CTA of 160 threads (4 channels
+// per active thread); the softmax over the block runs online (running maximum,
+// rescaled sum and weighted sum), four rows in flight at a time.
+__global__ void __launch_bounds__(kKvRowThreads)
+compress_hca_kernel(const float *__restrict__ x, const float *__restrict__ gate,
+                    const float *__restrict__ bias, const int32_t *cu_x,
+                    const int32_t *start_pos, int max_rows, const int32_t *page_table,
+                    int pt_stride, int fmt, uint8_t *out, int64_t num_slots, int32_t *status) {
+    pdl_begin();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t j = 0;
+    const int64_t row0 = compress_row(blockIdx.y, blockIdx.x, cu_x, start_pos, max_rows, status,
+                                      threadIdx.x == 0, &j, kHcaRatio);
+    if (row0 < 0) return;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (kv_active(warp, lane)) {
+        const int c = kv_channel(warp, lane);
+        float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float Z[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int i0 = 0; i0 < kHcaRatio; i0 += 4) {
+            float4 xv[4], zv[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                xv[i] = *reinterpret_cast<const float4 *>(x + (row0 + i0 + i) * kKvDim + c);
+                const float4 g = *reinterpret_cast<const float4 *>(gate + (row0 + i0 + i) * kKvDim + c);
+                const float4 bb = *reinterpret_cast<const float4 *>(bias + (i0 + i) * kKvDim + c);
+                zv[i] = make_float4(g.x + bb.x, g.y + bb.y, g.z + bb.z, g.w + bb.w);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float zz[4] = {zv[i].x, zv[i].y, zv[i].z, zv[i].w};
+                const float xx[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    if (zz[k] > m[k]) {
+                        const float sc = expf(m[k] - zz[k]);     // 0 on the first row
+                        Z[k] = Z[k] * sc + 1.0f;
+                        acc[k] = acc[k] * sc + xx[k];
+                        m[k] = zz[k];
+                    } else {
+                        const float e = expf(zz[k] - m[k]);
+                        Z[k] += e;
+                        acc[k] = fmaf(e, xx[k], acc[k]);
+                    }
+                }
+            }
+        }
+        y = make_float4(acc[0] / Z[0], acc[1] / Z[1], acc[2] / Z[2], acc[3] / Z[3]);
+    }
+    const int64_t slot = compress_slot(blockIdx.y, j, page_table, pt_stride, num_slots, status,
+                                       threadIdx.x == 0, kHcaPage);
+    if (slot < 0) return;
     const int row_bytes = fmt == CSA_FMT_FP8 ? kFp8RowBytes : kBf16RowBytes;
     write_kv_row(y, warp, lane, fmt, out + slot * row_bytes);
 }
@@ -339,6 +399,18 @@ cudaError_t launch_hadamard_quant(const void *x, int x_dtype, int64_t rows, int 
     else if (x_dtype == CSA_FMT_BF16) CSA_HQ(4, uint16_t);
     else CSA_HQ(4, float);
 #undef CSA_HQ
+    return cudaGetLastError();
+}
+
+cudaError_t launch_hca_compress(const float *x, const float *gate, const float *bias, int bs,
+                                const int32_t *cu_x, const int32_t *start_pos, int max_rows,
+                                const int32_t *page_table, int pt_stride, int out_kind, void *out,
+                                int64_t num_slots, int32_t *status, cudaStream_t s) {
+    const int max_blocks = max_rows / kHcaRatio;
+    if (bs == 0 || max_blocks == 0) return cudaSuccess;
+    const int fmt = out_kind == CSA_OUT_KV_FP8 ? CSA_FMT_FP8 : CSA_FMT_BF16;
+    launch_k(compress_hca_kernel, dim3(max_blocks, bs), kKvRowThreads, 0, s, x, gate, bias, cu_x,
+             start_pos, max_rows, page_table, pt_stride, fmt, (uint8_t *)out, num_slots, status);
     return cudaGetLastError();
 }
 

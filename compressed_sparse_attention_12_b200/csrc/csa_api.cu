@@ -86,6 +86,25 @@ csa_status_t csa_c4_compress(const float *x, const float *gate, const float *bia
                                                num_slots, status, as_stream(stream)));
 }
 
+csa_status_t csa_hca_compress(const float *x, const float *gate, const float *bias,
+                              int32_t dim, int32_t bs, const int32_t *cu_x, int64_t total_rows,
+                              const int32_t *start_pos, int32_t max_rows_per_req,
+                              const int32_t *page_table, int32_t page_table_stride,
+                              int32_t out_kind, void *out, int64_t num_slots, int32_t *status,
+                              void *stream) {
+    if (bs < 0 || total_rows < 0 || max_rows_per_req < 0 || page_table_stride < 0)
+        return CSA_ERR_INVALID;
+    if (out_kind != CSA_OUT_KV_BF16 && out_kind != CSA_OUT_KV_FP8) return CSA_ERR_UNSUPPORTED;
+    if (dim != CSA_KV_DIM) return CSA_ERR_UNSUPPORTED;
+    if (bs == 0 || total_rows == 0 || max_rows_per_req < CSA_HCA_RATIO) return CSA_OK;
+    if (!x || !gate || !bias || !cu_x || !start_pos || !page_table || !out) return CSA_ERR_INVALID;
+    if (bs > 65535 || max_rows_per_req / CSA_HCA_RATIO > 2147483647) return CSA_ERR_UNSUPPORTED;
+    return cuda_status(csa::launch_hca_compress(x, gate, bias, bs, cu_x, start_pos,
+                                                max_rows_per_req, page_table, page_table_stride,
+                                                out_kind, out, num_slots, status,
+                                                as_stream(stream)));
+}
+
 csa_status_t csa_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
                                 int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
                                 void *codes, uint8_t *block_scales, float *scales,
@@ -321,22 +340,24 @@ static csa_status_t sparse_mqa(const void *q, int32_t num_q, int32_t heads,
                                const int32_t *seq_lens, int32_t bs, const int32_t *cu_q,
                                const int32_t *q_pos, int32_t window, float sm_scale, void *out,
                                float *lse, void *workspace, size_t workspace_bytes,
-                               int32_t *status, void *stream, bool decode) {
+                               int32_t *status, void *stream, bool decode, int dense_ratio = 0,
+                               int max_sel = 512) {
     if (num_q < 0 || bs < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
     if (!kv_fmt_ok(kv_fmt)) return CSA_ERR_UNSUPPORTED;
     if (heads != 16 && heads != 32 && heads != 64 && heads != 128) return CSA_ERR_UNSUPPORTED;
     if (window < 0 || window > 1024) return CSA_ERR_UNSUPPORTED;
     if (num_q == 0) return CSA_OK;
-    if (bs < 1 || !q || !idx || !page_table || !cu_q || !out || !seq_lens) return CSA_ERR_INVALID;
+    if (bs < 1 || !q || (!idx && dense_ratio == 0) || !page_table || !cu_q || !out || !seq_lens)
+        return CSA_ERR_INVALID;
     if (!c4_cache && num_c4_slots > 0) return CSA_ERR_INVALID;
     if (window > 0 && !raw_cache) return CSA_ERR_INVALID;
     if (!q_pos && num_q != bs) return CSA_ERR_INVALID;
-    const size_t need = csa::attn_workspace_bytes(num_q, heads, window, decode);
+    const size_t need = csa::attn_workspace_bytes(num_q, heads, window, decode, max_sel);
     if (need > 0 && (!workspace || workspace_bytes < need)) return CSA_ERR_WORKSPACE;
     if (num_q > 2147483647 / 2) return CSA_ERR_UNSUPPORTED;
     csa::AttnArgs a{q, num_q, heads, c4_cache, raw_cache, kv_fmt, num_c4_slots, num_raw_slots,
                     idx, page_table, page_table_stride, seq_lens, bs, cu_q, q_pos, window,
-                    sm_scale, out, lse, workspace, status};
+                    sm_scale, out, lse, workspace, status, dense_ratio, max_sel};
     return cuda_status(csa::launch_sparse_mqa(a, decode, as_stream(stream)));
 }
 
@@ -371,3 +392,26 @@ csa_status_t csa_sparse_mqa_prefill(const void *q, int32_t num_q, int32_t heads,
 }
 
 }  // extern "C"
+
+size_t csa_hca_attention_workspace_size(int32_t num_q, int32_t heads, int32_t window,
+                                        int32_t decode, int32_t max_hca_len) {
+    if (num_q <= 0 || heads <= 0 || max_hca_len < 0) return 0;
+    return csa::attn_workspace_bytes(num_q, heads, window, decode != 0, max_hca_len);
+}
+
+csa_status_t csa_hca_attention(const void *q, int32_t num_q, int32_t heads, const void *hca_cache,
+                               const void *raw_cache, int32_t kv_fmt, int64_t num_hca_slots,
+                               int64_t num_raw_slots, const int32_t *page_table,
+                               int32_t page_table_stride, const int32_t *seq_lens, int32_t bs,
+                               const int32_t *cu_q, const int32_t *q_pos, int32_t max_hca_len,
+                               int32_t window, float sm_scale, int32_t decode, void *out,
+                               float *lse, void *workspace, size_t workspace_bytes,
+                               int32_t *status, void *stream) {
+    if (max_hca_len < 0) return CSA_ERR_INVALID;
+    // at most 16 splits of 48 tiles of 32 rows per query
+    if (max_hca_len + window > CSA_HCA_MAX_ROWS) return CSA_ERR_UNSUPPORTED;
+    return sparse_mqa(q, num_q, heads, hca_cache, raw_cache, kv_fmt, num_hca_slots, num_raw_slots,
+                      nullptr, page_table, page_table_stride, seq_lens, bs, cu_q, q_pos, window,
+                      sm_scale, out, lse, workspace, workspace_bytes, status, stream, decode != 0,
+                      CSA_HCA_RATIO, max_hca_len);
+}

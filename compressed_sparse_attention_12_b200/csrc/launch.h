@@ -49,6 +49,11 @@ cudaError_t launch_hadamard_quant(const void *x, int x_dtype, int64_t rows, int 
                                   uint8_t *block_scales, float *scales, const float *w_in,
                                   float *w_out, int32_t *status, cudaStream_t s);
 
+cudaError_t launch_hca_compress(const float *x, const float *gate, const float *bias, int bs,
+                                const int32_t *cu_x, const int32_t *start_pos, int max_rows,
+                                const int32_t *page_table, int pt_stride, int out_kind, void *out,
+                                int64_t num_slots, int32_t *status, cudaStream_t s);
+
 cudaError_t launch_c4_compress(const float *x, const float *gate, const float *bias, int dim,
                                int bs, const int32_t *cu_x, const int32_t *start_pos,
                                int max_rows, const int32_t *page_table, int pt_stride,
@@ -138,8 +143,13 @@ struct AttnArgs {
     float *lse;
     void *workspace;
     int32_t *status;
+    // 0: the first rows of a query are its selected list idx[t][0..512).
+    // HCA (128): they are all its visible compressed rows s < (p+1)/128, read
+    // from c4_cache at page_table[b][s/2]*2 + s%2; max_sel bounds their count.
+    int dense_ratio;
+    int max_sel;
 };
-size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode);
+size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode, int max_sel = 512);
 cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s);
 
 }  // namespace csa

@@ -363,6 +363,53 @@ csa_status_t csa_sparse_mqa_prefill(const void *q, int32_t num_q, int32_t heads,
                                     void *out, float *lse, void *workspace,
                                     size_t workspace_bytes, int32_t *status, void *stream);
 
+/*
+ * HCA branch ("DeepSeek-V4 的交錯壓縮注意力（CSA/HCA）", section "Heavily
+ * Compressed Attention（HCA）": about 128x compression, then dense attention over
+ * the compressed blocks).  The design's next row beyond the CSA path.
+ *
+ * csa_hca_compress -- csa_c4_compress with blocks of CSA_HCA_RATIO = 128 raw
+ * rows: per channel, alpha_i = softmax_i(gate[128j+i] + bias[i]) over the
+ * block, row j = sum_i alpha_i x[128j+i], produced only for complete blocks.
+ *   bias         [128, 576] fp32
+ *   start_pos    per request, a multiple of 128
+ *   out          HCA KV cache, packed rows (out_kind CSA_OUT_KV_BF16 or _FP8, the
+ *                layouts of csa_kv_store); row j of request b at slot
+ *                page_table[b*stride + j/2]*2 + j%2 (CSA_HCA_PAGE_SIZE = 256/128
+ *                compressed rows per 256-token page; the same page table as
+ *                the raw cache)
+ *   num_slots    rows of `out`
+ * Other arguments and errors as csa_c4_compress.
+ *
+ * csa_hca_attention -- dense attention of each query over all its visible HCA
+ * rows s < floor((p+1)/128) (and s < floor(seq_len/128)) joined with the raw
+ * window [p-W+1, p] under one softmax (the window is this design's reading:
+ * the pages describe it for CSA; window 0 gives the compressed rows alone).
+ * Arguments as csa_sparse_mqa_decode without the index list, plus
+ *   max_hca_len  an upper bound of any query's visible HCA rows;
+ *                max_hca_len + window <= CSA_HCA_MAX_ROWS
+ *   decode       1: few query rows per request (rows split over CTAs), 0: prefill
+ *   workspace    >= csa_hca_attention_workspace_size(num_q, heads, window,
+ *                   decode, max_hca_len) bytes
+ */
+enum { CSA_HCA_RATIO = 128, CSA_HCA_PAGE_SIZE = 2, CSA_HCA_MAX_ROWS = 16 * 48 * 32 };
+csa_status_t csa_hca_compress(const float *x, const float *gate, const float *bias,
+                              int32_t dim, int32_t bs, const int32_t *cu_x, int64_t total_rows,
+                              const int32_t *start_pos, int32_t max_rows_per_req,
+                              const int32_t *page_table, int32_t page_table_stride,
+                              int32_t out_kind, void *out, int64_t num_slots, int32_t *status,
+                              void *stream);
+size_t csa_hca_attention_workspace_size(int32_t num_q, int32_t heads, int32_t window,
+                                        int32_t decode, int32_t max_hca_len);
+csa_status_t csa_hca_attention(const void *q, int32_t num_q, int32_t heads, const void *hca_cache,
+                               const void *raw_cache, int32_t kv_fmt, int64_t num_hca_slots,
+                               int64_t num_raw_slots, const int32_t *page_table,
+                               int32_t page_table_stride, const int32_t *seq_lens, int32_t bs,
+                               const int32_t *cu_q, const int32_t *q_pos, int32_t max_hca_len,
+                               int32_t window, float sm_scale, int32_t decode, void *out,
+                               float *lse, void *workspace, size_t workspace_bytes,
+                               int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
