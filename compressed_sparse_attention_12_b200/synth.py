@@ -30,6 +30,15 @@ C4_PAGE = 64
 # stream numbers: one independent generator per drawn field
 _S_PAGES, _S_IDXK, _S_KVC4, _S_KVRAW, _S_QIDX, _S_W, _S_Q = 1, 2, 3, 4, 5, 6, 7
 _S_RAWKV, _S_GATE, _S_BIAS, _S_RAWIK, _S_IGATE, _S_IBIAS, _S_LENS = 8, 9, 10, 11, 12, 13, 14
+_S_HCA, _S_HGATE, _S_HBIAS = 15, 16, 17
+_S_DSAK, _S_DSAKV, _S_FREQ = 18, 19, 20
+
+# DSA comparison path: one index key per raw token, pages of 64 raw tokens
+DSA_PAGE = 64
+
+# HCA layers: 128 raw tokens per compressed row, 2 compressed rows per 256-token page
+HCA_RATIO = 128
+HCA_PAGE = PAGE_SIZE // HCA_RATIO
 
 
 @dataclass
@@ -287,6 +296,24 @@ def workload(name: str, scale: float = 1.0) -> Workload:
         new = 4096 if scale >= 1.0 else max(8, min(4096, int(4096 * scale)) // 4 * 4)
         return Workload("prefill", [ctx + new], [new], 64, 128, "fp8", 64, "fp8",
                         seed=3, page_slack=1)
+    if name == "dsa_128k":
+        # DSA over raw tokens on the 128K decode shapes: FP8 64x128 indexer (not
+        # rotated), 64 heads, FP8 KV, top-512 raw tokens, no window
+        w = Workload("dsa_128k", [sc(131072)] * 32, [1] * 32, 64, 128, "fp8", 64, "fp8",
+                     window=0, seed=5, page_slack=3, new_tokens=[0] * 32)
+        return w
+    if name.startswith("hca_"):
+        # HCA layers ("DeepSeek-V4 的交錯壓縮注意力（CSA/HCA）", "Heavily Compressed
+        # Attention（HCA）") on the shapes of the CSA workloads of the same size;
+        # the indexer fields are unused
+        base = {"hca_128k": "decode_128k", "hca_1m": "decode_1m",
+                "hca_prefill": "prefill"}.get(name)
+        if base is None:
+            raise KeyError(name)
+        w = workload(base, scale)
+        w.name = name
+        w.seed += 100
+        return w
     if name == "ragged":
         # 64 requests, log-uniform lengths, Q alternating 1 / 5, FP4 indexer, FP8 KV
         L = ragged_lens(64, sc(2048), sc(1048576), seed=4,
@@ -294,3 +321,93 @@ def workload(name: str, scale: float = 1.0) -> Workload:
         q = np.where(np.arange(64) % 2 == 0, 1, 5)
         return Workload("ragged", L, q, 64, 128, "fp4", 64, "fp8", seed=4, page_slack=5)
     raise KeyError(name)
+
+
+def hca_plan(w: Workload):
+    """HCA layer of the workload's requests: per request the raw position of
+    the first row handed to the 128-row compressor (the blocks whose last token
+    is one of this step's query tokens), how many raw rows it gets, and how
+    many HCA rows before them are drawn directly as post-compression values."""
+    L, Q = w.seq_lens, w.q_lens
+    j_min = -((-(L - Q - (HCA_RATIO - 1))) // HCA_RATIO)
+    j_max = L // HCA_RATIO - 1
+    start = np.where(j_min <= j_max, HCA_RATIO * np.maximum(j_min, 0), L).astype(np.int64)
+    new = (L - start).astype(np.int64)
+    direct = np.where(new > 0, start // HCA_RATIO, L // HCA_RATIO).astype(np.int64)
+    return start, new, direct
+
+
+def draw_hca(w: Workload, device="cpu") -> dict:
+    """Inputs of one HCA-layer step, on `device`:
+      hca_kv  [sum direct, 576] f32     HCA rows drawn directly (before the compressor's)
+      raw_pos [n_raw] int64, raw_req [n_raw] int32, kv_raw [n_raw, 576] f32
+              raw rows from the earliest query's window or the compressor's
+              first row, whichever is earlier, to L-1
+      raw_kv / gate [sum new, 576] f32  the compressor's rows (slice of kv_raw) and gate
+      bias    [128, 576] f32 ~N(0, 0.1^2)
+      q       [num_q, heads, 576] bf16
+    """
+    s = w.seed
+    start, new, direct = hca_plan(w)
+    out = {"hca_kv": normal((int(direct.sum()), KV_DIM), s, _S_HCA, device)}
+    first_q = w.seq_lens - w.q_lens
+    lo = np.maximum(0, np.minimum(first_q - w.window + 1, start))
+    pos = np.concatenate([np.arange(a, L) for a, L in zip(lo, w.seq_lens)]).astype(np.int64)
+    req = np.concatenate([np.full(L - a, b) for b, (a, L) in enumerate(zip(lo, w.seq_lens))]
+                         ).astype(np.int32)
+    out["raw_pos"], out["raw_req"] = pos, req
+    out["kv_raw"] = normal((pos.shape[0], KV_DIM), s, _S_KVRAW, device)
+    n_new = int(new.sum())
+    if n_new:
+        sel = np.concatenate([np.nonzero((req == b) & (pos >= a))[0] for b, a in enumerate(start)])
+        assert sel.shape[0] == n_new
+        out["raw_kv"] = out["kv_raw"][torch.as_tensor(sel, device=out["kv_raw"].device)]
+        out["gate"] = normal((n_new, KV_DIM), s, _S_HGATE, device)
+        out["bias"] = normal((HCA_RATIO, KV_DIM), s, _S_HBIAS, device, std=0.1)
+    out["q"] = normal((w.num_q, w.heads, KV_DIM), s, _S_Q, device, dtype=torch.bfloat16)
+    return out
+
+
+def dsa_page_table(w: Workload) -> np.ndarray:
+    """[bs, max 64-token pages] int32: a seeded permutation of the pool of
+    64-token pages; unused entries -1."""
+    per = (w.seq_lens + DSA_PAGE - 1) // DSA_PAGE
+    n = int(per.sum()) + w.page_slack
+    rng = np.random.default_rng(w.seed * 1_000_003 + _S_PAGES)
+    perm = rng.permutation(n).astype(np.int32)
+    pt = np.full((w.bs, int(per.max())), -1, dtype=np.int32)
+    o = 0
+    for b, k in enumerate(per):
+        pt[b, :k] = perm[o:o + k]
+        o += int(k)
+    return pt
+
+
+def draw_dsa(w: Workload, device="cpu") -> dict:
+    """Inputs of one DSA step, on `device` (every raw token has a KV row and an
+    index key; this step's query tokens are the last q_lens[b] of each request
+    and their rows are among them):
+      idx_k  [sum L, idx_dim] f32   index keys of every raw token, request-major
+      kv     [sum L, 576] f32       KV rows of every raw token
+      q_idx  [num_q, idx_heads, idx_dim] bf16, w [num_q, idx_heads] f32 U(0,1),
+      q      [num_q, heads, 576] bf16
+    """
+    s = w.seed
+    n = int(w.seq_lens.sum())
+    out = {"idx_k": normal((n, w.idx_dim), s, _S_DSAK, device),
+           "kv": normal((n, KV_DIM), s, _S_DSAKV, device)}
+    out["q_idx"] = normal((w.num_q, w.idx_heads, w.idx_dim), s, _S_QIDX, device,
+                          dtype=torch.bfloat16)
+    out["w"] = uniform((w.num_q, w.idx_heads), s, _S_W, device)
+    out["q"] = normal((w.num_q, w.heads, KV_DIM), s, _S_Q, device, dtype=torch.bfloat16)
+    return out
+
+
+def rope_freqs(max_pos: int, rope_dim: int, base: float = 10000.0) -> torch.Tensor:
+    """A rotary table [max_pos, rope_dim/2, 2] float32 of (cos, sin) of
+    pos * base^(-2i/rope_dim), computed in float64 on the host.  An input of
+    the fused RoPE kernels (the kernels never build it)."""
+    i = np.arange(rope_dim // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / rope_dim)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * theta[None, :]
+    return torch.from_numpy(np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32))

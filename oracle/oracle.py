@@ -262,7 +262,38 @@ def unpack_fp4(packed: np.ndarray) -> np.ndarray:
 def index_quantise(x: np.ndarray, fmt: str):
     """Rotation then quantisation of index queries/keys ([T] §3.1, §4).
     Returns a dict with the stored fields and the dequantised values."""
-    xr = hadamard_rotate(x)
+    return quantise_rows(hadamard_rotate(x), fmt)
+
+
+def dsa_index_quantise(x: np.ndarray, fmt: str):
+    """The DSA indexer's quantisation: the rows as given, no rotation ([T] §4:
+    the Hadamard step is what DSV4 adds on top of DSA)."""
+    return quantise_rows(x, fmt)
+
+
+def rope(x: np.ndarray, freqs: np.ndarray, rope_dim: int, pos) -> np.ndarray:
+    """Rotary embedding of the leading rope_dim values of each row ([T] §3.1
+    freqs_cis / positions): the pairs (x[2i], x[2i+1]) read as complex numbers
+    and multiplied by freqs[pos][i] = cos + i sin; the rest unchanged.
+    x [..., D]; pos broadcasts against x.shape[:-1]; freqs [max_pos, rope_dim/2, 2]."""
+    x = np.array(x, dtype=np.float64)
+    f = np.asarray(freqs, dtype=np.float64)
+    p = np.broadcast_to(np.asarray(pos, dtype=np.int64), x.shape[:-1])
+    z = x[..., 0:rope_dim:2] + 1j * x[..., 1:rope_dim:2]
+    rot = f[p, :, 0] + 1j * f[p, :, 1]
+    y = z * rot
+    x[..., 0:rope_dim:2] = y.real
+    x[..., 1:rope_dim:2] = y.imag
+    return x
+
+
+def rope_index_quantise(x: np.ndarray, freqs: np.ndarray, rope_dim: int, pos, fmt: str):
+    """[T] §3.1 / §4 fused order: RoPE, then the rotation, then quantisation."""
+    return index_quantise(rope(x, freqs, rope_dim, pos), fmt)
+
+
+def quantise_rows(xr: np.ndarray, fmt: str):
+    """Quantisation of (already rotated or plain) index rows into `fmt`."""
     if fmt == "fp8":
         codes, scales = quant_fp8_rows(xr)
         return {"codes": codes, "scales": scales, "deq": dequant_fp8_rows(codes, scales)}
@@ -504,4 +535,100 @@ def step(w, data, page_table, requests=None, sm_scale=None):
             o, lse = sparse_attention(qa[j], rows, sm_scale)
             out[t] = {"logical": logical, "phys": phys, "logits": lg[j, :nv[j]], "out": o,
                       "lse": lse, "n_vis": int(nv[j])}
+    return out
+
+
+def hca_step(w, data, page_table, requests=None, sm_scale=None):
+    """One HCA-layer step ([H] HCA: 128x compression, then dense attention over
+    the compressed blocks) for the requests listed (default: all), from the
+    same drawn buffers the GPU path reads (synth.draw_hca).
+
+    Block j of request b (raw rows 128j .. 128j+127) is pooled by the
+    compressor in this step when its last row is one of the step's query
+    positions; earlier blocks arrive as drawn post-compression rows.  Each
+    query at position p attends over the hca_visible(p) rows and its raw window
+    under one softmax.  Returns a dict keyed by query row with out and lse."""
+    import math
+    sm_scale = 1.0 / math.sqrt(KV_DIM) if sm_scale is None else sm_scale
+    fp8_kv = w.kv_fmt == "fp8"
+    L_all = np.asarray(w.seq_lens, dtype=np.int64)
+    Q_all = np.asarray(w.q_lens, dtype=np.int64)
+    requests = range(len(L_all)) if requests is None else requests
+    # which blocks each request's compressor pools in this step
+    pooled = []
+    for L, Q in zip(L_all, Q_all):
+        js = [j for j in range(int(L) // HCA_RATIO) if int(L - Q) <= HCA_RATIO * j + HCA_RATIO - 1]
+        pooled.append(js)
+    n_direct = [hca_len(int(L)) - len(js) for L, js in zip(L_all, pooled)]
+    d_off = np.concatenate([[0], np.cumsum(n_direct)]).astype(np.int64)
+    n_off = np.concatenate([[0], np.cumsum([HCA_RATIO * len(js) for js in pooled])]).astype(np.int64)
+    q_off = np.concatenate([[0], np.cumsum(Q_all)]).astype(np.int64)
+    raw_req = np.asarray(data["raw_req"])
+    raw_pos = np.asarray(data["raw_pos"])
+    out = {}
+    for b in requests:
+        L, Q = int(L_all[b]), int(Q_all[b])
+        rows = _t2n(data["hca_kv"][d_off[b]:d_off[b + 1]])
+        if pooled[b]:
+            sl = slice(n_off[b], n_off[b + 1])
+            rows = np.concatenate([rows, hca_compress(_t2n(data["raw_kv"][sl]),
+                                                      _t2n(data["gate"][sl]),
+                                                      _t2n(data["bias"]))])
+        assert rows.shape[0] == hca_len(L)
+        deq = kv_decode_rows(kv_encode_rows(rows, fp8_kv), fp8_kv) if rows.shape[0] else rows
+        sel = raw_req == b
+        raw_rows = dict(zip(raw_pos[sel].tolist(),
+                            kv_decode_rows(kv_encode_rows(_t2n(data["kv_raw"][sel]), fp8_kv),
+                                           fp8_kv)))
+        qa = _t2n(data["q"][q_off[b]:q_off[b + 1]])
+        for j in range(Q):
+            p = L - Q + j
+            nv = min(hca_len(L), hca_visible(p))
+            win = window_positions(p, w.window)
+            wrows = np.array([raw_rows[int(r)] for r in win]).reshape(-1, KV_DIM)
+            o, lse = hca_attention(qa[j], deq[:nv], wrows, sm_scale)
+            out[int(q_off[b] + j)] = {"out": o, "lse": lse, "n_hca": nv}
+    return out
+
+
+def dsa_n_visible(pos: int) -> int:
+    """Keys visible to a DSA query at raw position pos ([T] §1: one key per raw
+    token, causal): the tokens 0..pos."""
+    return pos + 1
+
+
+def dsa_step(w, data, page_table, requests=None, sm_scale=None):
+    """One DSA step ([T] §1: the indexer picks the top-k raw tokens, attention
+    reads their KV) for the requests listed, k = 512: index keys and queries
+    quantised without rotation, logits over keys s <= p, top-512 with the page
+    transform of 64-token pages, one softmax over the selected raw rows (no
+    window).  Returns a dict keyed by query row (logical, phys, out, lse)."""
+    import math
+    sm_scale = 1.0 / math.sqrt(KV_DIM) if sm_scale is None else sm_scale
+    fp8_kv = w.kv_fmt == "fp8"
+    L_all = np.asarray(w.seq_lens, dtype=np.int64)
+    Q_all = np.asarray(w.q_lens, dtype=np.int64)
+    requests = range(len(L_all)) if requests is None else requests
+    l_off = np.concatenate([[0], np.cumsum(L_all)])
+    q_off = np.concatenate([[0], np.cumsum(Q_all)])
+    out = {}
+    for b in requests:
+        L, Q = int(L_all[b]), int(Q_all[b])
+        keys = dsa_index_quantise(_t2n(data["idx_k"][l_off[b]:l_off[b + 1]]), w.idx_fmt)["deq"]
+        qs = slice(q_off[b], q_off[b + 1])
+        qi = dsa_index_quantise(_t2n(data["q_idx"][qs]), w.idx_fmt)["deq"]
+        ww = _t2n(data["w"][qs])
+        pos = np.arange(L - Q, L)
+        nv = np.array([min(L, dsa_n_visible(int(p))) for p in pos], dtype=np.int64)
+        lg = indexer_logits(qi, ww, keys, nv)
+        kv_rows = _t2n(data["kv"][l_off[b]:l_off[b + 1]])
+        qa = _t2n(data["q"][qs])
+        for j, p in enumerate(pos):
+            phys, logical = topk_transform(lg[j], int(nv[j]), page_table[b], 1 << 40, k=TOPK,
+                                           c4_page_size=64)
+            chosen = logical[logical >= 0]
+            rows = kv_decode_rows(kv_encode_rows(kv_rows[chosen], fp8_kv), fp8_kv)
+            o, lse = sparse_attention(qa[j], rows, sm_scale)
+            out[int(q_off[b] + j)] = {"logical": logical, "phys": phys, "out": o, "lse": lse,
+                                      "logits": lg[j, :nv[j]], "n_vis": int(nv[j])}
     return out

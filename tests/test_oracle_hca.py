@@ -83,3 +83,39 @@ def test_hca_attention_matches_sdpa(n_hca, n_win):
     s = (q @ k.numpy().T) / 24
     np.testing.assert_allclose(lse, np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) +
                                s.max(1), rtol=1e-12)
+
+
+def test_hca_step_flat_gate_block_is_the_mean_and_rows_follow_visibility():
+    # a whole oracle HCA step on a small workload with the compressor's gate and
+    # bias set flat: the freshly pooled row is the block mean, so every query's
+    # output equals dense attention over [drawn rows, block mean] cut at
+    # hca_visible(p), plus its window
+    import sys, os
+    sys.path.insert(0, os.path.join(os.path.dirname(__file__), ".."))
+    from compressed_sparse_attention_12_b200 import synth
+    w = synth.workload("hca_prefill", 1 / 16)
+    d = synth.draw_hca(w, "cpu")
+    d["gate"] = torch.zeros_like(d["gate"])
+    d["bias"] = torch.zeros_like(d["bias"])
+    pt = synth.page_table(w)
+    ref = orc.hca_step(w, d, pt)
+    L, Q = int(w.seq_lens[0]), int(w.q_lens[0])
+    direct = d["hca_kv"].double().numpy()
+    new = d["raw_kv"].double().numpy()
+    assert new.shape[0] % 128 == 0 and new.shape[0] > 0
+    rows = np.concatenate([direct, new.reshape(-1, 128, 576).mean(axis=1)])
+    assert rows.shape[0] == L // 128
+    deq = orc.kv_decode_rows(orc.kv_encode_rows(rows, True), True)
+    raw = dict(zip(d["raw_pos"].tolist(),
+                   orc.kv_decode_rows(orc.kv_encode_rows(d["kv_raw"].double().numpy(), True), True)))
+    q = d["q"].double().numpy()
+    for j in (0, Q // 2, Q - 1):
+        p = L - Q + j
+        nv = (p + 1) // 128
+        assert ref[j]["n_hca"] == nv
+        win = np.array([raw[r] for r in range(max(0, p - w.window + 1), p + 1)])
+        k = torch.tensor(np.concatenate([deq[:nv], win]))
+        want = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q[j])[None, None], k[None, None], k[None, None, :, :512],
+            scale=1 / 24)[0, 0].numpy()
+        np.testing.assert_allclose(ref[j]["out"], want, rtol=1e-10, atol=1e-10)
