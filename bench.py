@@ -36,6 +36,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "CSA decode query-tok/s at 128K/1M ctx; achieved HBM GB/s vs ~8 TB/s"
+METRIC_HCA = "HCA layer query-tok/s (dense attention over 128x-compressed rows + window)"
+METRIC_DSA = "DSA decode query-tok/s (top-512 over raw tokens, no compression)"
 UNIT = "query-tok/s"
 
 
@@ -106,10 +108,11 @@ def index_bytes_per_key(w):
     return {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}[w.idx_fmt]
 
 
-def indexer_alg_bytes(w):
+def indexer_alg_bytes(w, ratio=4):
     """Bytes one indexer launch must move: every visible key (codes + scales)
-    once per query row, the query codes and weights, and the logits written."""
-    nv = np.concatenate([np.minimum(w.c4_lens[b], (np.arange(L - q, L) + 1) // 4)
+    once per query row, the query codes and weights, and the logits written
+    (ratio raw tokens per key: 4 for C4, 1 for DSA)."""
+    nv = np.concatenate([np.minimum(w.seq_lens[b] // ratio, (np.arange(L - q, L) + 1) // ratio)
                          for b, (L, q) in enumerate(zip(w.seq_lens, w.q_lens))])
     qb = {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}
     return int(nv.sum() * (index_bytes_per_key(w) + 4) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4))
@@ -199,6 +202,79 @@ def max_over_ranks(values, world, device=None):
     return t.tolist()
 
 
+def time_graph(g, stream, args, l2_flush, inner, world, dev, local, check):
+    """Warm-up replays, then args.steps timed replays of graph g between CUDA
+    events on `stream` with an L2 flush before each (outside the events); the
+    `inner` event pair, recorded inside the graph, times one kernel.  Returns
+    (seconds per step, seconds of the inner kernel, clocks), max over ranks."""
+    import torch
+    import torch.distributed as dist
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            l2_flush()
+            g.replay()
+    torch.cuda.synchronize()
+    check()
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    step_ms, in_ms = [], []
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            l2_flush()
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            e1.synchronize()
+            step_ms.append(e0.elapsed_time(e1))
+            in_ms.append(inner[0].elapsed_time(inner[1]))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ck = clocks.stop()
+    check()
+    t_step = sum(step_ms) / len(step_ms) / 1e3
+    t_in = sum(in_ms) / len(in_ms) / 1e3
+    t_step, t_in = max_over_ranks([t_step, t_in], world, dev)
+    return t_step, t_in, ck
+
+
+def time_e2e(g, stream, args, l2_flush, data, dst, out, world, dev, num_q):
+    """The step end to end: every step copies its inputs (the fields of `dst`
+    present in `data`) from pinned host memory, replays the graph and copies
+    the output back, all inside the timed region."""
+    import torch
+    h_in = {k: data[k].cpu().pin_memory() for k in dst if data.get(k) is not None
+            and dst[k] is not None}
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+    d2h = h_out.numel() * h_out.element_size()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ms = []
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup + args.steps):
+            l2_flush()
+            e0.record(stream)
+            for k, v in h_in.items():
+                dst[k].copy_(v, non_blocking=True)
+            g.replay()
+            h_out.copy_(out, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                ms.append(e0.elapsed_time(e1))
+    t = sum(ms) / len(ms) / 1e3
+    t = max_over_ranks([t], world, dev)[0]
+    return {"value": world * num_q / t, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": t * 1e3}
+
+
 def cpu_baseline(w, data, pt, budget_s=20.0):
     """The oracle, as it stands, timed on this host's cores over a bounded
     sample: whole-step oracle runs of requests 0, 1, ... until ~budget_s."""
@@ -227,30 +303,252 @@ def run_reference(args):
     if rank != 0:
         return
     w = synth.workload(args.workload)
-    # draw the sampled request's inputs on the host (small): one request's slice
-    data = synth.draw(w, "cuda" if torch.cuda.is_available() else "cpu")
-    pt = synth.page_table(w)
+    hca = args.workload.startswith("hca_")
+    dsa = args.workload.startswith("dsa_")
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    if hca:
+        data, pt, run = synth.draw_hca(w, device), synth.page_table(w), oracle.hca_step
+    elif dsa:
+        data, pt, run = synth.draw_dsa(w, device), synth.dsa_page_table(w), oracle.dsa_step
+    else:
+        data, pt, run = synth.draw(w, device), synth.page_table(w), oracle.step
     oracle.build()
     for i in range(args.warmup):
-        oracle.step(w, data, pt, requests=[i % w.bs])
+        run(w, data, pt, requests=[i % w.bs])
     times = []
     for i in range(args.steps):
         t0 = time.perf_counter()
-        oracle.step(w, data, pt, requests=[i % w.bs])
+        run(w, data, pt, requests=[i % w.bs])
         times.append(time.perf_counter() - t0)
     per = sum(times) / len(times)
     q_per = float(np.mean(w.q_lens))
     v = q_per / per
-    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+    out = {"impl": "reference", "metric": METRIC_HCA if hca else METRIC_DSA if dsa else METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": workload_config(w),
+           "data": "synthetic",
+           "config": hca_workload_config(w) if hca else workload_config(w),
            "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.num_threads(),
                             "kind": "oracle",
                             "sample": "each step: the whole oracle step for one request "
                                       "(cycling through the batch)"},
            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
+
+
+def hca_workload_config(w):
+    from compressed_sparse_attention_12_b200 import synth
+    new = synth.hca_plan(w)[1]
+    return {"workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
+            "hca_seq_len": int((w.seq_lens // 128).max()), "query_tokens": w.num_q,
+            "heads": w.heads, "kv": w.kv_fmt, "window": w.window, "ratio": 128,
+            "page_size": 256, "compressed_rows_this_step": int(new.sum() // 128),
+            "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)"}
+
+
+def hca_attn_alg_bytes(w):
+    """Bytes one HCA attention call must move: per query every visible HCA row
+    and every window row once, the query and the output (+ lse)."""
+    row = 656 if w.kv_fmt == "fp8" else 1152
+    pos = np.concatenate([np.arange(L - q, L) for L, q in zip(w.seq_lens, w.q_lens)])
+    L = np.repeat(w.seq_lens, w.q_lens)
+    rows = np.minimum(L // 128, (pos + 1) // 128) + np.minimum(w.window, pos + 1)
+    return int(rows.sum() * row + w.num_q * w.heads * (576 * 2 + 512 * 2 + 4))
+
+
+def hca_step_alg_bytes(w, new_rows):
+    """The HCA step: the attention's bytes plus the compressor's (raw rows and
+    gates read as f32, the pooled rows written)."""
+    row = 656 if w.kv_fmt == "fp8" else 1152
+    return hca_attn_alg_bytes(w) + int(new_rows) * 576 * 4 * 2 + 128 * 576 * 4 + \
+        int(new_rows) // 128 * row
+
+
+def hca_cpu_baseline(w, data, pt, budget_s=20.0):
+    from oracle import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    done_q, reqs = 0, []
+    for b in range(w.bs):
+        oracle.hca_step(w, data, pt, requests=[b])
+        done_q += int(w.q_lens[b])
+        reqs.append(b)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done_q / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"whole oracle HCA step (128-row compressor, encode caches, dense "
+                      f"attention) for {len(reqs)} of {w.bs} requests ({done_q} query tokens) "
+                      f"in {dt:.1f} s"}
+
+
+def main_hca(args, world, rank, local, dev):
+    """An HCA layer step: the 128-row compressor over the blocks completed by
+    this step's tokens, then dense attention over every visible HCA row plus
+    the raw window, in one CUDA graph."""
+    import torch
+    import torch.distributed as dist
+    from compressed_sparse_attention_12_b200 import csa, pipeline, synth
+    w = rank_workload(args.workload, rank)
+    data = synth.draw_hca(w, dev)
+    batch = pipeline.HcaBatch(w, data, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_read = flush[: 256 << 20].view(torch.int64)
+
+    def l2_flush():
+        flush.fill_(1)
+        flush_read.max()
+
+    ev_a0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev_a1 = torch.cuda.Event(enable_timing=True, external=True)
+
+    def body(s):
+        batch.compress(s)
+        ev_a0.record(s)
+        batch.attend(s)
+        ev_a1.record(s)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            body(stream)
+        stream.synchronize()
+        batch.check_status()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            body(stream)
+    t_step, t_att, ck = time_graph(g, stream, args, l2_flush, (ev_a0, ev_a1), world, dev, local,
+                                   batch.check_status)
+    e2e = None
+    if not args.profile:
+        dst = {"q": batch.q, "raw_kv": batch.raw_kv, "gate": batch.gate}
+        e2e = time_e2e(g, stream, args, l2_flush, data, dst, batch.out, world, dev, w.num_q)
+    split = csa.csa_hca_attention_workspace_size(w.num_q, w.heads, w.window, batch.decode,
+                                                 batch.max_hca) > 0
+    launches = (1 if batch.max_new >= 128 else 0) + (2 if split else 1)
+    if rank == 0:
+        hbm, src = peaks()
+        ab = hca_attn_alg_bytes(w)
+        sb = hca_step_alg_bytes(w, int(batch.new_tokens.sum()))
+        achieved = ab / t_att / 1e9
+        cfg = hca_workload_config(w)
+        out = {"metric": METRIC_HCA, "value": world * w.num_q / t_step, "unit": UNIT,
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None,
+               "dtype": "f16 attention" if w.kv_fmt == "fp8" else "bf16 attention",
+               "data": "synthetic", "config": cfg,
+               "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
+                       "frac_of_peak": sb / t_step / 1e9 / hbm},
+               "roofline": {"kernel": "hca attention (sparse_mqa kernel, dense mode"
+                                      + (", + combine)" if split else ")"),
+                            "bound": "hbm", "achieved": achieved, "peak": hbm,
+                            "peak_source": src, "unit": "GB/s", "frac": achieved / hbm,
+                            "traffic": None, "alg_bytes_per_launch": ab,
+                            "launch_ms": t_att * 1e3},
+               "e2e": e2e, "gpu_launches": launches * args.steps, "clocks": ck}
+        if not args.no_cpu_baseline and not args.profile and world == 1:
+            out["cpu_baseline"] = hca_cpu_baseline(w, data, batch.pt_host)
+        print(json.dumps(out), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def dsa_step_alg_bytes(w):
+    """The DSA step: the indexer's bytes, the selected rows and the attention's
+    q/out, and this step's stored token rows."""
+    row = 656 if w.kv_fmt == "fp8" else 1152
+    pos = np.concatenate([np.arange(L - q, L) for L, q in zip(w.seq_lens, w.q_lens)])
+    sel = np.minimum(512, pos + 1)
+    return int(indexer_alg_bytes(w, 1) + sel.sum() * row + w.num_q * w.heads * (576 + 512) * 2
+               + w.num_q * (576 * 4 + row + w.idx_dim * 4 + w.idx_dim + 4))
+
+
+def main_dsa(args, world, rank, local, dev):
+    """The DSA comparison step: store this step's tokens, quantise the index
+    queries, indexer over every raw token, top-512 page transform, attention
+    over the selected raw rows; one CUDA graph."""
+    import torch
+    import torch.distributed as dist
+    from compressed_sparse_attention_12_b200 import csa, pipeline, synth
+    w = rank_workload(args.workload, rank)
+    data = synth.draw_dsa(w, dev)
+    batch = pipeline.DsaBatch(w, data, device=dev)
+    for k in ("kv", "idx_k"):
+        data.pop(k)
+    torch.cuda.empty_cache()
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_read = flush[: 256 << 20].view(torch.int64)
+
+    def l2_flush():
+        flush.fill_(1)
+        flush_read.max()
+
+    ev_i0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev_i1 = torch.cuda.Event(enable_timing=True, external=True)
+
+    def body(s):
+        batch.store(s)
+        csa.csa_index_quant(batch.q_idx, batch.idx_fmt, batch.q_codes, batch.q_bsc,
+                            batch.q_scales, w_in=batch.w_head, w_out=batch.w_fold,
+                            status=batch.status, stream=s)
+        ev_i0.record(s)
+        csa.csa_dsa_indexer_logits(batch.q_codes, batch.q_bsc, batch.w_fold, w.idx_heads,
+                                   w.idx_dim, batch.idx_fmt, batch.k_codes, batch.k_bsc,
+                                   batch.k_scales, batch.page_table, batch.seq_lens, batch.cu_q,
+                                   batch.q_pos, batch.max_len, batch.logits,
+                                   status=batch.status, stream=s)
+        ev_i1.record(s)
+        batch.select(s)
+        batch.attend(s)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            body(stream)
+        stream.synchronize()
+        batch.check_status()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            body(stream)
+    t_step, t_idx, ck = time_graph(g, stream, args, l2_flush, (ev_i0, ev_i1), world, dev, local,
+                                   batch.check_status)
+    e2e = None
+    if not args.profile:
+        dst = {"q_idx": batch.q_idx, "w": batch.w_head, "q": batch.q}
+        e2e = time_e2e(g, stream, args, l2_flush, data, dst, batch.out, world, dev, w.num_q)
+    split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, 0, batch.decode) > 0
+    launches = 2 + 1 + 1 + 2 + (2 if split else 1)
+    if rank == 0:
+        hbm, src = peaks()
+        ib = indexer_alg_bytes(w, 1)
+        sb = dsa_step_alg_bytes(w)
+        achieved = ib / t_idx / 1e9
+        cfg = {"workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
+               "keys_per_request": int(w.seq_lens.max()), "query_tokens": w.num_q,
+               "indexer": f"{w.idx_fmt} {w.idx_heads}x{w.idx_dim} (no rotation)",
+               "heads": w.heads, "kv": w.kv_fmt, "window": 0, "topk": 512, "page_size": 64,
+               "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)"}
+        out = {"metric": METRIC_DSA, "value": world * w.num_q / t_step, "unit": UNIT,
+               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": f"{w.idx_fmt} indexer, f16 attention",
+               "data": "synthetic", "config": cfg,
+               "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
+                       "frac_of_peak": sb / t_step / 1e9 / hbm},
+               "roofline": {"kernel": "dsa indexer_logits (indexer_tc_kernel, one key per token)",
+                            "bound": "hbm", "achieved": achieved, "peak": hbm,
+                            "peak_source": src, "unit": "GB/s", "frac": achieved / hbm,
+                            "traffic": None, "alg_bytes_per_launch": ib,
+                            "launch_ms": t_idx * 1e3},
+               "e2e": e2e, "gpu_launches": launches * args.steps, "clocks": ck}
+        print(json.dumps(out), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def main():
@@ -276,6 +574,12 @@ def main():
     if world > 1:
         dist.barrier()
     csa.lib()
+    if args.workload.startswith("hca_"):
+        main_hca(args, world, rank, local, dev)
+        return
+    if args.workload.startswith("dsa_"):
+        main_dsa(args, world, rank, local, dev)
+        return
 
     w = rank_workload(args.workload, rank)
     data = synth.draw(w, dev)
@@ -371,68 +675,15 @@ def main():
     launches_per_step = (2 if batch.max_new >= 4 else 0) + 1 + 1 + (1 if fused[0] else 2) + \
         (2 if csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, w.window, batch.decode) > 0 else 1)
 
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    for _ in range(args.warmup):
-        l2_flush()
-        g.replay()
-    torch.cuda.synchronize()
-    batch.check_status()
-
-    clocks = Clocks(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    step_ms, idx_ms = [], []
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            l2_flush()
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-            e1.synchronize()
-            step_ms.append(e0.elapsed_time(e1))
-            idx_ms.append(ev_i0.elapsed_time(ev_i1))
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ck = clocks.stop()
-    batch.check_status()
-    t_step = sum(step_ms) / len(step_ms) / 1e3
-    t_idx = sum(idx_ms) / len(idx_ms) / 1e3
-    t_step, t_idx = max_over_ranks([t_step, t_idx], world, dev)
+    t_step, t_idx, ck = time_graph(g, stream, args, l2_flush, (ev_i0, ev_i1), world, dev, local,
+                                   batch.check_status)
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.profile:
-        h_in = {k: data[k].cpu().pin_memory() for k in ("q_idx", "w", "q") if k in data}
-        for k in ("raw_kv", "gate", "raw_idx_k", "idx_gate"):
-            if data.get(k) is not None:
-                h_in[k] = data[k].cpu().pin_memory()
-        h_out = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
         dst = {"q_idx": batch.q_idx, "w": batch.w_head, "q": batch.q, "raw_kv": batch.raw_kv,
                "gate": batch.gate, "raw_idx_k": batch.raw_idx_k, "idx_gate": batch.idx_gate}
-        h2d = sum(v.numel() * v.element_size() for v in h_in.values())
-        d2h = h_out.numel() * h_out.element_size()
-        e2e_ms = []
-        with torch.cuda.stream(stream):
-            for i in range(args.warmup + args.steps):
-                l2_flush()
-                e0.record(stream)
-                for k, v in h_in.items():
-                    dst[k].copy_(v, non_blocking=True)
-                g.replay()
-                h_out.copy_(batch.out, non_blocking=True)
-                e1.record(stream)
-                e1.synchronize()
-                if i >= args.warmup:
-                    e2e_ms.append(e0.elapsed_time(e1))
-        t_e2e = sum(e2e_ms) / len(e2e_ms) / 1e3
-        t_e2e = max_over_ranks([t_e2e], world, dev)[0]
-        e2e = {"value": world * w.num_q / t_e2e, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": t_e2e * 1e3}
+        e2e = time_e2e(g, stream, args, l2_flush, data, dst, batch.out, world, dev, w.num_q)
 
     if rank == 0:
         hbm, src = peaks()

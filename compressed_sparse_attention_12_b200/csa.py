@@ -69,6 +69,19 @@ _SIGS = {
     "csa_hca_attention": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _I32, _P,
                                          _I32, _P, _P, _I32, _I32, _F, _I32, _P, _P, _P, _SZ,
                                          _P, _P]),
+    "csa_rope_hadamard_quant": (ctypes.c_int, [_P, _I32, _I64, _I32, _P, _I32, _I32, _P, _I32,
+                                               _I32, _P, _I64, _P, _P, _P, _P, _P, _P, _P]),
+    "csa_c4_compress_index_rope": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _P, _I64, _P, _I32, _P,
+                                                  _I32, _I32, _P, _I32, _I32, _P, _P, _P, _I64,
+                                                  _P, _P]),
+    "csa_index_quant": (ctypes.c_int, [_P, _I32, _I64, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P,
+                                       _P, _P]),
+    "csa_dsa_indexer_logits": (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P,
+                                              _I64, _P, _I32, _P, _I32, _P, _P, _I32, _P, _I64,
+                                              _P, _P]),
+    "csa_dsa_topk512_page_transform": (ctypes.c_int, [_P, _I64, _I32, _P, _I32, _P, _P, _P, _I32,
+                                                      _I64, _I32, _I32, _P, _P, _P, _SZ, _P,
+                                                      _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
     "csa_sparse_mqa_decode": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _P,
                                              _I32, _P, _I32, _P, _P, _I32, _F, _P, _P, _P, _SZ,
@@ -155,6 +168,75 @@ def csa_hadamard_quant(x, fmt, codes, block_scales=None, scales=None, row_map=No
     _check("csa_hadamard_quant", lib().csa_hadamard_quant(
         _ptr(x), x_dtype, rows, dim, fmt, _ptr(row_map), n_out, _ptr(codes), _ptr(block_scales),
         _ptr(scales), _ptr(w_in), _ptr(w_out), _ptr(status), _stream(stream)))
+
+
+def csa_index_quant(x, fmt, codes, block_scales=None, scales=None, row_map=None,
+                    w_in=None, w_out=None, status=None, stream=None):
+    """Quantisation of index rows without the rotation (the DSA indexer)."""
+    dim = x.shape[-1]
+    rows = x.numel() // dim
+    x_dtype = CSA_FMT_BF16 if x.dtype == torch.bfloat16 else CSA_FMT_F32
+    n_out = codes.shape[0] if row_map is not None else rows
+    _check("csa_index_quant", lib().csa_index_quant(
+        _ptr(x), x_dtype, rows, dim, fmt, _ptr(row_map), n_out, _ptr(codes), _ptr(block_scales),
+        _ptr(scales), _ptr(w_in), _ptr(w_out), _ptr(status), _stream(stream)))
+
+
+def csa_rope_hadamard_quant(x, freqs_cis, rope_dim, positions, rows_per_pos, fmt, codes,
+                            block_scales=None, scales=None, row_map=None, w_in=None, w_out=None,
+                            status=None, stream=None):
+    """Rotary embedding, rotation and quantisation in one pass (include/csa.h).
+    freqs_cis: [max_pos, rope_dim/2, 2] float32 (cos, sin)."""
+    dim = x.shape[-1]
+    rows = x.numel() // dim
+    x_dtype = CSA_FMT_BF16 if x.dtype == torch.bfloat16 else CSA_FMT_F32
+    n_out = codes.shape[0] if row_map is not None else rows
+    _check("csa_rope_hadamard_quant", lib().csa_rope_hadamard_quant(
+        _ptr(x), x_dtype, rows, dim, _ptr(freqs_cis), int(rope_dim), freqs_cis.shape[0],
+        _ptr(positions), int(rows_per_pos), fmt, _ptr(row_map), n_out, _ptr(codes),
+        _ptr(block_scales), _ptr(scales), _ptr(w_in), _ptr(w_out), _ptr(status),
+        _stream(stream)))
+
+
+def csa_c4_compress_index_rope(x, gate, bias, cu_x, start_pos, max_rows_per_req, page_table,
+                               out_kind, freqs_cis, rope_dim, out, out_block_scales=None,
+                               out_scales=None, num_slots=None, status=None, stream=None):
+    """C4 compressor in an index-key mode with the rotary embedding between the
+    pooling and the rotation (include/csa.h)."""
+    bs = start_pos.shape[0]
+    _check("csa_c4_compress_index_rope", lib().csa_c4_compress_index_rope(
+        _ptr(x), _ptr(gate), _ptr(bias), x.shape[1], bs, _ptr(cu_x), x.shape[0], _ptr(start_pos),
+        int(max_rows_per_req), _ptr(page_table), page_table.shape[1], out_kind, _ptr(freqs_cis),
+        int(rope_dim), freqs_cis.shape[0], _ptr(out), _ptr(out_block_scales), _ptr(out_scales),
+        out.shape[0] if num_slots is None else int(num_slots), _ptr(status), _stream(stream)))
+
+
+def csa_dsa_indexer_logits(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, fmt, k_codes,
+                           k_block_scales, k_scales, page_table, seq_lens, cu_q, q_pos,
+                           max_seq_len, logits, num_slots=None, status=None, stream=None):
+    """Indexer logits over raw tokens (one key per token, keys s <= p)."""
+    num_q = q_weights.shape[0]
+    _check("csa_dsa_indexer_logits", lib().csa_dsa_indexer_logits(
+        _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
+        _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
+        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos),
+        int(max_seq_len), _ptr(logits), logits.shape[1], _ptr(status), _stream(stream)))
+
+
+def csa_dsa_topk512_page_transform(logits, seq_lens, cu_q, q_pos, page_table, num_slots,
+                                   max_seq_len, out_indices, raw_indices=None, workspace=None,
+                                   page_size=64, status=None, stream=None):
+    """Top-512 over raw tokens with the 64-token page transform."""
+    num_q = out_indices.shape[0]
+    if workspace is None:
+        workspace = torch.empty(max(1, csa_topk512_workspace_size(num_q, max_seq_len)),
+                                dtype=torch.uint8, device=out_indices.device)
+    _check("csa_dsa_topk512_page_transform", lib().csa_dsa_topk512_page_transform(
+        _ptr(logits), logits.shape[1], num_q, _ptr(seq_lens), seq_lens.shape[0], _ptr(cu_q),
+        _ptr(q_pos), _ptr(page_table), page_table.shape[1], int(num_slots), int(page_size),
+        int(max_seq_len), _ptr(out_indices), _ptr(raw_indices), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)))
 
 
 def csa_indexer_logits(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, fmt, k_codes,

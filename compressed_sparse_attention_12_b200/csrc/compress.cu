@@ -143,12 +143,35 @@ __device__ __forceinline__ float quant_index_row(const float (&v)[E], int lane, 
     return st;
 }
 
-template <int E, typename T>
+// Rotary position embedding of the leading rope_dim values of a row held E per
+// lane: consecutive pairs (x[2i], x[2i+1]) taken as the complex number
+// x[2i] + i x[2i+1] and multiplied by freqs[pos][i] = (cos, sin); each product
+// and sum rounded to float separately (no contraction).
+template <int E>
+__device__ __forceinline__ void apply_rope(float (&v)[E], int lane, const float2 *freqs,
+                                           int rope_dim, int64_t pos) {
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+        const int d = lane * E + i;
+        if (d < rope_dim) {
+            const float2 cs = freqs[pos * (rope_dim / 2) + d / 2];
+            const float a = v[i], b = v[i + 1];
+            v[i] = __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y));
+            v[i + 1] = __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x));
+        }
+    }
+}
+
+// ROT: apply the Hadamard rotation (the index rows of the C4 indexer) or not
+// (plain per-row quantisation, the DSA indexer).  With rope.freqs set, the
+// rotary embedding runs first at position rope.pos[r / rope.rows_per_pos].
+template <int E, typename T, bool ROT>
 __global__ void __launch_bounds__(256)
 hadamard_quant_kernel(const T *__restrict__ x, int64_t rows, int fmt,
                       const int32_t *__restrict__ row_map, int64_t num_out_rows,
                       uint8_t *codes, uint8_t *block_scales, float *scales,
-                      const float *__restrict__ w_in, float *w_out, int32_t *status) {
+                      const float *__restrict__ w_in, float *w_out, int32_t *status,
+                      const RopeArgs rope) {
     pdl_begin();
     constexpr int D = 32 * E;
     const int lane = threadIdx.x & 31;
@@ -171,7 +194,15 @@ hadamard_quant_kernel(const T *__restrict__ x, int64_t rows, int fmt,
         else
             v[i] = x[r * D + lane * E + i];
     }
-    rotate<E>(v, lane);
+    if (rope.freqs) {
+        const int32_t p = rope.pos[r / rope.rows_per_pos];
+        if (p < 0 || p >= rope.max_pos) {
+            if (lane == 0) report(status, CSA_ERR_BOUNDS);
+            return;
+        }
+        apply_rope<E>(v, lane, rope.freqs, rope.rope_dim, p);
+    }
+    if constexpr (ROT) rotate<E>(v, lane);
     const float s = quant_index_row<E>(v, lane, fmt, orow, codes, block_scales, scales);
     if (w_in && w_out && lane == 0) w_out[r] = w_in[r] * s;
 }
@@ -343,7 +374,7 @@ compress_index_kernel(const float *__restrict__ x, const float *__restrict__ gat
                       const float *__restrict__ bias, const int32_t *cu_x,
                       const int32_t *start_pos, int max_rows, const int32_t *page_table,
                       int pt_stride, int fmt, uint8_t *codes, uint8_t *block_scales,
-                      float *scales, int64_t num_slots, int32_t *status) {
+                      float *scales, int64_t num_slots, int32_t *status, const RopeArgs rope) {
     pdl_begin();
     constexpr int D = 32 * E;
     const int lane = threadIdx.x & 31;
@@ -368,6 +399,15 @@ compress_index_kernel(const float *__restrict__ x, const float *__restrict__ gat
     float v[E];
 #pragma unroll
     for (int e = 0; e < E; e++) v[e] = pool4(xs[e], zs[e]);
+    if (rope.freqs) {
+        // the compressed key of block j stands at the raw position of its first row
+        const int64_t p = 4 * (int64_t)j;
+        if (p >= rope.max_pos) {
+            if (lane == 0) report(status, CSA_ERR_BOUNDS);
+            return;
+        }
+        apply_rope<E>(v, lane, rope.freqs, rope.rope_dim, p);
+    }
     rotate<E>(v, lane);
     quant_index_row<E>(v, lane, fmt, slot, codes, block_scales, scales);
 }
@@ -386,18 +426,20 @@ cudaError_t launch_kv_store(const float *rows, int64_t n, const int32_t *slots, 
 cudaError_t launch_hadamard_quant(const void *x, int x_dtype, int64_t rows, int dim, int fmt,
                                   const int32_t *row_map, int64_t num_out_rows, void *codes,
                                   uint8_t *block_scales, float *scales, const float *w_in,
-                                  float *w_out, int32_t *status, cudaStream_t s) {
+                                  float *w_out, int32_t *status, cudaStream_t s, bool rotate,
+                                  const RopeArgs &rope) {
     if (rows == 0) return cudaSuccess;
     const unsigned grid = (unsigned)((rows + 7) / 8);
     uint8_t *c = (uint8_t *)codes;
-#define CSA_HQ(E, T)                                                                        \
-    launch_k(hadamard_quant_kernel<E, T>, grid, 256, 0, s, (const T *)x, rows, fmt, row_map,      \
-                                                     num_out_rows, c, block_scales, scales, \
-                                                     w_in, w_out, status)
-    if (dim == 64 && x_dtype == CSA_FMT_BF16) CSA_HQ(2, uint16_t);
-    else if (dim == 64) CSA_HQ(2, float);
-    else if (x_dtype == CSA_FMT_BF16) CSA_HQ(4, uint16_t);
-    else CSA_HQ(4, float);
+#define CSA_HQ(E, T, R)                                                                     \
+    launch_k(hadamard_quant_kernel<E, T, R>, grid, 256, 0, s, (const T *)x, rows, fmt, row_map, \
+             num_out_rows, c, block_scales, scales, w_in, w_out, status, rope)
+#define CSA_HQ2(E, T) do { if (rotate) CSA_HQ(E, T, true); else CSA_HQ(E, T, false); } while (0)
+    if (dim == 64 && x_dtype == CSA_FMT_BF16) CSA_HQ2(2, uint16_t);
+    else if (dim == 64) CSA_HQ2(2, float);
+    else if (x_dtype == CSA_FMT_BF16) CSA_HQ2(4, uint16_t);
+    else CSA_HQ2(4, float);
+#undef CSA_HQ2
 #undef CSA_HQ
     return cudaGetLastError();
 }
@@ -419,7 +461,7 @@ cudaError_t launch_c4_compress(const float *x, const float *gate, const float *b
                                int max_rows, const int32_t *page_table, int pt_stride,
                                int out_kind, void *out, uint8_t *out_block_scales,
                                float *out_scales, int64_t num_slots, int32_t *status,
-                               cudaStream_t s) {
+                               cudaStream_t s, const RopeArgs &rope) {
     const int max_blocks = max_rows / 4;
     if (bs == 0 || max_blocks == 0) return cudaSuccess;
     if (out_kind == CSA_OUT_KV_BF16 || out_kind == CSA_OUT_KV_FP8) {
@@ -436,11 +478,11 @@ cudaError_t launch_c4_compress(const float *x, const float *gate, const float *b
         if (dim == 64)
             launch_k(compress_index_kernel<2>, grid, 256, 0, s, 
                 x, gate, bias, cu_x, start_pos, max_rows, page_table, pt_stride, fmt,
-                (uint8_t *)out, out_block_scales, out_scales, num_slots, status);
+                (uint8_t *)out, out_block_scales, out_scales, num_slots, status, rope);
         else
             launch_k(compress_index_kernel<4>, grid, 256, 0, s, 
                 x, gate, bias, cu_x, start_pos, max_rows, page_table, pt_stride, fmt,
-                (uint8_t *)out, out_block_scales, out_scales, num_slots, status);
+                (uint8_t *)out, out_block_scales, out_scales, num_slots, status, rope);
     }
     return cudaGetLastError();
 }

@@ -60,13 +60,18 @@ csa_status_t csa_kv_store(const float *rows, int64_t n, const int32_t *slots, in
                                             as_stream(stream)));
 }
 
-csa_status_t csa_c4_compress(const float *x, const float *gate, const float *bias, int32_t dim,
+static bool rope_ok(const float *freqs_cis, int32_t rope_dim, int32_t max_pos, int32_t dim) {
+    return freqs_cis && rope_dim > 0 && rope_dim <= dim && (rope_dim % 2) == 0 && max_pos > 0 &&
+           (reinterpret_cast<uintptr_t>(freqs_cis) & 7) == 0;
+}
+
+static csa_status_t c4_compress(const float *x, const float *gate, const float *bias, int32_t dim,
                              int32_t bs, const int32_t *cu_x, int64_t total_rows,
                              const int32_t *start_pos, int32_t max_rows_per_req,
                              const int32_t *page_table, int32_t page_table_stride,
                              int32_t out_kind, void *out, uint8_t *out_block_scales,
                              float *out_scales, int64_t num_slots, int32_t *status,
-                             void *stream) {
+                             void *stream, const csa::RopeArgs &rope) {
     if (bs < 0 || total_rows < 0 || max_rows_per_req < 0 || page_table_stride < 0)
         return CSA_ERR_INVALID;
     const bool kv = out_kind == CSA_OUT_KV_BF16 || out_kind == CSA_OUT_KV_FP8;
@@ -83,7 +88,41 @@ csa_status_t csa_c4_compress(const float *x, const float *gate, const float *bia
     return cuda_status(csa::launch_c4_compress(x, gate, bias, dim, bs, cu_x, start_pos,
                                                max_rows_per_req, page_table, page_table_stride,
                                                out_kind, out, out_block_scales, out_scales,
-                                               num_slots, status, as_stream(stream)));
+                                               num_slots, status, as_stream(stream), rope));
+}
+
+csa_status_t csa_c4_compress(const float *x, const float *gate, const float *bias, int32_t dim,
+                             int32_t bs, const int32_t *cu_x, int64_t total_rows,
+                             const int32_t *start_pos, int32_t max_rows_per_req,
+                             const int32_t *page_table, int32_t page_table_stride,
+                             int32_t out_kind, void *out, uint8_t *out_block_scales,
+                             float *out_scales, int64_t num_slots, int32_t *status,
+                             void *stream) {
+    return c4_compress(x, gate, bias, dim, bs, cu_x, total_rows, start_pos, max_rows_per_req,
+                       page_table, page_table_stride, out_kind, out, out_block_scales, out_scales,
+                       num_slots, status, stream, csa::RopeArgs());
+}
+
+csa_status_t csa_c4_compress_index_rope(const float *x, const float *gate, const float *bias,
+                                        int32_t dim, int32_t bs, const int32_t *cu_x,
+                                        int64_t total_rows, const int32_t *start_pos,
+                                        int32_t max_rows_per_req, const int32_t *page_table,
+                                        int32_t page_table_stride, int32_t out_kind,
+                                        const float *freqs_cis, int32_t rope_dim,
+                                        int32_t max_pos, void *out, uint8_t *out_block_scales,
+                                        float *out_scales, int64_t num_slots, int32_t *status,
+                                        void *stream) {
+    if (out_kind != CSA_OUT_INDEX_BF16 && out_kind != CSA_OUT_INDEX_FP8 &&
+        out_kind != CSA_OUT_INDEX_FP4)
+        return CSA_ERR_UNSUPPORTED;
+    if (!rope_ok(freqs_cis, rope_dim, max_pos, dim)) return CSA_ERR_INVALID;
+    csa::RopeArgs rope;
+    rope.freqs = reinterpret_cast<const float2 *>(freqs_cis);
+    rope.rope_dim = rope_dim;
+    rope.max_pos = max_pos;
+    return c4_compress(x, gate, bias, dim, bs, cu_x, total_rows, start_pos, max_rows_per_req,
+                       page_table, page_table_stride, out_kind, out, out_block_scales, out_scales,
+                       num_slots, status, stream, rope);
 }
 
 csa_status_t csa_hca_compress(const float *x, const float *gate, const float *bias,
@@ -105,10 +144,11 @@ csa_status_t csa_hca_compress(const float *x, const float *gate, const float *bi
                                                 as_stream(stream)));
 }
 
-csa_status_t csa_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+static csa_status_t index_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
                                 int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
                                 void *codes, uint8_t *block_scales, float *scales,
-                                const float *w_in, float *w_out, int32_t *status, void *stream) {
+                                const float *w_in, float *w_out, int32_t *status, void *stream,
+                                bool rotate, const csa::RopeArgs &rope) {
     if (rows < 0) return CSA_ERR_INVALID;
     if (x_dtype != CSA_FMT_BF16 && x_dtype != CSA_FMT_F32) return CSA_ERR_UNSUPPORTED;
     if (dim != 64 && dim != 128) return CSA_ERR_UNSUPPORTED;
@@ -119,10 +159,46 @@ csa_status_t csa_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, in
     if (row_map && num_out_rows < 0) return CSA_ERR_INVALID;
     return cuda_status(csa::launch_hadamard_quant(x, x_dtype, rows, dim, fmt, row_map,
                                                   num_out_rows, codes, block_scales, scales,
-                                                  w_in, w_out, status, as_stream(stream)));
+                                                  w_in, w_out, status, as_stream(stream), rotate,
+                                                  rope));
 }
 
-csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
+csa_status_t csa_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                                int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
+                                void *codes, uint8_t *block_scales, float *scales,
+                                const float *w_in, float *w_out, int32_t *status, void *stream) {
+    return index_quant(x, x_dtype, rows, dim, fmt, row_map, num_out_rows, codes, block_scales,
+                       scales, w_in, w_out, status, stream, true, csa::RopeArgs());
+}
+
+csa_status_t csa_index_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                             int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
+                             void *codes, uint8_t *block_scales, float *scales,
+                             const float *w_in, float *w_out, int32_t *status, void *stream) {
+    return index_quant(x, x_dtype, rows, dim, fmt, row_map, num_out_rows, codes, block_scales,
+                       scales, w_in, w_out, status, stream, false, csa::RopeArgs());
+}
+
+csa_status_t csa_rope_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                                     const float *freqs_cis, int32_t rope_dim, int32_t max_pos,
+                                     const int32_t *positions, int32_t rows_per_pos, int32_t fmt,
+                                     const int32_t *row_map, int64_t num_out_rows, void *codes,
+                                     uint8_t *block_scales, float *scales, const float *w_in,
+                                     float *w_out, int32_t *status, void *stream) {
+    if (rows < 0 || rows_per_pos < 1) return CSA_ERR_INVALID;
+    if (rows == 0) return CSA_OK;
+    if (!positions || !rope_ok(freqs_cis, rope_dim, max_pos, dim)) return CSA_ERR_INVALID;
+    csa::RopeArgs rope;
+    rope.freqs = reinterpret_cast<const float2 *>(freqs_cis);
+    rope.pos = positions;
+    rope.rope_dim = rope_dim;
+    rope.max_pos = max_pos;
+    rope.rows_per_pos = rows_per_pos;
+    return index_quant(x, x_dtype, rows, dim, fmt, row_map, num_out_rows, codes, block_scales,
+                       scales, w_in, w_out, status, stream, true, rope);
+}
+
+static csa_status_t indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
                                 const float *q_weights, int32_t num_q, int32_t idx_heads,
                                 int32_t idx_dim, int32_t fmt, const void *k_codes,
                                 const uint8_t *k_block_scales, const float *k_scales,
@@ -130,7 +206,7 @@ csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scal
                                 int32_t page_table_stride, const int32_t *c4_seq_lens,
                                 int32_t bs, const int32_t *cu_q, const int32_t *q_pos,
                                 int32_t max_c4_len, float *logits, int64_t logits_stride,
-                                int32_t *status, void *stream) {
+                                int32_t *status, void *stream, int ratio) {
     if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
     if (!index_fmt_ok(fmt)) return CSA_ERR_UNSUPPORTED;
     if (idx_dim != 64 && idx_dim != 128) return CSA_ERR_UNSUPPORTED;
@@ -146,7 +222,38 @@ csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scal
                        k_codes, k_block_scales, k_scales, num_slots, page_table,
                        page_table_stride, c4_seq_lens, bs, cu_q, q_pos, max_c4_len, logits,
                        logits_stride, status};
+    a.ratio = ratio;
     return cuda_status(csa::launch_indexer(a, as_stream(stream)));
+}
+
+csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
+                                const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                const uint8_t *k_block_scales, const float *k_scales,
+                                int64_t num_slots, const int32_t *page_table,
+                                int32_t page_table_stride, const int32_t *c4_seq_lens,
+                                int32_t bs, const int32_t *cu_q, const int32_t *q_pos,
+                                int32_t max_c4_len, float *logits, int64_t logits_stride,
+                                int32_t *status, void *stream) {
+    return indexer_logits(q_codes, q_block_scales, q_weights, num_q, idx_heads, idx_dim, fmt,
+                          k_codes, k_block_scales, k_scales, num_slots, page_table,
+                          page_table_stride, c4_seq_lens, bs, cu_q, q_pos, max_c4_len, logits,
+                          logits_stride, status, stream, CSA_C4_RATIO);
+}
+
+csa_status_t csa_dsa_indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
+                                    const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                    int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                    const uint8_t *k_block_scales, const float *k_scales,
+                                    int64_t num_slots, const int32_t *page_table,
+                                    int32_t page_table_stride, const int32_t *seq_lens,
+                                    int32_t bs, const int32_t *cu_q, const int32_t *q_pos,
+                                    int32_t max_seq_len, float *logits, int64_t logits_stride,
+                                    int32_t *status, void *stream) {
+    return indexer_logits(q_codes, q_block_scales, q_weights, num_q, idx_heads, idx_dim, fmt,
+                          k_codes, k_block_scales, k_scales, num_slots, page_table,
+                          page_table_stride, seq_lens, bs, cu_q, q_pos, max_seq_len, logits,
+                          logits_stride, status, stream, 1);
 }
 
 size_t csa_topk512_workspace_size(int32_t num_q, int32_t max_c4_len) {
@@ -154,14 +261,14 @@ size_t csa_topk512_workspace_size(int32_t num_q, int32_t max_c4_len) {
     return csa::topk_workspace_bytes(num_q, max_c4_len);
 }
 
-csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stride,
+static csa_status_t topk512(const float *logits, int64_t logits_stride,
                                         int32_t num_q, const int32_t *c4_seq_lens, int32_t bs,
                                         const int32_t *cu_q, const int32_t *q_pos,
                                         const int32_t *page_table, int32_t page_table_stride,
                                         int64_t num_slots, int32_t c4_page_size,
                                         int32_t max_c4_len, int32_t *c4_sparse_page_indices,
                                         int32_t *raw_indices, void *workspace,
-                                        size_t workspace_bytes, int32_t *status, void *stream) {
+                                        size_t workspace_bytes, int32_t *status, void *stream, int ratio) {
     if (num_q < 0 || bs < 0 || max_c4_len < 0 || page_table_stride < 0) return CSA_ERR_INVALID;
     if (c4_page_size != CSA_C4_PAGE_SIZE) return CSA_ERR_INVALID;
     if (num_q == 0) return CSA_OK;
@@ -174,7 +281,36 @@ csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stri
     csa::TopkArgs a{logits, logits_stride, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,
                     page_table_stride, num_slots, max_c4_len, c4_sparse_page_indices,
                     raw_indices, workspace, status};
+    a.ratio = ratio;
     return cuda_status(csa::launch_topk512(a, as_stream(stream)));
+}
+
+csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stride,
+                                        int32_t num_q, const int32_t *c4_seq_lens, int32_t bs,
+                                        const int32_t *cu_q, const int32_t *q_pos,
+                                        const int32_t *page_table, int32_t page_table_stride,
+                                        int64_t num_slots, int32_t c4_page_size,
+                                        int32_t max_c4_len, int32_t *c4_sparse_page_indices,
+                                        int32_t *raw_indices, void *workspace,
+                                        size_t workspace_bytes, int32_t *status, void *stream) {
+    return topk512(logits, logits_stride, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,
+                   page_table_stride, num_slots, c4_page_size, max_c4_len,
+                   c4_sparse_page_indices, raw_indices, workspace, workspace_bytes, status,
+                   stream, CSA_C4_RATIO);
+}
+
+csa_status_t csa_dsa_topk512_page_transform(const float *logits, int64_t logits_stride,
+                                            int32_t num_q, const int32_t *seq_lens, int32_t bs,
+                                            const int32_t *cu_q, const int32_t *q_pos,
+                                            const int32_t *page_table, int32_t page_table_stride,
+                                            int64_t num_slots, int32_t page_size,
+                                            int32_t max_seq_len, int32_t *sparse_page_indices,
+                                            int32_t *raw_indices, void *workspace,
+                                            size_t workspace_bytes, int32_t *status,
+                                            void *stream) {
+    return topk512(logits, logits_stride, num_q, seq_lens, bs, cu_q, q_pos, page_table,
+                   page_table_stride, num_slots, page_size, max_seq_len, sparse_page_indices,
+                   raw_indices, workspace, workspace_bytes, status, stream, 1);
 }
 
 size_t csa_indexer_topk512_workspace_size(int32_t num_q, int32_t bs, int32_t idx_heads,

@@ -88,7 +88,7 @@ indexer_simple_kernel(const IndexerArgs a) {
     }
     const int b = lo;
     int n = a.c4_seq_lens[b];
-    if (a.q_pos) n = min(n, (a.q_pos[t] + 1) / 4);
+    if (a.q_pos) n = min(n, (a.q_pos[t] + 1) / a.ratio);
     const int cap = min(a.max_c4_len, a.pt_stride * kC4Page);
     if (n > cap) {
         if (blockIdx.x == 0 && threadIdx.x == 0) report(a.status, CSA_ERR_BOUNDS);

@@ -115,7 +115,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         int n = 0;
         if (i < nq) {
             n = a.c4_seq_lens[b];
-            if (a.q_pos) n = min(n, (a.q_pos[t0 + i] + 1) / 4);
+            if (a.q_pos) n = min(n, (a.q_pos[t0 + i] + 1) / a.ratio);
             if (n > cap) {
                 if (threadIdx.x == 0 && blockIdx.x == 0) report(a.status, CSA_ERR_BOUNDS);
                 n = cap;

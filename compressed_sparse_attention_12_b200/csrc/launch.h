@@ -44,10 +44,20 @@ inline cudaError_t ensure_max_smem(const void *fn, int bytes, int *done) {
 cudaError_t launch_kv_store(const float *rows, int64_t n, const int32_t *slots, int fmt,
                             void *cache, int64_t num_slots, int32_t *status, cudaStream_t s);
 
+// Rotary embedding ahead of the rotation + quantisation: freqs [max_pos][rope_dim/2]
+// (cos, sin) pairs; row r of the input sits at position pos[r / rows_per_pos].
+// freqs == nullptr: no rotary embedding.
+struct RopeArgs {
+    const float2 *freqs = nullptr;
+    const int32_t *pos = nullptr;
+    int rope_dim = 0, max_pos = 0, rows_per_pos = 1;
+};
+
 cudaError_t launch_hadamard_quant(const void *x, int x_dtype, int64_t rows, int dim, int fmt,
                                   const int32_t *row_map, int64_t num_out_rows, void *codes,
                                   uint8_t *block_scales, float *scales, const float *w_in,
-                                  float *w_out, int32_t *status, cudaStream_t s);
+                                  float *w_out, int32_t *status, cudaStream_t s,
+                                  bool rotate = true, const RopeArgs &rope = RopeArgs());
 
 cudaError_t launch_hca_compress(const float *x, const float *gate, const float *bias, int bs,
                                 const int32_t *cu_x, const int32_t *start_pos, int max_rows,
@@ -59,7 +69,7 @@ cudaError_t launch_c4_compress(const float *x, const float *gate, const float *b
                                int max_rows, const int32_t *page_table, int pt_stride,
                                int out_kind, void *out, uint8_t *out_block_scales,
                                float *out_scales, int64_t num_slots, int32_t *status,
-                               cudaStream_t s);
+                               cudaStream_t s, const RopeArgs &rope = RopeArgs());
 
 // Shape of one indexer launch (validated by the caller).
 struct IndexerArgs {
@@ -81,6 +91,7 @@ struct IndexerArgs {
     float *logits;
     int64_t logits_stride;
     int32_t *status;
+    int ratio = 4;      // raw tokens per key: visible keys s < floor((p+1)/ratio)
 };
 cudaError_t launch_indexer(const IndexerArgs &a, cudaStream_t s);
 
@@ -102,6 +113,7 @@ struct TopkArgs {
     int32_t *out_raw;
     void *workspace;
     int32_t *status;
+    int ratio = 4;      // raw tokens per key, as in IndexerArgs
 };
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s);
 // Same, with the scratch in the library's own device array (no workspace).

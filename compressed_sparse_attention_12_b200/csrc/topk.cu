@@ -40,7 +40,7 @@ struct RowInfo {
 // published to the block through shared memory.
 __device__ RowInfo row_info(int t, const int32_t *cu_q, int bs, const int32_t *q_pos,
                             const int32_t *c4_lens, int max_c4_len, int pt_stride,
-                            int32_t *status, bool leader, TkShared &sh) {
+                            int32_t *status, bool leader, TkShared &sh, int ratio) {
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         const int pos = q_pos ? q_pos[t] : 0;
@@ -60,7 +60,7 @@ __device__ RowInfo row_info(int t, const int32_t *cu_q, int bs, const int32_t *q
         }
         if (lane == 0) {
             int n = len;
-            if (q_pos) n = min(n, (pos + 1) / 4);
+            if (q_pos) n = min(n, (pos + 1) / ratio);
             const int cap = min(max_c4_len, pt_stride * kC4Page);
             if (n > cap) {
                 if (leader) report(status, CSA_ERR_BOUNDS);
@@ -84,14 +84,14 @@ __global__ void __launch_bounds__(kTkThreads)
 topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens,
                    int bs, const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
                    int pt_stride, int max_chunks, uint32_t *cand_key, int32_t *cand_idx,
-                   uint2 *chunk_info, int32_t *status) {
+                   uint2 *chunk_info, int32_t *status, int ratio) {
     pdl_begin();
     extern __shared__ __align__(16) uint8_t tk_smem[];
     TkShared &sh = *reinterpret_cast<TkShared *>(tk_smem);
     uint32_t *skeys = reinterpret_cast<uint32_t *>(tk_smem + kTkKeysOffset);
     const int t = blockIdx.y, c = blockIdx.x;
     const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
-                                c == 0, sh);
+                                c == 0, sh, ratio);
     const int lo = c * kTkChunk;
     if (lo >= ri.n_vis) return;
     const int len = min(kTkChunk, ri.n_vis - lo);
@@ -121,8 +121,7 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
                    int max_c4_len, const int32_t *page_table, int pt_stride, int64_t num_slots,
                    int max_chunks, int chunk_len, const uint32_t *cand_key,
                    const int32_t *cand_idx, const uint2 *chunk_info, int32_t *out_phys,
-                   int32_t *out_raw,
-                   int32_t *status) {
+                   int32_t *out_raw, int32_t *status, int ratio) {
     pdl_begin();
     extern __shared__ __align__(16) uint8_t tk2_smem[];
     TkShared &sh = *reinterpret_cast<TkShared *>(tk2_smem);
@@ -130,7 +129,7 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
     int32_t *sidx = reinterpret_cast<int32_t *>(skeys + kTk2Smem);
     const int t = blockIdx.x;
     const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
-                                false, sh);
+                                false, sh, ratio);
     const int n = ri.n_vis;
     int total = 0, nch = 0;
     if (n > 0) {
@@ -290,7 +289,7 @@ cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
     dim3 g1(mc, a.num_q);
     launch_k(topk_stage1_kernel, g1, kTkThreads, smem1, s, a.logits, a.logits_stride, a.c4_seq_lens, a.bs,
                                                  a.cu_q, a.q_pos, a.max_c4_len, a.pt_stride, mc,
-                                                 ck, ci, info, a.status);
+                                                 ck, ci, info, a.status, a.ratio);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_topk_stage2(a, mc, kTkChunk, ck, ci, info, s);
@@ -305,7 +304,7 @@ cudaError_t launch_topk_stage2(const TopkArgs &a, int max_chunks, int chunk_len,
     if (e != cudaSuccess) return e;
     launch_k(topk_stage2_kernel, a.num_q, kTkThreads, smem2, s, a.c4_seq_lens, a.bs, a.cu_q,
              a.q_pos, a.max_c4_len, a.page_table, a.pt_stride, a.num_slots, max_chunks, chunk_len,
-             cand_key, cand_idx, chunk_info, a.out_phys, a.out_raw, a.status);
+             cand_key, cand_idx, chunk_info, a.out_phys, a.out_raw, a.status, a.ratio);
     return cudaGetLastError();
 }
 

@@ -410,6 +410,98 @@ csa_status_t csa_hca_attention(const void *q, int32_t num_q, int32_t heads, cons
                                float *lse, void *workspace, size_t workspace_bytes,
                                int32_t *status, void *stream);
 
+/*
+ * Fused rotary embedding ahead of the rotation + quantisation ([T] §3.1
+ * fused_q_indexer_rope_hadamard[_fp4]_quant and §4: Q goes rope -> Hadamard ->
+ * quant; K goes rope -> Hadamard -> quant -> index K cache).
+ *
+ * Rotary embedding: the leading rope_dim values of a row, taken as rope_dim/2
+ * complex numbers x[2i] + i*x[2i+1], are multiplied by freqs_cis[pos][i]:
+ *   x'[2i]   = x[2i]*cos - x[2i+1]*sin,   x'[2i+1] = x[2i]*sin + x[2i+1]*cos
+ * (float32, each product and sum rounded separately); the remaining
+ * dim - rope_dim values pass unchanged.
+ *   freqs_cis   [max_pos, rope_dim/2, 2] float32 (cos, sin), 8-byte aligned,
+ *               caller-owned; the library never builds the table
+ *   rope_dim    even, 2 <= rope_dim <= dim
+ *
+ * csa_rope_hadamard_quant -- csa_hadamard_quant with the rotary embedding
+ * first.  Row r of x sits at raw position positions[r / rows_per_pos]
+ * (rows_per_pos = idx_heads for index queries laid out [num_q, idx_heads,
+ * dim], 1 for keys).  A position outside [0, max_pos) records CSA_ERR_BOUNDS
+ * and leaves that row unwritten (and its w_out).  Other arguments as
+ * csa_hadamard_quant.
+ */
+csa_status_t csa_rope_hadamard_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                                     const float *freqs_cis, int32_t rope_dim, int32_t max_pos,
+                                     const int32_t *positions, int32_t rows_per_pos, int32_t fmt,
+                                     const int32_t *row_map, int64_t num_out_rows, void *codes,
+                                     uint8_t *block_scales, float *scales, const float *w_in,
+                                     float *w_out, int32_t *status, void *stream);
+
+/*
+ * csa_c4_compress_index_rope -- csa_c4_compress in an index-key mode
+ * (out_kind CSA_OUT_INDEX_*) with the rotary embedding applied to each pooled
+ * key between the pooling and the rotation, in the same pass: pool ->
+ * rope -> Hadamard -> quant -> index K cache.  The compressed key of block j
+ * (raw rows 4j..4j+3) takes the raw position 4j of the block's first row; a
+ * position >= max_pos records CSA_ERR_BOUNDS and leaves the key unwritten.
+ * Other arguments and errors as csa_c4_compress.
+ */
+csa_status_t csa_c4_compress_index_rope(const float *x, const float *gate, const float *bias,
+                                        int32_t dim, int32_t bs, const int32_t *cu_x,
+                                        int64_t total_rows, const int32_t *start_pos,
+                                        int32_t max_rows_per_req, const int32_t *page_table,
+                                        int32_t page_table_stride, int32_t out_kind,
+                                        const float *freqs_cis, int32_t rope_dim,
+                                        int32_t max_pos, void *out, uint8_t *out_block_scales,
+                                        float *out_scales, int64_t num_slots, int32_t *status,
+                                        void *stream);
+
+/*
+ * DSA comparison path ([T] §1 从 DSA 到 DSV4: the DSA indexer picks the top-k
+ * raw tokens, no compression; its index K cache is FP8 (§3.1) and is not
+ * Hadamard-rotated (§4); its pages hold 64 raw tokens).  The same kernels as
+ * the C4 path with one key per raw token: a query at raw position p sees the
+ * keys s <= p (s < min(seq_lens[b], p+1)), and key s of request b sits at
+ * slot page_table[b*stride + s/64]*64 + s%64 of a cache paged by 64 tokens.
+ * The attention over the selected raw rows is csa_sparse_mqa_decode/_prefill
+ * with c4_cache = that 64-token-paged KV cache and window = 0.
+ *
+ * csa_index_quant -- csa_hadamard_quant without the rotation (the row is
+ * quantised as given).
+ *
+ * csa_dsa_indexer_logits -- csa_indexer_logits over raw tokens: seq_lens are
+ * raw lengths, n_vis = min(seq_lens[b], p+1), max_seq_len bounds seq_lens[].
+ *
+ * csa_dsa_topk512_page_transform -- csa_topk512_page_transform over raw
+ * tokens (the same n_vis); page_size must be CSA_DSA_PAGE_SIZE (64); the
+ * workspace is csa_topk512_workspace_size(num_q, max_seq_len) bytes.
+ */
+enum { CSA_DSA_PAGE_SIZE = 64 };
+
+csa_status_t csa_index_quant(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                             int32_t fmt, const int32_t *row_map, int64_t num_out_rows,
+                             void *codes, uint8_t *block_scales, float *scales,
+                             const float *w_in, float *w_out, int32_t *status, void *stream);
+csa_status_t csa_dsa_indexer_logits(const void *q_codes, const uint8_t *q_block_scales,
+                                    const float *q_weights, int32_t num_q, int32_t idx_heads,
+                                    int32_t idx_dim, int32_t fmt, const void *k_codes,
+                                    const uint8_t *k_block_scales, const float *k_scales,
+                                    int64_t num_slots, const int32_t *page_table,
+                                    int32_t page_table_stride, const int32_t *seq_lens,
+                                    int32_t bs, const int32_t *cu_q, const int32_t *q_pos,
+                                    int32_t max_seq_len, float *logits, int64_t logits_stride,
+                                    int32_t *status, void *stream);
+csa_status_t csa_dsa_topk512_page_transform(const float *logits, int64_t logits_stride,
+                                            int32_t num_q, const int32_t *seq_lens, int32_t bs,
+                                            const int32_t *cu_q, const int32_t *q_pos,
+                                            const int32_t *page_table, int32_t page_table_stride,
+                                            int64_t num_slots, int32_t page_size,
+                                            int32_t max_seq_len, int32_t *sparse_page_indices,
+                                            int32_t *raw_indices, void *workspace,
+                                            size_t workspace_bytes, int32_t *status,
+                                            void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -191,3 +191,53 @@ def test_hca_attention_too_long_is_unsupported():
                               dev(c["L"].astype(np.int32)), dev(c["cu_q"]), dev(c["q_pos"]),
                               csa.HCA_MAX_ROWS, 128, 0.04, True, out)
     assert e.value.code == csa.CSA_ERR_UNSUPPORTED
+
+
+def _hca_step_check(name, scale, sample=None):
+    """A whole HCA-layer step (compressor + dense attention) through HcaBatch, in
+    the benchmark's launch shapes, against oracle.hca_step on the same drawn
+    buffers (each side encodes its own caches)."""
+    from compressed_sparse_attention_12_b200 import pipeline, synth
+    w = synth.workload(name, scale)
+    data = synth.draw_hca(w, "cuda")
+    batch = pipeline.HcaBatch(w, data)
+    batch.step()
+    torch.cuda.synchronize()
+    batch.check_status()
+    reqs = None
+    if sample is not None:
+        reqs = sorted(set(int(np.searchsorted(w.cu_q, t, side="right") - 1) for t in sample))
+    ref = orc.hca_step(w, data, batch.pt_host, requests=reqs, sm_scale=batch.sm_scale)
+    go = batch.out.float().cpu().numpy()
+    gl = batch.lse.cpu().numpy()
+    tol = 2e-2 if w.kv_fmt == "fp8" else 5e-3
+    rows = sample if sample is not None else sorted(ref)
+    assert rows
+    for t in rows:
+        r = ref[t]
+        err = np.abs(go[t] - r["out"]) - bf16_bound(r["out"], rel=0.0)
+        assert err.max() <= tol, (t, err.max())
+        assert np.abs(gl[t] - r["lse"]).max() <= 2e-2, t
+    return w, ref
+
+
+@pytest.mark.parametrize("name,scale", [("hca_128k", 1 / 64), ("hca_1m", 1 / 64),
+                                        ("hca_prefill", 1 / 16)])
+def test_hca_step_end_to_end(name, scale):
+    w, ref = _hca_step_check(name, scale)
+    # the step's compressor wrote at least one of the rows attended to
+    from compressed_sparse_attention_12_b200 import synth
+    assert synth.hca_plan(w)[1].sum() > 0
+
+
+def test_hca_full_size_decode_128k():
+    _hca_step_check("hca_128k", 1.0)
+
+
+def test_hca_full_size_decode_1m():
+    _hca_step_check("hca_1m", 1.0)
+
+
+def test_hca_full_size_prefill_sampled():
+    # first, a middle and the last query tokens of the 4096-token prefill
+    _hca_step_check("hca_prefill", 1.0, sample=[0, 1, 127, 2047, 4094, 4095])
