@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--workload", default="decode_128k")
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--topk-form", default="auto", choices=["auto", "fused", "separate"],
+                   help="indexer + top-512 form: the selecting indexer + row merge, the plain "
+                        "indexer + top-k, or whichever probes faster (default)")
     p.add_argument("--profile", action="store_true",
                    help="profiling run: no CPU baseline or end-to-end leg; the drawn float "
                         "inputs are freed once the caches are built")
@@ -661,12 +664,14 @@ def main():
 
     fused = [True]
     candidates = []
-    try:
-        candidates.append((True,) + capture(True))
-    except csa.CsaError as e:
-        if e.code != csa.CSA_ERR_UNSUPPORTED:
-            raise
-    candidates.append((False,) + capture(False))
+    if args.topk_form in ("auto", "fused"):
+        try:
+            candidates.append((True,) + capture(True))
+        except csa.CsaError as e:
+            if e.code != csa.CSA_ERR_UNSUPPORTED or args.topk_form == "fused":
+                raise
+    if args.topk_form in ("auto", "separate"):
+        candidates.append((False,) + capture(False))
     best = min(candidates, key=lambda c: c[2])
     fused[0], g = best[0], best[1]
     topk_forms = {("fused" if c[0] else "separate"): round(c[2] * 1e3, 2) for c in candidates}

@@ -217,6 +217,8 @@ struct AtSmem8 {
     float qmul[G * kAtHeads];                     // power-of-two scale of each query head
     float red_max[G][4][kAtHeads];
     float red_sum[G][4][kAtHeads];
+    // per warp of a group, its block's partial scores [head][row] (rows padded)
+    alignas(16) float red_s[G][4][kAtHeads][kAtPStride];
     int32_t slot[kAtMaxTiles * kAtRows];          // row slots of the split's tiles (-1: masked)
     int8_t is_raw[kAtMaxTiles * kAtRows];
     int16_t tiles[kAtMaxTiles];                   // non-empty tiles of this split (local index)
@@ -329,7 +331,10 @@ template <int G>
 __global__ void __launch_bounds__(kAtThreads * G, G == 1 ? 2 : 1)
 sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *part_o,
                       float *part_ml) {
-    pdl_begin();
+    // Only inputs of the step (q, cu_q, q_pos, seq_lens) are read before the
+    // wait on the preceding kernel: the query rows are loaded and converted
+    // while it finishes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int kThr = kAtThreads * G;
     extern __shared__ __align__(16) uint8_t at_smem_raw[];
     AtSmem8<G> &sm = *reinterpret_cast<AtSmem8<G> *>(at_smem_raw);
@@ -342,14 +347,7 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
     const int n_rows = qq.nsel + qq.nw;
     const int tile0 = sp * tiles_per_split;
     const int tile1 = min((n_rows + kAtRows - 1) / kAtRows, tile0 + tiles_per_split);
-
     const int n_local = max(0, tile1 - tile0);
-    for (int u = tid; u < n_local * kAtRows; u += kThr) {
-        int32_t raw;
-        const int32_t slot = row_slot(a, qq, t, tile0 * kAtRows + u, &raw);
-        sm.slot[u] = slot;
-        sm.is_raw[u] = (int8_t)raw;
-    }
     {
         const __nv_bfloat16 *qsrc = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                                     ((int64_t)t * a.heads + blockIdx.y * G * kAtHeads) * kKvDim;
@@ -359,28 +357,10 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
         }
         cp_async_commit();
     }
-    __syncthreads();
-    for (int lt = warp; lt < n_local; lt += 4 * G) {
-        const bool any = __any_sync(0xffffffffu, sm.slot[lt * kAtRows + lane] >= 0);
-        if (lane == 0) sm.tiles[lt] = any ? 1 : 0;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int n = 0;
-        for (int lt = 0; lt < n_local; lt++)
-            if (sm.tiles[lt]) sm.tiles[n++] = (int16_t)lt;
-        sm.n_tiles = n;
-    }
-    __syncthreads();
-    const int nt = sm.n_tiles;
-    for (int j = 0; j < 2; j++) {
-        if (j < nt) issue_loads8(a, sm.tiles[j], j, sm);
-        else cp_async_commit();
-    }
     // Q to fp16 in place: warp w converts heads 4w..4w+3, each times a power
     // of two that brings its largest magnitude into [2^13, 2^14), so every
     // bf16 value above 2^-30 of that maximum converts exactly
-    cp_async_wait<2>();
+    cp_async_wait<0>();
     __syncthreads();
     {
         uint16_t *qh = reinterpret_cast<uint16_t *>(sm.q);
@@ -402,7 +382,32 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
             if (lane == 0) sm.qmul[h] = 1.0f / m;
         }
     }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    for (int u = tid; u < n_local * kAtRows; u += kThr) {
+        int32_t raw;
+        const int32_t slot = row_slot(a, qq, t, tile0 * kAtRows + u, &raw);
+        sm.slot[u] = slot;
+        sm.is_raw[u] = (int8_t)raw;
+    }
     __syncthreads();
+    for (int lt = warp; lt < n_local; lt += 4 * G) {
+        const bool any = __any_sync(0xffffffffu, sm.slot[lt * kAtRows + lane] >= 0);
+        if (lane == 0) sm.tiles[lt] = any ? 1 : 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int n = 0;
+        for (int lt = 0; lt < n_local; lt++)
+            if (sm.tiles[lt]) sm.tiles[n++] = (int16_t)lt;
+        sm.n_tiles = n;
+    }
+    __syncthreads();
+    const int nt = sm.n_tiles;
+    for (int j = 0; j < 2; j++) {
+        if (j < nt) issue_loads8(a, sm.tiles[j], j, sm);
+        else cp_async_commit();
+    }
 
     float qscale[2];
 #pragma unroll
@@ -420,6 +425,8 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
     const __half *tile = reinterpret_cast<const __half *>(sm.region + 2 * kStageBytes);
     const uint32_t k_base =
         smem_u32(tile) + (uint32_t)((wq * 8 + (lane & 7)) * kAtStride + (lane >> 3) * 8) * 2;
+    const uint32_t kb_base =
+        smem_u32(tile) + (uint32_t)((lane & 7) * kAtStride + (lane >> 3) * 8) * 2;
     const uint32_t v_base =
         smem_u32(tile) + (uint32_t)(((lane & 7) + ((lane >> 3) & 1) * 8) * kAtStride + wq * 128 +
                                     (lane >> 4) * 8) * 2;
@@ -433,26 +440,67 @@ sparse_mqa_fp8_kernel(const AttnArgs a, int splits, int tiles_per_split, float *
         expand8(lt, st, sm);
         __syncthreads();
 
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int blk = 0; blk < 5; blk++) {
-            float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-            const int k0 = blk * 8, nk = blk < 4 ? 8 : 4;
-#pragma unroll 4
-            for (int kk = k0; kk < k0 + nk; kk += 2) {
-                uint32_t a0[4], a1[4], bf[4];
-                ldsm_x4(a0, q_base + kk * 32);
-                ldsm_x4(a1, q_base + (kk + 1) * 32);
-                ldsm_x4(bf, k_base + kk * 32);
-                mma16816_f16(acc0, a0, bf[0], bf[1]);
-                mma16816_f16(acc1, a1, bf[2], bf[3]);
-            }
+        // S = Q K^T split by channel block: warp wq takes latent block wq
+        // (8 k-steps) for all 32 rows and the RoPE block (4 k-steps) for rows
+        // 8wq..8wq+7; each partial is scaled by its rows' block scale, and the
+        // four warps' partials are summed through shared memory.
+        float sl[4][4], sr[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int jj = 0; jj < 4; jj++) {
-                const int row = wq * 8 + 2 * tq + (jj & 1);
-                const float sc = blk < 4 ? sm.rscale[st][row][blk] : sm.rope_mul[st][row];
-                s[jj] = fmaf(acc0[jj] + acc1[jj], sc, s[jj]);
+        for (int nb = 0; nb < 4; nb++) sl[nb][0] = sl[nb][1] = sl[nb][2] = sl[nb][3] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int kk = 8 * wq + 2 * i;
+            uint32_t a0[4], a1[4];
+            ldsm_x4(a0, q_base + kk * 32);
+            ldsm_x4(a1, q_base + (kk + 1) * 32);
+#pragma unroll
+            for (int nb = 0; nb < 4; nb++) {
+                uint32_t bf[4];
+                ldsm_x4(bf, kb_base + (uint32_t)(nb * 8 * kAtStride * 2 + kk * 32));
+                mma16816_f16(sl[nb], a0, bf[0], bf[1]);
+                mma16816_f16(sl[nb], a1, bf[2], bf[3]);
             }
+        }
+#pragma unroll
+        for (int i = 0; i < 2; i++) {
+            const int kk = 32 + 2 * i;
+            uint32_t a0[4], a1[4], bf[4];
+            ldsm_x4(a0, q_base + kk * 32);
+            ldsm_x4(a1, q_base + (kk + 1) * 32);
+            ldsm_x4(bf, k_base + kk * 32);
+            mma16816_f16(sr, a0, bf[0], bf[1]);
+            mma16816_f16(sr, a1, bf[2], bf[3]);
+        }
+        {
+            float (*rs)[kAtPStride] = sm.red_s[grp][wq];
+#pragma unroll
+            for (int nb = 0; nb < 4; nb++) {
+                const int r0 = nb * 8 + 2 * tq;
+                const float c0 = sm.rscale[st][r0][wq], c1 = sm.rscale[st][r0 + 1][wq];
+                float v0 = sl[nb][0] * c0, v1 = sl[nb][1] * c1;
+                float v2 = sl[nb][2] * c0, v3 = sl[nb][3] * c1;
+                if (nb == wq) {
+                    const float e0 = sm.rope_mul[st][r0], e1 = sm.rope_mul[st][r0 + 1];
+                    v0 = fmaf(sr[0], e0, v0);
+                    v1 = fmaf(sr[1], e1, v1);
+                    v2 = fmaf(sr[2], e0, v2);
+                    v3 = fmaf(sr[3], e1, v3);
+                }
+                *reinterpret_cast<float2 *>(&rs[gq][r0]) = make_float2(v0, v1);
+                *reinterpret_cast<float2 *>(&rs[gq + 8][r0]) = make_float2(v2, v3);
+            }
+        }
+        group_sync(grp);
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+            const float2 x = *reinterpret_cast<const float2 *>(&sm.red_s[grp][w][gq][wq * 8 + 2 * tq]);
+            const float2 y =
+                *reinterpret_cast<const float2 *>(&sm.red_s[grp][w][gq + 8][wq * 8 + 2 * tq]);
+            s[0] += x.x;
+            s[1] += x.y;
+            s[2] += y.x;
+            s[3] += y.y;
         }
         float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll

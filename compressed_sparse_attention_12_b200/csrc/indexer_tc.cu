@@ -426,12 +426,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     for (int x = 0; x < nq; x++) {
         const int len = min(tile_end * kTcTile, nv_s[x]) - k0;
         if (len <= 0) continue;                    // uniform over the CTA
-        const float *row = a.logits + (int64_t)(t0 + x) * a.logits_stride + k0;
-        const int n4 = (reinterpret_cast<uintptr_t>(row) & 15) == 0 ? len / 4 : 0;
-        for (int i = threadIdx.x; i < n4; i += kTcThreads)
-            reinterpret_cast<uint4 *>(skeys)[i] = reinterpret_cast<const uint4 *>(row)[i];
-        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTcThreads)
-            skeys[i] = __float_as_uint(row[i]);
+        stage_row_keys<kTcThreads>(skeys, a.logits + (int64_t)(t0 + x) * a.logits_stride + k0,
+                                   len);
         __syncthreads();
         const int64_t c = (int64_t)(t0 + x) * sel.max_chunks + blockIdx.x;
         select_chunk<kTcThreads>(skeys, len, k0, sel.cand_key + c * kTopK, sel.cand_idx + c * kTopK,

@@ -38,9 +38,10 @@ struct RowInfo {
 // Request and visible length of query row t, found by warp 0 with coalesced
 // reads of cu_q and c4_lens (one round trip for up to 32 requests) and
 // published to the block through shared memory.
+template <int NT>
 __device__ RowInfo row_info(int t, const int32_t *cu_q, int bs, const int32_t *q_pos,
                             const int32_t *c4_lens, int max_c4_len, int pt_stride,
-                            int32_t *status, bool leader, TkShared &sh, int ratio) {
+                            int32_t *status, bool leader, TkSharedT<NT> &sh, int ratio) {
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         const int pos = q_pos ? q_pos[t] : 0;
@@ -90,21 +91,12 @@ topk_stage1_kernel(const float *__restrict__ logits, int64_t stride, const int32
     TkShared &sh = *reinterpret_cast<TkShared *>(tk_smem);
     uint32_t *skeys = reinterpret_cast<uint32_t *>(tk_smem + kTkKeysOffset);
     const int t = blockIdx.y, c = blockIdx.x;
-    const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
-                                c == 0, sh, ratio);
+    const RowInfo ri = row_info<kTkThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride,
+                                            status, c == 0, sh, ratio);
     const int lo = c * kTkChunk;
     if (lo >= ri.n_vis) return;
     const int len = min(kTkChunk, ri.n_vis - lo);
-    const float *row = logits + (int64_t)t * stride + lo;
-    if ((reinterpret_cast<uintptr_t>(row) & 15) == 0) {
-        const int n4 = len / 4;
-        for (int i = threadIdx.x; i < n4; i += kTkThreads)
-            reinterpret_cast<uint4 *>(skeys)[i] = reinterpret_cast<const uint4 *>(row)[i];
-        for (int i = 4 * n4 + threadIdx.x; i < len; i += kTkThreads)
-            skeys[i] = __float_as_uint(row[i]);
-    } else {
-        for (int i = threadIdx.x; i < len; i += kTkThreads) skeys[i] = __float_as_uint(row[i]);
-    }
+    stage_row_keys<kTkThreads>(skeys, logits + (int64_t)t * stride + lo, len);
     __syncthreads();
     select_chunk<kTkThreads>(skeys, len, lo, cand_key + ((int64_t)t * max_chunks + c) * kTopK,
                              cand_idx + ((int64_t)t * max_chunks + c) * kTopK,
@@ -128,8 +120,8 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
     uint32_t *skeys = reinterpret_cast<uint32_t *>(tk2_smem + kTkKeysOffset);
     int32_t *sidx = reinterpret_cast<int32_t *>(skeys + kTk2Smem);
     const int t = blockIdx.x;
-    const RowInfo ri = row_info(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
-                                false, sh, ratio);
+    const RowInfo ri = row_info<kTkThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride,
+                                            status, false, sh, ratio);
     const int n = ri.n_vis;
     int total = 0, nch = 0;
     if (n > 0) {
@@ -265,6 +257,114 @@ topk_stage2_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const in
     }
 }
 
+// Rows of at most kTkRowMax logits in one launch: one CTA of 1024 threads per
+// query row stages the whole row in shared memory as keys, selects its
+// top-512 and writes the physical slots, raw indices and -1 padding.
+constexpr int kTkRowThreads = 1024;
+constexpr int kTkRowMax = 49152;
+using TkRowShared = TkSharedT<kTkRowThreads>;
+constexpr size_t kTkRowKeysOffset = (sizeof(TkRowShared) + 15) & ~(size_t)15;
+
+__global__ void __launch_bounds__(kTkRowThreads, 1)
+topk_row_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens, int bs,
+                const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
+                const int32_t *page_table, int pt_stride, int64_t num_slots, int32_t *out_phys,
+                int32_t *out_raw, int32_t *status, int ratio) {
+    pdl_begin();
+    extern __shared__ __align__(16) uint8_t tkr_smem[];
+    TkRowShared &sh = *reinterpret_cast<TkRowShared *>(tkr_smem);
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(tkr_smem + kTkRowKeysOffset);
+    const int t = blockIdx.x;
+    const RowInfo ri = row_info<kTkRowThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len,
+                                               pt_stride, status, true, sh, ratio);
+    const int len = min(ri.n_vis, kTkRowMax);     // the host keeps max_c4_len <= kTkRowMax
+    stage_row_keys<kTkRowThreads>(skeys, logits + (int64_t)t * stride, len);
+    __syncthreads();
+    const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
+    int32_t *op = out_phys + (int64_t)t * kTopK;
+    int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
+    uint32_t T, kmax;
+    const int K = select_top512<kTkRowThreads>(skeys, len, sh, status, &T, &kmax,
+                                               [&](int pos, int s, uint32_t) {
+        const int32_t page = pt_row[s / kC4Page];
+        const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
+        int32_t phys = (int32_t)slot;
+        if (page < 0 || slot >= num_slots) {
+            report(status, CSA_ERR_BOUNDS);
+            phys = -1;
+        }
+        op[pos] = phys;
+        if (orw) orw[pos] = s;
+    });
+    for (int p = K + threadIdx.x; p < kTopK; p += kTkRowThreads) {
+        op[p] = -1;
+        if (orw) orw[p] = -1;
+    }
+}
+
+// Rows of at most kTkRegMax logits: one CTA of 1024 threads per query row
+// holds the row in registers (32 keys per thread, loaded in coalesced 16-byte
+// slices), so every sweep over the row is register-only; shared memory holds
+// the radix histogram and the staged candidates.
+constexpr int kTkRegKpt = 32;
+constexpr int kTkRegMax = kTkRowThreads * kTkRegKpt;
+constexpr int kTkRegCap = 3072;      // staged candidates (keys >= the group bound)
+
+__global__ void __launch_bounds__(kTkRowThreads, 1)
+topk_reg_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens, int bs,
+                const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
+                const int32_t *page_table, int pt_stride, int64_t num_slots, int32_t *out_phys,
+                int32_t *out_raw, int32_t *status, int ratio) {
+    pdl_begin();
+    __shared__ TkRowShared sh;
+    __shared__ uint32_t cand_key[kTkRegCap];
+    __shared__ int32_t cand_idx[kTkRegCap];
+    const int t = blockIdx.x;
+    const RowInfo ri = row_info<kTkRowThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len,
+                                               pt_stride, status, true, sh, ratio);
+    const int len = min(ri.n_vis, kTkRegMax);     // the host keeps max_c4_len <= kTkRegMax
+    const float *row = logits + (int64_t)t * stride;
+    // coalesced: slice j of lane l in warp w is keys 1024w + 128j + 4l .. +3
+    const int w0 = (int)(threadIdx.x >> 5) * 1024 + 4 * (int)(threadIdx.x & 31);
+    const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+    uint32_t keys[kTkRegKpt];
+#pragma unroll
+    for (int j = 0; j < kTkRegKpt / 4; j++) {
+        const int i0 = w0 + 128 * j;
+        if (vec && i0 + 4 <= len) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(row + i0);
+            keys[4 * j] = x.x;
+            keys[4 * j + 1] = x.y;
+            keys[4 * j + 2] = x.z;
+            keys[4 * j + 3] = x.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                keys[4 * j + e] = i0 + e < len ? __float_as_uint(row[i0 + e]) : 0u;
+        }
+    }
+    const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
+    int32_t *op = out_phys + (int64_t)t * kTopK;
+    int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
+    const int K = select_top512_regs<kTkRowThreads, kTkRegKpt>(keys, len, sh, cand_key, cand_idx,
+                                                               kTkRegCap, status,
+                                                               [&](int pos, int s) {
+        const int32_t page = pt_row[s / kC4Page];
+        const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
+        int32_t phys = (int32_t)slot;
+        if (page < 0 || slot >= num_slots) {
+            report(status, CSA_ERR_BOUNDS);
+            phys = -1;
+        }
+        op[pos] = phys;
+        if (orw) orw[pos] = s;
+    });
+    for (int p = K + threadIdx.x; p < kTopK; p += kTkRowThreads) {
+        op[p] = -1;
+        if (orw) orw[p] = -1;
+    }
+}
+
 static int topk_max_chunks(int max_c4_len) {
     return max_c4_len <= 0 ? 1 : (max_c4_len + kTkChunk - 1) / kTkChunk;
 }
@@ -278,6 +378,23 @@ size_t topk_workspace_bytes(int num_q, int max_c4_len) {
 
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
     if (a.num_q == 0) return cudaSuccess;
+    if (a.max_c4_len <= kTkRegMax) {
+        launch_k(topk_reg_kernel, a.num_q, kTkRowThreads, 0, s, a.logits, a.logits_stride,
+                 a.c4_seq_lens, a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.page_table, a.pt_stride,
+                 a.num_slots, a.out_phys, a.out_raw, a.status, a.ratio);
+        return cudaGetLastError();
+    }
+    if (a.max_c4_len <= kTkRowMax) {
+        const size_t smem = kTkRowKeysOffset + (size_t)((a.max_c4_len + 3) & ~3) * 4;
+        static int done_row[64] = {0};
+        cudaError_t e = ensure_max_smem((const void *)topk_row_kernel,
+                                        (int)(kTkRowKeysOffset + (size_t)kTkRowMax * 4), done_row);
+        if (e != cudaSuccess) return e;
+        launch_k(topk_row_kernel, a.num_q, kTkRowThreads, smem, s, a.logits, a.logits_stride,
+                 a.c4_seq_lens, a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.page_table, a.pt_stride,
+                 a.num_slots, a.out_phys, a.out_raw, a.status, a.ratio);
+        return cudaGetLastError();
+    }
     const int mc = topk_max_chunks(a.max_c4_len);
     uint32_t *ck = (uint32_t *)a.workspace;
     int32_t *ci = (int32_t *)((uint8_t *)a.workspace + (size_t)a.num_q * mc * kTopK * 4);

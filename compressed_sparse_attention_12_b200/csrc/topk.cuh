@@ -33,34 +33,37 @@ struct TkSharedT {
 };
 
 // Exclusive scan of one value per thread over the block; returns the prefix
-// and writes the block total to *total.  Uses sh.warp_a.
+// and writes the block total to *total.  Warp totals go through sh.warp_a and
+// are scanned by every warp with shuffles (NT <= 1024).
 template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total,
                                                     TkSharedT<NT> &sh) {
+    constexpr int W = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += n;
     }
     if (lane == 31) sh.warp_a[warp] = incl;
     __syncthreads();
-    uint32_t before = 0, tot = 0;
+    uint32_t x = lane < W ? sh.warp_a[lane] : 0u;
 #pragma unroll
-    for (int w = 0; w < NT / 32; w++) {
-        const uint32_t x = sh.warp_a[w];
-        before += (w < warp) ? x : 0u;
-        tot += x;
+    for (int o = 1; o < W; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += n;
     }
+    const uint32_t upto = __shfl_sync(0xffffffffu, x, warp > 0 ? warp - 1 : 0);
+    *total = __shfl_sync(0xffffffffu, x, W - 1);
     __syncthreads();
-    *total = tot;
-    return before + incl - v;
+    return (warp > 0 ? upto : 0u) + incl - v;
 }
 
 // Block-wide min and max of one value pair per thread (uses sh.warp_a/b).
 template <int NT>
 __device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, TkSharedT<NT> &sh) {
+    constexpr int W = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -72,12 +75,12 @@ __device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, TkShare
         sh.warp_b[warp] = hi;
     }
     __syncthreads();
-    lo = 0xffffffffu;
-    hi = 0u;
+    lo = lane < W ? sh.warp_a[lane] : 0xffffffffu;
+    hi = lane < W ? sh.warp_b[lane] : 0u;
 #pragma unroll
-    for (int w = 0; w < NT / 32; w++) {
-        lo = min(lo, sh.warp_a[w]);
-        hi = max(hi, sh.warp_b[w]);
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
     __syncthreads();
 }
@@ -195,19 +198,61 @@ __device__ int ordered_compact(const uint32_t *keys, int n, uint32_t T, int need
     return (int)(gt_all + min(eq_all, (uint32_t)need_eq));
 }
 
-// One chunk of a row: skeys[0..len) hold the float bits of the chunk's logits
-// (index base + i).  Converts them to keys in place, then writes the chunk's
-// top-512 (or all of it when shorter) in index order to ok/oi and the chunk's
-// (512th-largest key or 0 when it holds fewer, largest key) to *info.
+// Copies row[0..len) (float logits, as bits) into skeys[0..len).  Every
+// thread keeps up to 8 loads of 16 bytes in flight before storing them, so the
+// copy costs a few memory round trips rather than one per vector.
+template <int NT>
+__device__ __forceinline__ void stage_row_keys(uint32_t *skeys, const float *__restrict__ row,
+                                               int len) {
+    if ((reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+        const int n4 = len / 4;
+        const uint4 *src = reinterpret_cast<const uint4 *>(row);
+        uint4 *dst = reinterpret_cast<uint4 *>(skeys);
+        for (int base = 0; base < n4; base += 8 * NT) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int i = base + u * NT + (int)threadIdx.x;
+                if (i < n4) v[u] = src[i];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int i = base + u * NT + (int)threadIdx.x;
+                if (i < n4) dst[i] = v[u];
+            }
+        }
+        for (int i = 4 * n4 + threadIdx.x; i < len; i += NT) skeys[i] = __float_as_uint(row[i]);
+    } else {
+        for (int base = 0; base < len; base += 8 * NT) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int i = base + u * NT + (int)threadIdx.x;
+                if (i < len) v[u] = row[i];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                const int i = base + u * NT + (int)threadIdx.x;
+                if (i < len) skeys[i] = __float_as_uint(v[u]);
+            }
+        }
+    }
+}
+
+// The top-512 of skeys[0..len), which hold the float bits of the logits
+// (index i): converts them to keys in place, finds the threshold and calls
+// emit(pos, i, key) for the selected ones in index order (pos = rank in that
+// order).  Returns min(512, len); *T_out gets the 512th-largest key (0 when
+// len <= 512) and *kmax_out the largest.
 //
 // Lower bound: thread t's keys i = t + j*NT fall into G = ceil(512/NT) groups by
 // j % G.  When all NT*G groups are non-empty the smallest group maximum is at
 // most the 512th-largest key (the NT*G >= 512 group maxima are distinct keys
 // not below it), so the radix digits start from that bound; otherwise the
 // bound is 0.
-template <int NT>
-__device__ void select_chunk(uint32_t *skeys, int len, int base, uint32_t *ok, int32_t *oi,
-                             uint2 *info, TkSharedT<NT> &sh, int32_t *status) {
+template <int NT, typename Emit>
+__device__ __forceinline__ int select_top512(uint32_t *skeys, int len, TkSharedT<NT> &sh, int32_t *status,
+                             uint32_t *T_out, uint32_t *kmax_out, Emit emit) {
     constexpr int G = (kTopK + NT - 1) / NT;
     uint32_t gmax[G];
 #pragma unroll
@@ -235,11 +280,245 @@ __device__ void select_chunk(uint32_t *skeys, int len, int base, uint32_t *ok, i
     uint32_t T = 0;
     int need_eq = len;
     if (len > kTopK) radix_threshold<NT>(skeys, len, K, lbound, kmax, sh, &T, &need_eq);
-    if (threadIdx.x == 0) *info = make_uint2(len > kTopK ? T : 0u, kmax);
-    ordered_compact<NT>(skeys, len, T, need_eq, sh, [&](int pos, int i, uint32_t k) {
+    *T_out = len > kTopK ? T : 0u;
+    *kmax_out = kmax;
+    ordered_compact<NT>(skeys, len, T, need_eq, sh, emit);
+    return K;
+}
+
+// One chunk of a row: skeys[0..len) hold the float bits of the chunk's logits
+// (index base + i).  Writes the chunk's top-512 (or all of it when shorter) in
+// index order to ok/oi and the chunk's (512th-largest key or 0 when it holds
+// fewer, largest key) to *info.
+template <int NT>
+__device__ void select_chunk(uint32_t *skeys, int len, int base, uint32_t *ok, int32_t *oi,
+                             uint2 *info, TkSharedT<NT> &sh, int32_t *status) {
+    uint32_t T, kmax;
+    select_top512<NT>(skeys, len, sh, status, &T, &kmax, [&](int pos, int i, uint32_t k) {
         ok[pos] = k;
         oi[pos] = base + i;
     });
+    if (threadIdx.x == 0) *info = make_uint2(T, kmax);
 }
 
+
+// ---------------------------------------------------------------- register rows
+// A row of at most NT*KPT keys held in registers: thread t owns the contiguous
+// keys [KPT*t, KPT*t + KPT) of the row (those at or past len are absent).
+
+// The K-th largest key T among the present keys >= kmin (as radix_threshold,
+// reading the keys from registers) and how many keys equal to T are taken.
+// present(j) tells which of the thread's keys take part.  With one_pass the
+// result is only the top digit's lower edge: a lower bound of T.
+template <int NT, int KPT, typename Present>
+__device__ __forceinline__ void radix_threshold_regs(const uint32_t (&keys)[KPT], Present present,
+                                                     int K, uint32_t kmin, uint32_t kmax,
+                                                     TkSharedT<NT> &sh, uint32_t *T_out,
+                                                     int *need_eq_out, bool one_pass = false) {
+    const uint32_t range = kmax - kmin;
+    const int B = range == 0 ? 0 : 32 - __clz(range);
+    uint32_t prefix = 0;
+    int remaining = K;
+#pragma unroll 1
+    for (int done = 0; done < B && !(one_pass && done > 0);) {
+        const int width = min(12, B - done);
+        const int shift = B - done - width;
+        const int hi = shift + width;
+        const uint32_t nb = 1u << width;
+        for (uint32_t i = threadIdx.x; i < nb; i += NT) sh.hist[i] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < KPT; j++) {
+            const uint32_t k = keys[j];
+            const uint32_t d = k - kmin;
+            const bool match = present(j) && k >= kmin && (hi >= 32 || ((d ^ prefix) >> hi) == 0);
+            if (match) atomicAdd(&sh.hist[(d >> shift) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+        const int per = (int)((nb + NT - 1) / NT);
+        constexpr int kMaxPer = (kHistBins + NT - 1) / NT;
+        uint32_t c[kMaxPer];
+        uint32_t mine = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxPer; j++) {
+            const int bin = (int)nb - 1 - ((int)threadIdx.x * per + j);
+            c[j] = (j < per && bin >= 0) ? sh.hist[bin] : 0u;
+            mine += c[j];
+        }
+        uint32_t total;
+        const uint32_t excl = block_excl_scan<NT>(mine, &total, sh);
+        if (excl < (uint32_t)remaining && (uint32_t)remaining <= excl + mine) {
+            uint32_t acc = excl;
+            bool found = false;
+#pragma unroll
+            for (int j = 0; j < kMaxPer; j++) {
+                if (!found && j < per && acc + c[j] >= (uint32_t)remaining) {
+                    found = true;
+                    sh.digit = nb - 1 - (threadIdx.x * per + j);
+                    sh.above = acc;
+                }
+                acc += c[j];
+            }
+        }
+        __syncthreads();
+        prefix |= sh.digit << shift;
+        remaining -= (int)sh.above;
+        done += width;
+        __syncthreads();
+    }
+    *T_out = kmin + prefix;
+    *need_eq_out = remaining;
+}
+
+// Index-order ranks for a register row: thread (warp w, lane l) holds the
+// 16-byte slices j = 0..KPT/4-1 at keys 1024w + 128j + 4l .. +3 (NT = 1024,
+// KPT = 32: warp w owns keys [1024w, 1024w + 1024), slices in index order,
+// lanes in index order within a slice).  v[j] are per-thread counts for
+// slice j (two 16-bit fields may be packed: every total stays below 2^16);
+// each becomes the number of counted keys before slice j of this thread in
+// index order over the whole row, in place of v[j]; returns the row total.
+template <int NT, int NS>
+__device__ __forceinline__ uint32_t ordered_starts(uint32_t (&v)[NS], TkSharedT<NT> &sh) {
+    const int lane = threadIdx.x & 31;
+    uint32_t run = 0;
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        uint32_t incl = v[j];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        v[j] = run + incl - v[j];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    uint32_t tot;
+    const uint32_t woff = block_excl_scan<NT>(lane == 31 ? run : 0u, &tot, sh);
+#pragma unroll
+    for (int j = 0; j < NS; j++) v[j] += woff;
+    return tot;
+}
+
+// Top-512 of a register row of len <= NT*KPT keys in the layout of
+// ordered_starts (`keys` hold the float bits on entry; key slot 4j+e is row
+// index 1024w + 128j + 4l + e).  Calls emit(pos, index) for the selected keys
+// with pos their rank in index order; returns min(512, len).
+//
+// Lower bound: the keys fall into groups of 8 (two slices of a thread); when
+// there are at least 512 non-empty groups, any value at most their
+// 512th-largest maximum is at most the row's 512th-largest key (512 groups
+// hold a key >= it).  One radix pass over the group maxima gives such a value
+// L (the lower edge of the bin holding that maximum).  The keys >= L (usually
+// a little over 512) are staged in index order in cand_key/cand_idx (cap
+// entries) and the selection runs over them; rows with more (heavy ties)
+// select from the registers directly.
+template <int NT, int KPT, typename Emit>
+__device__ __forceinline__ int select_top512_regs(uint32_t (&keys)[KPT], int len,
+                                                  TkSharedT<NT> &sh, uint32_t *cand_key,
+                                                  int32_t *cand_idx, int cap, int32_t *status,
+                                                  Emit emit) {
+    static_assert(NT == 1024 && KPT == 32, "layout of ordered_starts");
+    constexpr int NS = KPT / 4, NG = KPT / 8;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto index_of = [&](int kk) { return 1024 * warp + 128 * (kk >> 2) + 4 * lane + (kk & 3); };
+    auto present = [&](int kk) { return index_of(kk) < len; };
+    uint32_t gmax[NG];
+    uint32_t gany = 0;        // bit g: group g holds a key
+#pragma unroll
+    for (int g = 0; g < NG; g++) gmax[g] = 0u;
+#pragma unroll
+    for (int kk = 0; kk < KPT; kk++) {
+        const bool p = present(kk);
+        const uint32_t k = p ? order_key(__uint_as_float(keys[kk]), status) : 0u;
+        keys[kk] = k;
+        if (p) {
+            gmax[kk / 8] = max(gmax[kk / 8], k);
+            gany |= 1u << (kk / 8);
+        }
+    }
+    uint32_t gmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+    for (int g = 0; g < NG; g++)
+        if (gany & (1u << g)) {
+            gmin = min(gmin, gmax[g]);
+            kmax = max(kmax, gmax[g]);
+        }
+    block_minmax<NT>(gmin, kmax, sh);
+    uint32_t ng_total;
+    block_excl_scan<NT>((uint32_t)__popc(gany), &ng_total, sh);
+    const int K = min(kTopK, len);
+    uint32_t L = 0u;
+    if (len > kTopK && ng_total >= (uint32_t)kTopK) {
+        int unused;
+        radix_threshold_regs<NT, NG>(gmax, [&](int g) { return (gany >> g) & 1u; }, kTopK, gmin,
+                                     kmax, sh, &L, &unused, true);
+    }
+    uint32_t T = 0;
+    int need_eq = len;
+    // candidates: the keys >= L, in index order
+    uint32_t at[NS];
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        at[j] = 0;
+#pragma unroll
+        for (int e = 0; e < 4; e++) at[j] += (present(4 * j + e) && keys[4 * j + e] >= L) ? 1u : 0u;
+    }
+    const uint32_t n_cand = ordered_starts<NT, NS>(at, sh);
+    if (n_cand <= (uint32_t)cap) {                 // uniform over the block
+#pragma unroll
+        for (int j = 0; j < NS; j++) {
+            uint32_t a = at[j];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int kk = 4 * j + e;
+                if (present(kk) && keys[kk] >= L) {
+                    cand_key[a] = keys[kk];
+                    cand_idx[a] = index_of(kk);
+                    a++;
+                }
+            }
+        }
+        __syncthreads();
+        if (len > kTopK)
+            radix_threshold<NT>(cand_key, (int)n_cand, K, L, kmax, sh, &T, &need_eq);
+        ordered_compact<NT>(cand_key, (int)n_cand, T, need_eq, sh,
+                            [&](int pos, int i, uint32_t) { emit(pos, cand_idx[i]); });
+        return K;
+    }
+    if (len > kTopK) radix_threshold_regs<NT, KPT>(keys, present, K, L, kmax, sh, &T, &need_eq);
+    // ordered output from the registers: counts of keys above T and equal to
+    // T per slice, packed 16/16 bits (totals <= 32768)
+    uint32_t st[NS];
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        uint32_t gt = 0, eq = 0;
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int kk = 4 * j + e;
+            gt += (present(kk) && keys[kk] > T) ? 1u : 0u;
+            eq += (present(kk) && keys[kk] == T) ? 1u : 0u;
+        }
+        st[j] = gt | (eq << 16);
+    }
+    ordered_starts<NT, NS>(st, sh);
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        uint32_t gt_before = st[j] & 0xFFFFu, eq_seen = st[j] >> 16;
+        uint32_t pos = gt_before + min(eq_seen, (uint32_t)need_eq);
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int kk = 4 * j + e;
+            if (present(kk)) {
+                const uint32_t k = keys[kk];
+                bool take = k > T;
+                if (k == T) {
+                    take = eq_seen < (uint32_t)need_eq;
+                    eq_seen++;
+                }
+                if (take) emit((int)pos++, index_of(kk));
+            }
+        }
+    }
+    return K;
+}
 }  // namespace csa

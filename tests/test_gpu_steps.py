@@ -382,6 +382,19 @@ def _topk_case(case, rng):
         c4, ql = [262144, 100000], [1, 1]
     elif case == "causal":
         c4, ql = [3000, 9000, 700], [5, 5, 4]
+    elif case == "regmax":
+        # the longest rows the one-launch top-k holds in registers (32768 keys)
+        c4, ql = [32768, 5, 600, 2047], [1, 1, 2, 1]
+    elif case == "regmax1":
+        c4, ql = [32769, 31000], [1, 1]
+    elif case == "allequal_reg":
+        c4, ql = [32768, 9000], [1, 1]
+    elif case == "rowmax":
+        # the longest rows the one-launch top-k stages whole (49152 keys), with ties
+        c4, ql = [49152, 30000, 4], [1, 3, 1]
+    elif case == "rowmax1":
+        # one key more: the two-stage path
+        c4, ql = [49153, 2], [1, 1]
     else:
         c4, ql = [50000, 1000], [1, 1]
     c4 = np.asarray(c4, dtype=np.int64)
@@ -404,10 +417,10 @@ def _topk_case(case, rng):
     stride_l = max_c4 + 3
     lg = np.full((nq, stride_l), np.nan, dtype=np.float32)
     for t in range(nq):
-        if case == "ties":
+        if case in ("ties", "rowmax", "rowmax1", "regmax", "regmax1"):
             v = np.round(rng.standard_normal(max_c4) * 3) / 2
             v[rng.integers(0, max_c4, 50)] = -0.0
-        elif case == "allequal":
+        elif case in ("allequal", "allequal_reg"):
             v = np.full(max_c4, 2.5)
         elif case == "long":
             v = rng.standard_t(3, max_c4)
@@ -424,7 +437,8 @@ def _topk_case(case, rng):
                 max_c4=max_c4, nq=nq)
 
 
-@pytest.mark.parametrize("case", ["short", "ties", "long", "causal", "allequal"])
+@pytest.mark.parametrize("case", ["short", "ties", "long", "causal", "allequal", "rowmax",
+                                  "rowmax1", "regmax", "regmax1", "allequal_reg"])
 def test_topk512_bit_exact(case):
     csa = _csa()
     c = _topk_case(case, np.random.default_rng(len(case)))
