@@ -58,7 +58,7 @@ def parse():
     return p.parse_args()
 
 
-INDEXER_SOURCES = ("indexer_tc.cu", "tc.cuh", "common.cuh", "launch.h")
+INDEXER_SOURCES = ("indexer_tc.cu", "tc.cuh", "topk.cuh", "common.cuh", "launch.h")
 
 
 def indexer_source_hash() -> str:
@@ -247,15 +247,33 @@ def time_graph(g, stream, args, l2_flush, inner, world, dev, local, check):
     return t_step, t_in, ck
 
 
-def time_e2e(g, stream, args, l2_flush, data, dst, out, world, dev, num_q):
-    """The step end to end: every step copies its inputs (the fields of `dst`
-    present in `data`) from pinned host memory, replays the graph and copies
-    the output back, all inside the timed region."""
+def pack_inputs(batch, names, dev):
+    """Moves the step inputs batch.<name> into one device buffer (views, 256-byte
+    aligned), so that a step's inputs arrive in one host-to-device copy.
+    Call before capturing the step's graph."""
     import torch
-    h_in = {k: data[k].cpu().pin_memory() for k in dst if data.get(k) is not None
-            and dst[k] is not None}
+    items = [(n, getattr(batch, n)) for n in names if getattr(batch, n, None) is not None]
+    offs, total = [], 0
+    for _, t in items:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    arena = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
+    for (n, t), o in zip(items, offs):
+        nb = t.numel() * t.element_size()
+        view = arena[o:o + nb].view(t.dtype).view(t.shape)
+        view.copy_(t)
+        setattr(batch, n, view)
+    return arena
+
+
+def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q):
+    """The step end to end: every step copies its inputs (the packed arena)
+    from pinned host memory in one copy, replays the graph and copies the
+    output back, all inside the timed region."""
+    import torch
+    h_in = arena.cpu().pin_memory()
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+    h2d = h_in.numel()
     d2h = h_out.numel() * h_out.element_size()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -264,8 +282,7 @@ def time_e2e(g, stream, args, l2_flush, data, dst, out, world, dev, num_q):
         for i in range(args.warmup + args.steps):
             l2_flush()
             e0.record(stream)
-            for k, v in h_in.items():
-                dst[k].copy_(v, non_blocking=True)
+            arena.copy_(h_in, non_blocking=True)
             g.replay()
             h_out.copy_(out, non_blocking=True)
             e1.record(stream)
@@ -395,6 +412,7 @@ def main_hca(args, world, rank, local, dev):
     w = rank_workload(args.workload, rank)
     data = synth.draw_hca(w, dev)
     batch = pipeline.HcaBatch(w, data, device=dev)
+    arena = pack_inputs(batch, ["q", "raw_kv", "gate"], dev)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     flush_read = flush[: 256 << 20].view(torch.int64)
@@ -424,8 +442,7 @@ def main_hca(args, world, rank, local, dev):
                                    batch.check_status)
     e2e = None
     if not args.profile:
-        dst = {"q": batch.q, "raw_kv": batch.raw_kv, "gate": batch.gate}
-        e2e = time_e2e(g, stream, args, l2_flush, data, dst, batch.out, world, dev, w.num_q)
+        e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q)
     split = csa.csa_hca_attention_workspace_size(w.num_q, w.heads, w.window, batch.decode,
                                                  batch.max_hca) > 0
     launches = (1 if batch.max_new >= 128 else 0) + (2 if split else 1)
@@ -479,6 +496,7 @@ def main_dsa(args, world, rank, local, dev):
     w = rank_workload(args.workload, rank)
     data = synth.draw_dsa(w, dev)
     batch = pipeline.DsaBatch(w, data, device=dev)
+    arena = pack_inputs(batch, ["q_idx", "w_head", "q", "new_kv", "new_k"], dev)
     for k in ("kv", "idx_k"):
         data.pop(k)
     torch.cuda.empty_cache()
@@ -520,8 +538,7 @@ def main_dsa(args, world, rank, local, dev):
                                    batch.check_status)
     e2e = None
     if not args.profile:
-        dst = {"q_idx": batch.q_idx, "w": batch.w_head, "q": batch.q}
-        e2e = time_e2e(g, stream, args, l2_flush, data, dst, batch.out, world, dev, w.num_q)
+        e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q)
     split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, 0, batch.decode) > 0
     launches = 2 + 1 + 1 + 2 + (2 if split else 1)
     if rank == 0:
@@ -587,6 +604,8 @@ def main():
     w = rank_workload(args.workload, rank)
     data = synth.draw(w, dev)
     batch = pipeline.CsaBatch(w, data, device=dev)
+    arena = pack_inputs(batch, ["q_idx", "w_head", "q", "raw_kv", "gate", "raw_idx_k", "idx_gate"],
+                        dev)
     if args.profile:
         for k in ("kv_c4", "idx_k", "kv_raw"):
             data.pop(k, None)
@@ -604,13 +623,32 @@ def main():
     ev_i1 = torch.cuda.Event(enable_timing=True, external=True)
     launches_per_step = 0
 
+    # The compressor's two launches (index keys, KV rows) and the query
+    # quantisation depend on nothing else in the step: the compressor runs on
+    # two side streams next to the quantisation, all three joined before the
+    # indexer (which keeps its programmatic-launch link to the attention
+    # chain that follows it on the main stream).
+    side_k = torch.cuda.Stream(device=dev)
+    side_v = torch.cuda.Stream(device=dev)
+    ev_fork = torch.cuda.Event()
+    ev_keys = torch.cuda.Event()
+    ev_rows = torch.cuda.Event()
+
     def step_body(s):
-        batch.compress(s)
+        ev_fork.record(s)
+        side_k.wait_event(ev_fork)
+        side_v.wait_event(ev_fork)
+        batch.compress_index(side_k)
+        ev_keys.record(side_k)
+        batch.compress_kv(side_v)
+        ev_rows.record(side_v)
         batch_q = batch
         from compressed_sparse_attention_12_b200 import csa as c
         c.csa_hadamard_quant(batch_q.q_idx, batch_q.idx_fmt, batch_q.q_codes, batch_q.q_bsc,
                              batch_q.q_scales, w_in=batch_q.w_head, w_out=batch_q.w_fold,
                              status=batch_q.status, stream=s)
+        s.wait_event(ev_keys)
+        s.wait_event(ev_rows)
         if not fused[0]:
             ev_i0.record(s)
             c.csa_indexer_logits(batch_q.q_codes, batch_q.q_bsc, batch_q.w_fold, w.idx_heads,
@@ -675,9 +713,11 @@ def main():
     best = min(candidates, key=lambda c: c[2])
     fused[0], g = best[0], best[1]
     topk_forms = {("fused" if c[0] else "separate"): round(c[2] * 1e3, 2) for c in candidates}
-    # kernels per step: compress (2 when blocks complete), quantise, selecting indexer,
-    # top-k merge, attention (1, +1 combine when split)
-    launches_per_step = (2 if batch.max_new >= 4 else 0) + 1 + 1 + (1 if fused[0] else 2) + \
+    # kernels per step: compress (2 when blocks complete), quantise, indexer (selecting
+    # or plain), top-k (merge, or one or two launches), attention (1, +1 combine when split)
+    # the top-512 is one launch for rows of at most 49152 keys, else two
+    topk_launches = 1 if batch.max_c4 <= 49152 else 2
+    launches_per_step = (2 if batch.max_new >= 4 else 0) + 1 + 1 + (1 if fused[0] else topk_launches) + \
         (2 if csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, w.window, batch.decode) > 0 else 1)
 
     t_step, t_idx, ck = time_graph(g, stream, args, l2_flush, (ev_i0, ev_i1), world, dev, local,
@@ -686,9 +726,7 @@ def main():
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.profile:
-        dst = {"q_idx": batch.q_idx, "w": batch.w_head, "q": batch.q, "raw_kv": batch.raw_kv,
-               "gate": batch.gate, "raw_idx_k": batch.raw_idx_k, "idx_gate": batch.idx_gate}
-        e2e = time_e2e(g, stream, args, l2_flush, data, dst, batch.out, world, dev, w.num_q)
+        e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q)
 
     if rank == 0:
         hbm, src = peaks()

@@ -135,6 +135,11 @@ class CsaBatch:
 
     # ------------------------------------------------------------------ steps
     def compress(self, stream=None):
+        self.compress_kv(stream)
+        self.compress_index(stream)
+
+    def compress_kv(self, stream=None):
+        """The compressor over this step's completed blocks, KV rows."""
         w = self.w
         if self.max_new < 4 or self.raw_kv is None:
             return
@@ -142,6 +147,12 @@ class CsaBatch:
         csa.csa_c4_compress(self.raw_kv, self.gate, self.bias, self.cu_new, self.start_pos,
                             self.max_new, self.page_table, kv_kind, self.c4_cache,
                             status=self.status, stream=stream)
+
+    def compress_index(self, stream=None):
+        """The compressor over this step's completed blocks, index keys."""
+        w = self.w
+        if self.max_new < 4 or self.raw_idx_k is None:
+            return
         ik = {"bf16": csa.CSA_OUT_INDEX_BF16, "fp8": csa.CSA_OUT_INDEX_FP8,
               "fp4": csa.CSA_OUT_INDEX_FP4}[w.idx_fmt]
         csa.csa_c4_compress(self.raw_idx_k, self.idx_gate, self.idx_bias, self.cu_new,
