@@ -83,6 +83,7 @@ _SIGS = {
                                                       _I64, _I32, _I32, _P, _P, _P, _SZ, _P,
                                                       _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
+    "csa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
     "csa_sparse_mqa_decode": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _P,
                                              _I32, _P, _I32, _P, _P, _I32, _F, _P, _P, _P, _SZ,
                                              _P, _P]),
@@ -389,3 +390,13 @@ def csa_hca_attention(q, hca_cache, raw_cache, kv_fmt, page_table, seq_lens, cu_
         _ptr(seq_lens), seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos), int(max_hca_len),
         int(window), float(sm_scale), int(bool(decode)), _ptr(out), _ptr(lse), _ptr(workspace),
         workspace.numel(), _ptr(status), _stream(stream)))
+
+
+CSA_OP_TOPK512, CSA_OP_INDEXER_TOPK512, CSA_OP_SPARSE_MQA, CSA_OP_HCA_ATTENTION = 1, 2, 3, 4
+
+
+def csa_workspace_size(op, bs=0, max_rows=0, max_len=0, heads=0, window=0, decode=True,
+                       idx_dim=0, fmt=0) -> int:
+    """Workspace bytes of one operation by code (include/csa.h)."""
+    return lib().csa_workspace_size(op, bs, max_rows, max_len, heads, window, int(bool(decode)),
+                                    idx_dim, fmt)

@@ -551,3 +551,20 @@ csa_status_t csa_hca_attention(const void *q, int32_t num_q, int32_t heads, cons
                       sm_scale, out, lse, workspace, workspace_bytes, status, stream, decode != 0,
                       CSA_HCA_RATIO, max_hca_len);
 }
+
+size_t csa_workspace_size(int32_t op, int32_t bs, int32_t max_rows, int32_t max_len,
+                          int32_t heads, int32_t window, int32_t decode, int32_t idx_dim,
+                          int32_t fmt) {
+    switch (op) {
+    case CSA_OP_TOPK512:
+        return csa_topk512_workspace_size(max_rows, max_len);
+    case CSA_OP_INDEXER_TOPK512:
+        return csa_indexer_topk512_workspace_size(max_rows, bs, heads, idx_dim, fmt, max_len);
+    case CSA_OP_SPARSE_MQA:
+        return csa_sparse_mqa_workspace_size(max_rows, heads, window, decode);
+    case CSA_OP_HCA_ATTENTION:
+        return csa_hca_attention_workspace_size(max_rows, heads, window, decode, max_len);
+    default:
+        return 0;
+    }
+}

@@ -502,6 +502,25 @@ csa_status_t csa_dsa_topk512_page_transform(const float *logits, int64_t logits_
                                             size_t workspace_bytes, int32_t *status,
                                             void *stream);
 
+/*
+ * csa_workspace_size -- the workspace bytes of one operation, by operation
+ * code (the per-operation *_workspace_size calls, behind one entry point):
+ *   CSA_OP_TOPK512          csa_topk512_page_transform / csa_dsa_...: uses
+ *                           max_rows (= num_q) and max_len
+ *   CSA_OP_INDEXER_TOPK512  csa_indexer_topk512 / csa_indexer_select: uses
+ *                           max_rows, bs, heads (= idx_heads), idx_dim, fmt, max_len
+ *   CSA_OP_SPARSE_MQA       csa_sparse_mqa_decode/_prefill: uses max_rows,
+ *                           heads, window, decode
+ *   CSA_OP_HCA_ATTENTION    csa_hca_attention: uses max_rows, heads, window,
+ *                           decode, max_len (= max_hca_len)
+ * Unused arguments are ignored; an unknown op returns 0.
+ */
+enum { CSA_OP_TOPK512 = 1, CSA_OP_INDEXER_TOPK512 = 2, CSA_OP_SPARSE_MQA = 3,
+       CSA_OP_HCA_ATTENTION = 4 };
+size_t csa_workspace_size(int32_t op, int32_t bs, int32_t max_rows, int32_t max_len,
+                          int32_t heads, int32_t window, int32_t decode, int32_t idx_dim,
+                          int32_t fmt);
+
 #ifdef __cplusplus
 }
 #endif

@@ -123,3 +123,18 @@ def test_product_path_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"(import|from)\s+oracle|liboracle|csa_oracle", txt), f
+
+
+def test_generic_workspace_size_matches_the_per_operation_calls():
+    from compressed_sparse_attention_12_b200 import csa
+    assert csa.csa_workspace_size(csa.CSA_OP_TOPK512, max_rows=32, max_len=32768) == \
+        csa.csa_topk512_workspace_size(32, 32768)
+    assert csa.csa_workspace_size(csa.CSA_OP_INDEXER_TOPK512, bs=32, max_rows=32, max_len=32768,
+                                  heads=64, idx_dim=128, fmt=csa.CSA_FMT_FP8) == \
+        csa.csa_indexer_topk512_workspace_size(32, 32, 64, 128, csa.CSA_FMT_FP8, 32768)
+    assert csa.csa_workspace_size(csa.CSA_OP_SPARSE_MQA, max_rows=32, heads=64, window=128,
+                                  decode=True) == csa.csa_sparse_mqa_workspace_size(32, 64, 128, True)
+    assert csa.csa_workspace_size(csa.CSA_OP_HCA_ATTENTION, max_rows=32, heads=64, window=128,
+                                  decode=True, max_len=1024) == \
+        csa.csa_hca_attention_workspace_size(32, 64, 128, True, 1024)
+    assert csa.csa_workspace_size(99) == 0
