@@ -66,6 +66,12 @@ struct TcSelect {
 };
 
 constexpr int kKsRing = 8;     // key-scale tiles in flight per epilogue group
+// FP4 block scales of Di = 64 keys (4 bytes a key): copied as 16-byte chunks
+// into a staging ring and moved into the tensor-core scale layout kSfLag
+// tiles later (kSfLag < stages); Di = 128 keys gather theirs 4 bytes at a
+// time straight into the layout (measured faster there)
+constexpr int kSfLag = 4;
+constexpr int kSfSlots = kSfLag + 1;
 
 template <int FMT, int RB>
 __global__ void __launch_bounds__(kTcThreads, 2)
@@ -78,11 +84,13 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     constexpr bool kFp4 = FMT == CSA_FMT_FP4;
+    constexpr bool kSfStaged = kFp4 && RB == 32;
     uint8_t *stage_buf = base;
     uint8_t *q_buf = stage_buf + p.stages * G::kStageBytes;
     uint8_t *sfa_buf = q_buf + ((p.n * RB + 1023) & ~1023);            // [stages][ksteps][512]
     uint8_t *sfb_buf = sfa_buf + (kFp4 ? p.stages * G::kKSteps * 512 : 0);  // [ksteps][512]
-    float *w_s = reinterpret_cast<float *>(sfb_buf + (kFp4 ? G::kKSteps * 512 : 0));
+    uint8_t *sf_stage = sfb_buf + (kFp4 ? G::kKSteps * 512 : 0);    // [kSfSlots][16 * RB]
+    float *w_s = reinterpret_cast<float *>(sf_stage + (kSfStaged ? kSfSlots * 16 * RB : 0));
     int *nv_s = reinterpret_cast<int *>(w_s + 256);
     uint64_t *bars = reinterpret_cast<uint64_t *>(nv_s + 16);
     uint64_t *full = bars, *empty = bars + p.stages, *tfull = bars + 2 * p.stages;
@@ -136,9 +144,10 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     if (warp == 0) tc::tmem_alloc(tc::saddr(tmem_slot), (uint32_t)p.tmem_cols);
     if (threadIdx.x == 32) {
         for (int s = 0; s < p.stages; s++) {
-            // one arrival (the producer's expect_tx); FP4 block-scale copies
-            // add and complete their own pending arrivals
-            tc::mbar_init(tc::saddr(&full[s]), 1);
+            // the producer's expect_tx arrival, and with staged block scales a
+            // second one once they are in place (gathered ones add and
+            // complete their own pending arrivals)
+            tc::mbar_init(tc::saddr(&full[s]), kSfStaged ? 2 : 1);
             tc::mbar_init(tc::saddr(&empty[s]), 1);
         }
         for (int i = 0; i < p.nacc; i++) {
@@ -199,6 +208,37 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     if (warp == 0) {
         // ---------------- TMA producer (lane 0) and FP4 block-scale gather (all lanes)
         int issued = 0;
+        // FP4: moves tile j's staged block scales into the scale layout of 128
+        // rows (row m = m0 + 32*m1 keeps its four scales of K-step ks at byte
+        // ks*512 + m0*16 + m1*4) of stage j % stages, then releases the
+        // stage's second arrival.  Each lane moves the chunks it copied.
+        auto sf_place = [&](int j) {
+            if constexpr (kSfStaged) {
+                constexpr int nsf = RB / 8;
+                constexpr int kChunksPerPage = 4 * nsf;
+                constexpr int KS = G::kKSteps;            // = nsf / 4
+                const uint8_t *stg = sf_stage + (j % kSfSlots) * 16 * RB;
+                uint8_t *dst = sfa_buf + (j % p.stages) * KS * 512;
+#pragma unroll
+                for (int q = lane; q < 2 * kChunksPerPage; q += 32) {
+                    const int half = q / kChunksPerPage, c = q % kChunksPerPage;
+                    const int32_t page = pg_s[j * 2 + half];
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (page >= 0 && page < p.num_pages)
+                        v = *reinterpret_cast<const uint4 *>(stg + q * 16);
+                    const int m0 = half * 64 + c * (16 / nsf);
+#pragma unroll
+                    for (int w = 0; w < 4; w++) {
+                        const int m = m0 + w / KS, ks = w % KS;
+                        const uint32_t x = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+                        *reinterpret_cast<uint32_t *>(dst + ks * 512 + (m & 31) * 16 + (m >> 5) * 4) = x;
+                    }
+                }
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(tc::saddr(&full[j % p.stages]));
+            }
+        };
         for (int i = 0; i < my_tiles; i++) {
             const int s = i % p.stages;
             const uint32_t ph = (uint32_t)((i / p.stages) & 1);
@@ -212,8 +252,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            const int tile = tile_begin + i;
-            if constexpr (kFp4) {
+            if constexpr (kFp4 && !kSfStaged) {
                 // key m = lane + 32*m1 of the tile: its block scales of K-step ks go
                 // to byte (s*ksteps + ks)*512 + lane*16 + m1*4 by 4-byte cp.async;
                 // each lane's copies hold the stage's phase open until they land
@@ -222,7 +261,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
                 for (int m1 = 0; m1 < 4; m1++) {
                     const int m = lane + 32 * m1;
-                    const int sk = tile * kTcTile + m;
+                    const int sk = (tile_begin + i) * kTcTile + m;
                     int64_t slot = -1;
                     if (sk < nv_max) {
                         const int32_t page = pg_s[i * 2 + (m >> 6)];
@@ -240,6 +279,22 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 tc::cp_async_mbar_arrive(tc::saddr(&full[s]));
                 __syncwarp();
             }
+            if constexpr (kSfStaged) {
+                // the tile's block scales: 16-byte chunks of each page's
+                // contiguous 64 x Di/16 bytes into staging slot i % kSfSlots
+                constexpr int nsf = RB / 8;               // Di/16 block scales per key
+                constexpr int kChunksPerPage = 4 * nsf;   // 16-byte chunks per page
+                uint8_t *stg = sf_stage + (i % kSfSlots) * 16 * RB;
+#pragma unroll
+                for (int q = lane; q < 2 * kChunksPerPage; q += 32) {
+                    const int32_t page = pg_s[i * 2 + q / kChunksPerPage];
+                    if (page >= 0 && page < p.num_pages)
+                        tc::cp_async16(tc::saddr(stg + q * 16),
+                                       a.k_block_scales + (int64_t)page * kC4Page * nsf +
+                                           (q % kChunksPerPage) * 16);
+                }
+                tc::cp_async_commit();
+            }
             if (lane == 0) {
                 tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
 #pragma unroll
@@ -255,6 +310,16 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 }
             }
             issued++;
+            if constexpr (kSfStaged) {
+                if (i >= kSfLag) {
+                    tc::cp_async_wait<kSfLag>();
+                    sf_place(i - kSfLag);
+                }
+            }
+        }
+        if constexpr (kSfStaged) {
+            tc::cp_async_wait<0>();
+            for (int j = max(0, issued - kSfLag); j < issued; j++) sf_place(j);
         }
         // before leaving, every load issued must have landed
         if (lane == 0)
@@ -477,16 +542,18 @@ static bool make_key_map(CUtensorMap *m, const void *codes, int64_t num_slots, i
 static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p) {
     const size_t ks = rb / 32;
     return 1024 + (size_t)p.stages * kTcTile * rb + (((size_t)p.n * rb + 1023) & ~(size_t)1023) +
-           (fp4 ? (p.stages + 1) * ks * 512 : 0) + 256 * 4 + 16 * 4 + (2 * p.stages + 2 * p.nacc + 1) * 8 + 32 +
+           (fp4 ? (p.stages + 1) * ks * 512 + (rb == 32 ? (size_t)kSfSlots * 16 * rb : 0) : 0) +
+           256 * 4 + 16 * 4 +
+           (2 * p.stages + 2 * p.nacc + 1) * 8 + 32 +
            (size_t)2 * p.tiles_per_cta * 4 + 16 + (size_t)2 * kKsRing * kTcTile * 4;
 }
 
 bool indexer_tc_supported(const IndexerArgs &a) {
     const bool fmt_ok = (a.dim == 64 || a.dim == 128) &&
                         (a.fmt == CSA_FMT_FP8 || a.fmt == CSA_FMT_BF16 || a.fmt == CSA_FMT_FP4);
-    // FP4 block scales are gathered four at a time (32-bit loads)
+    // FP4 key block scales are copied in 16-byte chunks, query ones four at a time
     const bool sf_ok = a.fmt != CSA_FMT_FP4 ||
-                       ((reinterpret_cast<uintptr_t>(a.k_block_scales) % 4) == 0 &&
+                       ((reinterpret_cast<uintptr_t>(a.k_block_scales) % 16) == 0 &&
                         (reinterpret_cast<uintptr_t>(a.q_block_scales) % 4) == 0);
     return fmt_ok && sf_ok && a.heads <= 128 && (a.num_slots % kC4Page) == 0 &&
            a.num_slots >= kC4Page && (reinterpret_cast<uintptr_t>(a.k_codes) % 16) == 0 &&
