@@ -84,6 +84,7 @@ _SIGS = {
                                                       _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
     "csa_workspace_size": (_SZ, [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32]),
+    "csa_selftest_wait_timeout": (ctypes.c_int, [_P, _P, _P]),
     "csa_sparse_mqa_decode": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _I32, _I64, _I64, _P, _P,
                                              _I32, _P, _I32, _P, _P, _I32, _F, _P, _P, _P, _SZ,
                                              _P, _P]),
@@ -400,3 +401,9 @@ def csa_workspace_size(op, bs=0, max_rows=0, max_len=0, heads=0, window=0, decod
     """Workspace bytes of one operation by code (include/csa.h)."""
     return lib().csa_workspace_size(op, bs, max_rows, max_len, heads, window, int(bool(decode)),
                                     idx_dim, fmt)
+
+
+def csa_selftest_wait_timeout(status, waited_ns=None, stream=None):
+    """One bounded device wait that runs out (include/csa.h)."""
+    _check("csa_selftest_wait_timeout", lib().csa_selftest_wait_timeout(
+        _ptr(status), _ptr(waited_ns), _stream(stream)))

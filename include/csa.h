@@ -521,6 +521,16 @@ size_t csa_workspace_size(int32_t op, int32_t bs, int32_t max_rows, int32_t max_
                           int32_t heads, int32_t window, int32_t decode, int32_t idx_dim,
                           int32_t fmt);
 
+/*
+ * csa_selftest_wait_timeout -- checks the library's bounded device waits: one
+ * CTA waits on an mbarrier phase that nothing completes; the wait gives up
+ * after the library's limit (1 s) and CSA_ERR_TIMEOUT is recorded in *status
+ * (device int32, caller-owned; an earlier non-zero code is kept).  waited_ns
+ * (nullable device int32) receives the time the wait took.  Asynchronous on
+ * `stream`; the CUDA context stays usable.
+ */
+csa_status_t csa_selftest_wait_timeout(int32_t *status, int32_t *waited_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
