@@ -138,3 +138,53 @@ def test_generic_workspace_size_matches_the_per_operation_calls():
                                   decode=True, max_len=1024) == \
         csa.csa_hca_attention_workspace_size(32, 64, 128, True, 1024)
     assert csa.csa_workspace_size(99) == 0
+
+
+def test_host_validation_of_the_next_rows(L):
+    """HCA, fused RoPE, DSA, unrotated quantisation and the wait self-test
+    reject bad arguments on the host, before any launch."""
+    from compressed_sparse_attention_12_b200 import csa
+    # HCA compressor: KV output kinds only, dim 576
+    r = L.csa_hca_compress(_p(), _p(), _p(), 576, 1, _p(), 256, _p(), 256, _p(), 4,
+                           csa.CSA_OUT_INDEX_FP8, _p(), 64, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    r = L.csa_hca_compress(_p(), _p(), _p(), 512, 1, _p(), 256, _p(), 256, _p(), 4,
+                           csa.CSA_OUT_KV_FP8, _p(), 64, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    # HCA attention: negative or too many rows
+    args = [_p(), 1, 64, _p(), _p(), csa.CSA_FMT_FP8, 64, 256, _p(), 4, _p(), 1, _p(), None, -1,
+            128, 0.1, 1, _p(), None, _p(), 1 << 30, None, None]
+    assert L.csa_hca_attention(*args) == csa.CSA_ERR_INVALID
+    args[14] = csa.HCA_MAX_ROWS
+    assert L.csa_hca_attention(*args) == csa.CSA_ERR_UNSUPPORTED
+    # fused RoPE: odd or oversized rope_dim, no positions, rows_per_pos < 1, misaligned table
+    def rope(rope_dim=64, positions=_p(), rows_per_pos=1, freqs=_p()):
+        return L.csa_rope_hadamard_quant(_p(), csa.CSA_FMT_BF16, 4, 128, freqs, rope_dim, 1024,
+                                         positions, rows_per_pos, csa.CSA_FMT_FP8, None, 0, _p(),
+                                         None, _p(), None, None, None, None)
+    assert rope(rope_dim=63) == csa.CSA_ERR_INVALID
+    assert rope(rope_dim=130) == csa.CSA_ERR_INVALID
+    assert rope(positions=None) == csa.CSA_ERR_INVALID
+    assert rope(rows_per_pos=0) == csa.CSA_ERR_INVALID
+    assert rope(freqs=ctypes.c_void_p(256 + 4)) == csa.CSA_ERR_INVALID
+    r = L.csa_c4_compress_index_rope(_p(), _p(), _p(), 576, 1, _p(), 8, _p(), 8, _p(), 4,
+                                     csa.CSA_OUT_KV_FP8, _p(), 64, 1024, _p(), None, None, 64,
+                                     None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    # unrotated quantisation and the DSA calls share the C4 checks
+    r = L.csa_index_quant(_p(), csa.CSA_FMT_BF16, 4, 96, csa.CSA_FMT_FP8, None, 0, _p(), None,
+                          _p(), None, None, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    r = L.csa_dsa_indexer_logits(_p(), None, _p(), 1, 64, 96, csa.CSA_FMT_FP8, _p(), None, _p(),
+                                 64, _p(), 1, _p(), 1, _p(), None, 64, _p(), 64, None, None)
+    assert r == csa.CSA_ERR_UNSUPPORTED
+    r = L.csa_dsa_topk512_page_transform(_p(), 64, 1, _p(), 1, _p(), None, _p(), 4, 256, 32, 64,
+                                         _p(), None, _p(), 1 << 20, None, None)
+    assert r == csa.CSA_ERR_INVALID
+    # fused indexer + top-512 with a workspace below its size
+    r = L.csa_indexer_topk512(_p(), None, _p(), 1, 64, 128, csa.CSA_FMT_FP8, _p(), None, _p(), 64,
+                              _p(), 1, _p(), 1, _p(), None, 64, 64, _p(), 64, _p(), None, _p(),
+                              16, None, None)
+    assert r == csa.CSA_ERR_WORKSPACE
+    # the wait self-test needs a status word
+    assert L.csa_selftest_wait_timeout(None, None, None) == csa.CSA_ERR_INVALID

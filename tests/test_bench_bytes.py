@@ -1,0 +1,45 @@
+"""The algorithmic byte counts behind the benchmark's roofline figures,
+against the closed forms of the workloads they describe."""
+import os
+import sys
+
+sys.path.insert(0, os.path.join(os.path.dirname(__file__), ".."))
+
+import bench  # noqa: E402
+from compressed_sparse_attention_12_b200 import synth  # noqa: E402
+
+
+def test_indexer_bytes_decode_128k():
+    # 32 rows x 32768 visible keys of (128 FP8 codes + 4 B scale) + a 4 B logit
+    # each, plus 64 query heads of (128 + 4) B codes and a 4 B weight per row
+    w = synth.workload("decode_128k")
+    assert bench.indexer_alg_bytes(w) == 32 * 32768 * (132 + 4) + 32 * 64 * (132 + 4)
+
+
+def test_indexer_bytes_decode_1m_fp4():
+    # FP4 8x64: a key is 32 code bytes + 4 block scales + a 4 B row scale
+    w = synth.workload("decode_1m")
+    assert bench.index_bytes_per_key(w) == 40
+    assert bench.indexer_alg_bytes(w) == 8 * 262144 * (40 + 4) + 8 * 8 * (40 + 4)
+
+
+def test_indexer_bytes_dsa_counts_every_raw_key():
+    # ratio 1: query at position L-1 sees L keys
+    w = synth.workload("dsa_128k")
+    assert bench.indexer_alg_bytes(w, 1) == 32 * 131072 * (132 + 4) + 32 * 64 * (132 + 4)
+
+
+def test_step_bytes_decode_128k():
+    # keys once, q codes + weights, 512 selected + 128 window rows of 656 B,
+    # attention q (576 bf16) and out (512 bf16) per head
+    w = synth.workload("decode_128k")
+    want = (32 * 32768 * 132 + 32 * 64 * (132 + 4) + 32 * 640 * 656 +
+            32 * 64 * (576 + 512) * 2)
+    assert bench.step_alg_bytes(w) == want
+
+
+def test_hca_attention_bytes():
+    # every HCA row (131072/128 = 1024) and 128 window rows per query, plus q,
+    # out and lse per head
+    w = synth.workload("hca_128k")
+    assert bench.hca_attn_alg_bytes(w) == 32 * (1024 + 128) * 656 + 32 * 64 * (1152 + 1024 + 4)
