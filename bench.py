@@ -111,26 +111,77 @@ def index_bytes_per_key(w):
     return {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}[w.idx_fmt]
 
 
-def indexer_alg_bytes(w, ratio=4):
-    """Bytes one indexer launch must move: every visible key (codes + scales)
-    once per query row, the query codes and weights, and the logits written
-    (ratio raw tokens per key: 4 for C4, 1 for DSA)."""
+def _visible(w, ratio):
+    """Visible keys of every query row, and of every request (those of its
+    last query, at position L-1: all floor(L/ratio) keys)."""
     nv = np.concatenate([np.minimum(w.seq_lens[b] // ratio, (np.arange(L - q, L) + 1) // ratio)
                          for b, (L, q) in enumerate(zip(w.seq_lens, w.q_lens))])
+    return nv, w.seq_lens // ratio
+
+
+def indexer_alg_bytes(w, ratio=4):
+    """Bytes one indexer launch must move: every request's visible keys (codes
+    + scales) once, the query codes and weights, and the logits written
+    (ratio raw tokens per key: 4 for C4, 1 for DSA)."""
+    nv, per_req = _visible(w, ratio)
     qb = {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}
-    return int(nv.sum() * (index_bytes_per_key(w) + 4) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4))
+    return int(per_req.sum() * index_bytes_per_key(w) + nv.sum() * 4 +
+               w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4))
+
+
+def indexer_flops(w, ratio=4):
+    """Multiply-adds x 2 of one indexer launch: every visible (query row, key)
+    pair takes a dot product of idx_dim per index head."""
+    nv, _ = _visible(w, ratio)
+    return int(nv.sum()) * w.idx_heads * w.idx_dim * 2
+
+
+def tensor_peak(fmt):
+    """Dense tensor peak (TFLOP/s) for the indexer's operand type: the measured
+    bf16 figure for a kernel timed inside a long step (sustained) times the
+    nominal ratio of the type to bf16 (FP8 2x, FP4 4x)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        base, src = float(d["bf16_tflops_sustained"]), "measured bf16 sustained"
+    except Exception:
+        base, src = 1400.0, "fallback bf16 sustained"
+    ratio = {"bf16": 1, "fp8": 2, "fp4": 4}[fmt]
+    return base * ratio, src + (f" x {ratio} (nominal {fmt}/bf16)" if ratio > 1 else "")
+
+
+def indexer_roofline(w, t_idx, hbm, hbm_src, traffic, ratio=4):
+    """The indexer's roofline line: HBM-bound (algorithmic bytes over time
+    against the measured copy bandwidth) or, when its arithmetic intensity is
+    above the ridge point (prefill: many queries per request share each key),
+    tensor-bound (flops over time against the dense peak of its type)."""
+    ib = indexer_alg_bytes(w, ratio)
+    fl = indexer_flops(w, ratio)
+    tpk, tsrc = tensor_peak(w.idx_fmt)
+    ridge = tpk * 1e12 / (hbm * 1e9)
+    line = {"alg_bytes_per_launch": ib, "flops_per_launch": fl, "launch_ms": t_idx * 1e3,
+            "intensity_flop_per_byte": fl / ib, "ridge_flop_per_byte": ridge}
+    if fl / ib > ridge:
+        ach = fl / t_idx / 1e12
+        line.update({"bound": "tensor", "achieved": ach, "peak": tpk, "peak_source": tsrc,
+                     "unit": "TFLOP/s", "frac": ach / tpk, "traffic": traffic})
+    else:
+        ach = ib / t_idx / 1e9
+        line.update({"bound": "hbm", "achieved": ach, "peak": hbm, "peak_source": hbm_src,
+                     "unit": "GB/s", "frac": ach / hbm, "traffic": traffic})
+    return line
 
 
 def step_alg_bytes(w):
-    """Algorithmic bytes of one whole step (keys, q, selected + window rows,
-    attention q/out; logits excluded as an implementation detail)."""
+    """Algorithmic bytes of one whole step: every request's keys once, the
+    index queries and weights, the selected + window rows of every query and
+    the attention q/out (logits excluded as an implementation detail)."""
     row = 656 if w.kv_fmt == "fp8" else 1152
-    nv = np.concatenate([np.minimum(w.c4_lens[b], (np.arange(L - q, L) + 1) // 4)
-                         for b, (L, q) in enumerate(zip(w.seq_lens, w.q_lens))])
+    nv, per_req = _visible(w, 4)
     pos = np.concatenate([np.arange(L - q, L) for L, q in zip(w.seq_lens, w.q_lens)])
     rows = np.minimum(nv, 512) + np.minimum(w.window, pos + 1)
     qb = {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}
-    return int(nv.sum() * index_bytes_per_key(w) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4)
+    return int(per_req.sum() * index_bytes_per_key(w) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4)
                + rows.sum() * row + w.num_q * w.heads * (576 + 512) * 2)
 
 
@@ -604,9 +655,7 @@ def main_dsa(args, world, rank, local, dev):
     launches = 2 + 1 + 1 + 2 + (2 if split else 1)
     if rank == 0:
         hbm, src = peaks()
-        ib = indexer_alg_bytes(w, 1)
         sb = dsa_step_alg_bytes(w)
-        achieved = ib / t_idx / 1e9
         cfg = {"workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
                "keys_per_request": int(w.seq_lens.max()), "query_tokens": w.num_q,
                "indexer": f"{w.idx_fmt} {w.idx_heads}x{w.idx_dim} (no rotation)",
@@ -619,11 +668,9 @@ def main_dsa(args, world, rank, local, dev):
                "data": "synthetic", "config": cfg,
                "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
                        "frac_of_peak": sb / t_step / 1e9 / hbm},
-               "roofline": {"kernel": "dsa indexer_logits (indexer_tc_kernel, one key per token)",
-                            "bound": "hbm", "achieved": achieved, "peak": hbm,
-                            "peak_source": src, "unit": "GB/s", "frac": achieved / hbm,
-                            "traffic": None, "alg_bytes_per_launch": ib,
-                            "launch_ms": t_idx * 1e3},
+               "roofline": dict({"kernel": "dsa indexer_logits (indexer_tc_kernel, one key per "
+                                           "token)"},
+                                **indexer_roofline(w, t_idx, hbm, src, None, ratio=1)),
                "e2e": e2e, "gpu_launches": launches * args.steps, "clocks": ck}
         print(json.dumps(out), flush=True)
     del g
@@ -792,9 +839,7 @@ def main():
 
     if rank == 0:
         hbm, src = peaks()
-        ib = indexer_alg_bytes(w)
         traffic = profiled_traffic(w)
-        achieved = ib / t_idx / 1e9
         sb = step_alg_bytes(w)
         out = {"metric": METRIC, "value": world * w.num_q / t_step, "unit": UNIT, "n_gpus": world,
                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
@@ -805,12 +850,10 @@ def main():
                               indexer_topk_probe_us=topk_forms),
                "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
                        "frac_of_8tbs": sb / t_step / 8e12, "frac_of_peak": sb / t_step / 1e9 / hbm},
-               "roofline": {"kernel": ("indexer_select (indexer_tc_kernel: logits + chunk top-512)"
-                                       if fused[0] else "indexer_logits (indexer_tc_kernel)"),
-                            "bound": "hbm", "achieved": achieved,
-                            "peak": hbm, "peak_source": src, "unit": "GB/s",
-                            "frac": achieved / hbm, "traffic": traffic,
-                            "alg_bytes_per_launch": ib, "launch_ms": t_idx * 1e3},
+               "roofline": dict({"kernel": ("indexer_select (indexer_tc_kernel: logits + chunk "
+                                            "top-512)" if fused[0] else
+                                            "indexer_logits (indexer_tc_kernel)")},
+                                **indexer_roofline(w, t_idx, hbm, src, traffic)),
                "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": ck}
         if not args.no_cpu_baseline and not args.profile and world == 1:
             out["cpu_baseline"] = cpu_baseline(w, data, batch.pt_host)

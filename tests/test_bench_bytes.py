@@ -43,3 +43,26 @@ def test_hca_attention_bytes():
     # out and lse per head
     w = synth.workload("hca_128k")
     assert bench.hca_attn_alg_bytes(w) == 32 * (1024 + 128) * 656 + 32 * 64 * (1152 + 1024 + 4)
+
+
+def test_prefill_counts_each_key_once_and_is_tensor_bound():
+    # 4096 queries of one request share its 66560 keys: bytes count them once,
+    # flops count every (query, key) pair; the intensity is far above the ridge
+    w = synth.workload("prefill")
+    L = 262144 + 4096
+    nv = sum(min(L // 4, (p + 1) // 4) for p in range(L - 4096, L))
+    assert bench.indexer_flops(w) == nv * 64 * 128 * 2
+    assert bench.indexer_alg_bytes(w) == (L // 4) * 132 + nv * 4 + 4096 * 64 * 136
+    line = bench.indexer_roofline(w, 7.8e-3, 6551.4, "measured", None)
+    assert line["bound"] == "tensor" and line["unit"] == "TFLOP/s"
+    assert abs(line["achieved"] - nv * 64 * 128 * 2 / 7.8e-3 / 1e12) < 1e-6
+    assert line["frac"] == line["achieved"] / line["peak"]
+
+
+def test_decode_roofline_is_hbm_bound():
+    w = synth.workload("decode_128k")
+    line = bench.indexer_roofline(w, 43.1e-6, 6551.4, "measured", 144419328)
+    assert line["bound"] == "hbm" and line["unit"] == "GB/s"
+    assert line["alg_bytes_per_launch"] == 142884864
+    assert line["traffic"] == 144419328
+    assert line["intensity_flop_per_byte"] < line["ridge_flop_per_byte"]
