@@ -215,6 +215,8 @@ csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scal
  *   raw_indices[t][i]            = s            (nullable output)
  *   c4_page_size   must be 64 (= 256/4)
  *   workspace      >= csa_topk512_workspace_size(num_q, max_c4_len) bytes
+ *                  (always checked; written only when max_c4_len > 49152, the
+ *                  rows shorter than that being selected in one launch)
  */
 size_t csa_topk512_workspace_size(int32_t num_q, int32_t max_c4_len);
 csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stride,
