@@ -343,6 +343,12 @@ csa_status_t csa_topk512_merge(int32_t num_q, int32_t idx_heads, int32_t idx_dim
  * The two entry points compute the same function; _decode splits each
  * query's rows across CTAs (few queries, many rows each), _prefill gives each
  * query its own CTA (many queries).
+ * Ordering: like every kernel of the library this one is launched with
+ * programmatic dependent launch; with FP8 rows it reads q, cu_q, q_pos and
+ * seq_lens before waiting for the kernel enqueued just before it, so these
+ * must not be written by a kernel that lets its successor start early and
+ * runs immediately before this call (the library's own kernels never write
+ * them; data written by a copy or by earlier work is safe).
  */
 size_t csa_sparse_mqa_workspace_size(int32_t num_q, int32_t heads, int32_t window,
                                      int32_t decode);
