@@ -475,10 +475,11 @@ def _t2n(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def step(w, data, page_table, requests=None, sm_scale=None):
+def step(w, data, page_table, requests=None, sm_scale=None, queries=None):
     """One decode/prefill step of C4 compressed sparse attention, composed from
     the steps above in the pages' order ([T] §1-§4; [H] "Compressed Sparse
-    Attention（CSA）"), for the requests listed (default: all).
+    Attention（CSA）"), for the requests listed (default: all) and, within
+    them, the query rows listed in `queries` (default: all).
 
     w is the workload's shape record and data its drawn inputs (the same
     buffers the GPU path reads).  The oracle keeps its own copies of the
@@ -518,15 +519,19 @@ def step(w, data, page_table, requests=None, sm_scale=None):
         raw_rows = dict(zip(raw_pos[sel].tolist(),
                             kv_decode_rows(kv_encode_rows(_t2n(data["kv_raw"][sel]), fp8_kv),
                                            fp8_kv)))
-        qs = slice(q_off[b], q_off[b + 1])
-        qi = index_quantise(_t2n(data["q_idx"][qs]), w.idx_fmt)["deq"]
-        ww = _t2n(data["w"][qs])
-        pos = q_pos[qs]
+        rows_t = [t for t in range(int(q_off[b]), int(q_off[b + 1]))
+                  if queries is None or t in queries]
+        if not rows_t:
+            continue
+        qsel = np.asarray(rows_t, dtype=np.int64)
+        qi = index_quantise(_t2n(data["q_idx"][qsel]), w.idx_fmt)["deq"]
+        ww = _t2n(data["w"][qsel])
+        pos = q_pos[qsel]
         nv = np.array([min(n_c4, n_visible(int(p))) for p in pos], dtype=np.int64)
         lg = indexer_logits(qi, ww, k_deq, nv) if n_c4 else np.zeros((len(pos), 0))
-        qa = _t2n(data["q"][qs])
+        qa = _t2n(data["q"][qsel])
         for j, p in enumerate(pos):
-            t = int(q_off[b] + j)
+            t = rows_t[j]
             phys, logical = topk_transform(lg[j], int(nv[j]), page_table[b], 1 << 40, k=w.topk)
             chosen = logical[logical >= 0]
             win = window_positions(int(p), w.window)

@@ -298,3 +298,21 @@ def test_kv_row_codec(orc):
     b16 = orc.kv_encode_rows(x, fp8=False)
     d16 = orc.kv_decode_rows(b16, fp8=False)
     assert np.array_equal(d16, torch.tensor(x).float().bfloat16().double().numpy())
+
+
+def test_step_query_filter_matches_the_full_step(orc):
+    # computing only some query rows of a request gives those rows unchanged
+    import os
+    import sys
+    sys.path.insert(0, os.path.join(os.path.dirname(__file__), ".."))
+    from compressed_sparse_attention_12_b200 import synth
+    w = synth.workload("prefill", 1 / 64)
+    d = synth.draw(w, "cpu")
+    pt = synth.page_table(w)
+    full = orc.step(w, d, pt)
+    part = orc.step(w, d, pt, queries={0, 5, w.num_q - 1})
+    assert sorted(part) == [0, 5, w.num_q - 1]
+    for t, r in part.items():
+        assert np.array_equal(r["logical"], full[t]["logical"])
+        assert np.array_equal(r["logits"], full[t]["logits"])
+        assert np.array_equal(r["out"], full[t]["out"])
