@@ -93,3 +93,15 @@ def test_dsa_step_selects_everything_when_short():
             d["q"][t].double()[None, None], k[None, None], k[None, None, :, :512],
             scale=1 / 24)[0, 0].numpy()
         np.testing.assert_allclose(r[t]["out"], want, rtol=1e-10, atol=1e-10)
+
+
+def test_rope_golden():
+    import json
+    path = os.path.join(os.path.dirname(__file__), "golden", "rope_example.json")
+    with open(path) as f:
+        gold = json.load(f)
+    f = np.array(gold["freqs"], dtype=np.float64)
+    x = np.array([gold["x"]], dtype=np.float64)
+    for case in gold["cases"]:
+        y = orc.rope(x, f, gold["rope_dim"], [case["pos"]])
+        np.testing.assert_allclose(y[0], case["y"], rtol=0, atol=1e-15)

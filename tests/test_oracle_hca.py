@@ -119,3 +119,18 @@ def test_hca_step_flat_gate_block_is_the_mean_and_rows_follow_visibility():
             torch.tensor(q[j])[None, None], k[None, None], k[None, None, :, :512],
             scale=1 / 24)[0, 0].numpy()
         np.testing.assert_allclose(ref[j]["out"], want, rtol=1e-10, atol=1e-10)
+
+
+def test_hca_pool_golden():
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "hca_pool_example.json")
+    with open(path) as f:
+        gold = json.load(f)
+    for case in gold["cases"]:
+        x = np.array(case["x"], dtype=np.float64)[:, None]
+        g = np.array(case["gate"], dtype=np.float64)[:, None]
+        b = np.array(case["bias"], dtype=np.float64)[:, None]
+        y = orc.hca_compress(x, g, b)
+        assert y.shape == (len(case["x"]) // 128, 1)
+        np.testing.assert_allclose(y[:, 0], case["y"], rtol=1e-13)
