@@ -163,5 +163,9 @@ struct AttnArgs {
 };
 size_t attn_workspace_bytes(int num_q, int heads, int window, bool decode, int max_sel = 512);
 cudaError_t launch_sparse_mqa(const AttnArgs &a, bool decode, cudaStream_t s);
+// The tcgen05 form for FP8 rows and 64 heads per CTA (no workspace: splits of
+// a query merge inside their thread-block cluster).
+bool sparse_mqa_tc_supported(const AttnArgs &a);
+cudaError_t launch_sparse_mqa_tc(const AttnArgs &a, bool decode, cudaStream_t s);
 
 }  // namespace csa
