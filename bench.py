@@ -49,6 +49,8 @@ def parse():
     p.add_argument("--workload", default="decode_128k")
     p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="leave the 1M decode workloads out of the default line")
     p.add_argument("--topk-form", default="auto", choices=["auto", "fused", "separate"],
                    help="indexer + top-512 form: the selecting indexer + row merge, the plain "
                         "indexer + top-k, or whichever probes faster (default)")
@@ -72,22 +74,19 @@ def indexer_source_hash() -> str:
 
 
 def profiled_traffic(w):
-    """DRAM bytes (read + write) per indexer launch from the committed ncu
-    summary of this workload, or None when there is none or the indexer's
-    sources changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", f"indexer_tc_{w.name.replace('_', '')}.md")
-    if not os.path.exists(path):
+    """DRAM bytes (read + write) per indexer launch from the committed capture
+    record profiles/indexer_tc_<workload>.json (written from an ncu capture of
+    this workload), or None when there is none or the indexer's sources have
+    changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"indexer_tc_{w.name.replace('_', '')}.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
         return None
-    vals = {}
-    with open(path) as fh:
-        for line in fh:
-            if ":" in line and line.split(":", 1)[0].strip() in ("traffic_bytes_per_launch",
-                                                                  "source_sha256"):
-                k, v = line.split(":", 1)
-                vals[k.strip()] = v.split()[0].strip("`") if v.split() else ""
-    if vals.get("source_sha256") != indexer_source_hash() or "traffic_bytes_per_launch" not in vals:
+    if rec.get("source_sha256") != indexer_source_hash():
         return None
-    return int(vals["traffic_bytes_per_launch"])
+    return int(rec["traffic_bytes_per_launch"])
 
 
 def peaks():
@@ -121,12 +120,20 @@ def _visible(w, ratio):
 
 def indexer_alg_bytes(w, ratio=4):
     """Bytes one indexer launch must move: every request's visible keys (codes
-    + scales) once, the query codes and weights, and the logits written
-    (ratio raw tokens per key: 4 for C4, 1 for DSA)."""
-    nv, per_req = _visible(w, ratio)
+    + scales) once, and the query codes, scales and folded weights (ratio raw
+    tokens per key: 4 for C4, 1 for DSA).  The logits it writes are an
+    implementation detail of the separate indexer + top-512 form and are
+    counted apart (indexer_logit_bytes)."""
+    _, per_req = _visible(w, ratio)
     qb = {"bf16": 2 * w.idx_dim, "fp8": w.idx_dim + 4, "fp4": w.idx_dim // 2 + w.idx_dim // 16 + 4}
-    return int(per_req.sum() * index_bytes_per_key(w) + nv.sum() * 4 +
-               w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4))
+    return int(per_req.sum() * index_bytes_per_key(w) + w.num_q * w.idx_heads * (qb[w.idx_fmt] + 4))
+
+
+def indexer_logit_bytes(w, ratio=4):
+    """Bytes of the fp32 logits one indexer launch writes (one per visible
+    (query row, key) pair)."""
+    nv, _ = _visible(w, ratio)
+    return int(nv.sum() * 4)
 
 
 def indexer_flops(w, ratio=4):
@@ -159,7 +166,8 @@ def indexer_roofline(w, t_idx, hbm, hbm_src, traffic, ratio=4):
     fl = indexer_flops(w, ratio)
     tpk, tsrc = tensor_peak(w.idx_fmt)
     ridge = tpk * 1e12 / (hbm * 1e9)
-    line = {"alg_bytes_per_launch": ib, "flops_per_launch": fl, "launch_ms": t_idx * 1e3,
+    line = {"alg_bytes_per_launch": ib, "logit_bytes_per_launch": indexer_logit_bytes(w, ratio),
+            "flops_per_launch": fl, "launch_ms": t_idx * 1e3,
             "intensity_flop_per_byte": fl / ib, "ridge_flop_per_byte": ridge}
     if fl / ib > ridge:
         ach = fl / t_idx / 1e12
@@ -400,8 +408,11 @@ def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_byte
     return {"value": world * num_q / t, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": t * 1e3,
             "pipelined": f"depth 2: inputs of step i+1 copied in and outputs of step i-1 read "
-                         f"back while step i computes; no L2 flush (working set "
-                         f"{step_bytes / 1e6:.0f} MB > L2 {l2 / 1e6:.0f} MB)",
+                         f"back while step i computes; no L2 flush between steps, so this is "
+                         f"a warm-L2 figure (working set {step_bytes / 1e6:.0f} MB, L2 "
+                         f"{l2 / 1e6:.0f} MB: part of it stays resident); the flushed "
+                         f"one-step-at-a-time figure is beside it",
+            "l2": "warm (pipelined)",
             "ms_per_step_one_at_a_time": t_seq * 1e3}
 
 
@@ -556,7 +567,8 @@ def main_hca(args, world, rank, local, dev):
                        hca_step_alg_bytes(w, int(batch.new_tokens.sum())))
     split = csa.csa_hca_attention_workspace_size(w.num_q, w.heads, w.window, batch.decode,
                                                  batch.max_hca) > 0
-    launches = (1 if batch.max_new >= 128 else 0) + (2 if split else 1)
+    tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0    # merges its own splits
+    launches = (1 if batch.max_new >= 128 else 0) + (1 if tc_attention or not split else 2)
     if rank == 0:
         hbm, src = peaks()
         ab = hca_attn_alg_bytes(w)
@@ -571,8 +583,10 @@ def main_hca(args, world, rank, local, dev):
                "data": "synthetic", "config": cfg,
                "hbm": {"step_alg_bytes": sb, "step_gbs": sb / t_step / 1e9,
                        "frac_of_peak": sb / t_step / 1e9 / hbm},
-               "roofline": {"kernel": "hca attention (sparse_mqa kernel, dense mode"
-                                      + (", + combine)" if split else ")"),
+               "roofline": {"kernel": ("hca attention (sparse_mqa_tc_kernel, dense mode)"
+                                       if tc_attention else
+                                       "hca attention (sparse_mqa kernel, dense mode"
+                                       + (", + combine)" if split else ")")),
                             "bound": "hbm", "achieved": achieved, "peak": hbm,
                             "peak_source": src, "unit": "GB/s", "frac": achieved / hbm,
                             "traffic": None, "alg_bytes_per_launch": ab,
@@ -652,7 +666,8 @@ def main_dsa(args, world, rank, local, dev):
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
                        dsa_step_alg_bytes(w))
     split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, 0, batch.decode) > 0
-    launches = 2 + 1 + 1 + 2 + (2 if split else 1)
+    tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0    # merges its own splits
+    launches = 2 + 1 + 1 + 2 + (1 if tc_attention or not split else 2)
     if rank == 0:
         hbm, src = peaks()
         sb = dsa_step_alg_bytes(w)
@@ -679,37 +694,16 @@ def main_dsa(args, world, rank, local, dev):
         dist.destroy_process_group()
 
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        run_reference(args)
-        return
+def measure_csa(args, name, world, rank, local, dev, full=True):
+    """One CSA decode workload on this rank's GPU: caches built from seeded
+    synthetic draws, the step captured in a CUDA graph and timed (max over
+    ranks).  Returns the JSON line's fields on rank 0 (None elsewhere); with
+    full=False the end-to-end leg and the CPU baseline are left out."""
     import torch
-    import torch.distributed as dist
 
-    from compressed_sparse_attention_12_b200 import build, csa, pipeline, synth
+    from compressed_sparse_attention_12_b200 import csa, pipeline, synth
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local)
-    if rank == 0:
-        build.build()
-    if world > 1:
-        dist.barrier()
-    csa.lib()
-    if args.workload.startswith("hca_"):
-        main_hca(args, world, rank, local, dev)
-        return
-    if args.workload.startswith("dsa_"):
-        main_dsa(args, world, rank, local, dev)
-        return
-
-    w = rank_workload(args.workload, rank)
+    w = rank_workload(name, rank)
     data = synth.draw(w, dev)
     batch = pipeline.CsaBatch(w, data, device=dev)
     arena = pack_inputs(batch, ["q_idx", "w_head", "q", "raw_kv", "gate", "raw_idx_k", "idx_gate"],
@@ -822,18 +816,22 @@ def main():
     fused[0], g = best[0], best[1]
     topk_forms = {("fused" if c[0] else "separate"): round(c[2] * 1e3, 2) for c in candidates}
     # kernels per step: compress (2 when blocks complete), quantise, indexer (selecting
-    # or plain), top-k (merge, or one or two launches), attention (1, +1 combine when split)
+    # or plain), top-k (merge, or one or two launches), attention (the tensor-core
+    # kernel for FP8 rows and 64-head groups merges its splits itself; the
+    # warp-level kernels add a combine launch when they split)
     # the top-512 is one launch for rows of at most 49152 keys, else two
     topk_launches = 1 if batch.max_c4 <= 49152 else 2
+    tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0
+    split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, w.window, batch.decode) > 0
     launches_per_step = (2 if batch.max_new >= 4 else 0) + 1 + 1 + (1 if fused[0] else topk_launches) + \
-        (2 if csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, w.window, batch.decode) > 0 else 1)
+        (1 if tc_attention or not split else 2)
 
     t_step, t_idx, ck = time_graph(g, stream, args, l2_flush, (ev_i0, ev_i1), world, dev, local,
                                    batch.check_status)
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.profile:
+    if full and not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
                        step_alg_bytes(w))
 
@@ -855,10 +853,68 @@ def main():
                                             "indexer_logits (indexer_tc_kernel)")},
                                 **indexer_roofline(w, t_idx, hbm, src, traffic)),
                "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": ck}
-        if not args.no_cpu_baseline and not args.profile and world == 1:
+        if full and not args.no_cpu_baseline and not args.profile and world == 1:
             out["cpu_baseline"] = cpu_baseline(w, data, batch.pt_host)
+        return out
+    return None
+
+
+EXTRA_WORKLOADS = ("decode_1m", "decode_1m_wide")
+
+
+def extra_line(o):
+    """The fields of one extra workload's measurement kept in the main line."""
+    keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "hbm",
+            "roofline", "gpu_launches", "clocks")
+    return {k: o[k] for k in keep if k in o}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from compressed_sparse_attention_12_b200 import build, csa, pipeline, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    csa.lib()
+    if args.workload.startswith("hca_"):
+        main_hca(args, world, rank, local, dev)
+        return
+    if args.workload.startswith("dsa_"):
+        main_dsa(args, world, rank, local, dev)
+        return
+
+    out = measure_csa(args, args.workload, world, rank, local, dev, full=True)
+    # The metric is quoted at 128K and 1M contexts: the default line also
+    # carries the two 1M decode workloads (device-timed step, same contract).
+    if args.workload == "decode_128k" and not args.profile and not args.no_extra:
+        ea = argparse.Namespace(**vars(args))
+        ea.steps, ea.warmup = min(args.steps, 100), max(3, min(args.warmup, 5))
+        extras = []
+        for name in EXTRA_WORKLOADS:
+            torch.cuda.empty_cache()
+            o = measure_csa(ea, name, world, rank, local, dev, full=False)
+            if o is not None:
+                extras.append(extra_line(o))
+        if out is not None:
+            out["configs"] = extras
+    if rank == 0:
         print(json.dumps(out), flush=True)
-    del g
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

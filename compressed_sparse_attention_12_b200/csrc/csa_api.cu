@@ -454,7 +454,7 @@ csa_status_t csa_topk512_page_transform_noalloc(const float *logits, int64_t log
     if (bs < 1 || !c4_seq_lens || !cu_q || !page_table || !c4_sparse_page_indices)
         return CSA_ERR_INVALID;
     if (max_c4_len > 0 && (!logits || logits_stride < max_c4_len)) return CSA_ERR_INVALID;
-    if (csa_topk512_workspace_size(num_q, max_c4_len) > (size_t)CSA_TOPK_NOALLOC_MAX_BYTES)
+    if (csa::topk_scratch_bytes(num_q, max_c4_len) > (size_t)CSA_TOPK_NOALLOC_MAX_BYTES)
         return CSA_ERR_WORKSPACE;
     if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
     csa::TopkArgs a{logits, logits_stride, num_q, c4_seq_lens, bs, cu_q, q_pos, page_table,

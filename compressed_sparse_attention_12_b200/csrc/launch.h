@@ -118,6 +118,9 @@ struct TopkArgs {
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s);
 // Same, with the scratch in the library's own device array (no workspace).
 cudaError_t launch_topk512_noalloc(const TopkArgs &a, cudaStream_t s);
+// Bytes of scratch the selection uses for these sizes (0 when it runs in one
+// launch, rows of at most 49152 logits).
+size_t topk_scratch_bytes(int num_q, int max_c4_len);
 // Row-level merge of per-chunk candidates (chunk_len keys per chunk, the last
 // one shorter; every chunk but a single one must hold >= 512 keys).
 cudaError_t launch_topk_stage2(const TopkArgs &a, int max_chunks, int chunk_len,

@@ -19,6 +19,8 @@
 //            page_table[s/64]*64 + s%64 and raw indices.
 #include "common.cuh"
 #include "launch.h"
+#include <atomic>
+
 #include "topk.cuh"
 
 namespace csa {
@@ -376,6 +378,13 @@ size_t topk_workspace_bytes(int num_q, int max_c4_len) {
     return chunks * kTopK * 8 + chunks * sizeof(uint2);
 }
 
+// Scratch the selection actually uses: none for rows of at most kTkRowMax
+// logits (one launch, the row in registers or shared memory), the two-stage
+// candidate buffer for longer rows.
+size_t topk_scratch_bytes(int num_q, int max_c4_len) {
+    return max_c4_len <= kTkRowMax ? 0 : topk_workspace_bytes(num_q, max_c4_len);
+}
+
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
     if (a.num_q == 0) return cudaSuccess;
     if (a.max_c4_len <= kTkRegMax) {
@@ -431,24 +440,27 @@ cudaError_t launch_topk_stage2(const TopkArgs &a, int max_chunks, int chunk_len,
 // file-scope device array (held by every GPU that loads the library until the
 // process exits).  Host code may not use the array's name as a device
 // address, so its address is looked up once per device with that device
-// current and cached.  Nothing in the array needs to start at zero: stage 1
-// writes every entry stage 2 reads.  Concurrent calls share it and race.
+// current and cached (an atomic per device: host threads may make the first
+// call concurrently; they store the same value).  The cached address belongs
+// to the device's context at that time and is not refreshed after a device
+// reset.  Nothing in the array needs to start at zero: stage 1 writes every
+// entry stage 2 reads.  Concurrent calls share it and race.
 static __device__ __align__(256) uint8_t g_topk_scratch[CSA_TOPK_NOALLOC_MAX_BYTES];
 
 cudaError_t launch_topk512_noalloc(const TopkArgs &a, cudaStream_t s) {
-    static void *scratch_addr[64] = {nullptr};
+    static std::atomic<void *> scratch_addr[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!scratch_addr[dev]) {
-        void *ptr = nullptr;
+    void *ptr = scratch_addr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
         e = cudaGetSymbolAddress(&ptr, g_topk_scratch);
         if (e != cudaSuccess) return e;
-        scratch_addr[dev] = ptr;
+        scratch_addr[dev].store(ptr, std::memory_order_release);
     }
     TopkArgs b = a;
-    b.workspace = scratch_addr[dev];
+    b.workspace = ptr;
     return launch_topk512(b, s);
 }
 

@@ -239,8 +239,13 @@ csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stri
  * Scratch lives in one file-scope device array of CSA_TOPK_NOALLOC_MAX_BYTES
  * bytes inside libcsa.so: every GPU that loads the library holds that memory
  * until the process exits.  The first call on a device (with that device
- * current) looks up the array's device address once; make that first call
- * before any stream capture.  Calls return CSA_ERR_WORKSPACE without launching
+ * current) looks up the array's device address once and caches it for the
+ * process; make that first call before any stream capture.  The cached
+ * address belongs to the device's context of that time: after cudaDeviceReset
+ * on a device, do not call this entry point again in the same process (load
+ * the library in a fresh process).  Rows of at most 49152 compressed keys are
+ * selected in one launch that needs no scratch, so any number of them is
+ * accepted; for longer rows calls return CSA_ERR_WORKSPACE without launching
  * when csa_topk512_workspace_size(num_q, max_c4_len) exceeds the maximum.
  * Every call shares the one array (its contents persist between calls and
  * nothing in it needs to start at zero), so calls that overlap on the GPU --
@@ -342,13 +347,19 @@ csa_status_t csa_topk512_merge(int32_t num_q, int32_t idx_heads, int32_t idx_dim
  *   workspace >= csa_sparse_mqa_workspace_size(num_q, heads, window, decode)
  * The two entry points compute the same function; _decode splits each
  * query's rows across CTAs (few queries, many rows each), _prefill gives each
- * query its own CTA (many queries).
+ * query its own CTA (many queries).  FP8 rows with heads a multiple of 64 run
+ * on the tensor-core kernel, whose splits (a thread-block cluster of at most 8
+ * CTAs per query) merge inside the kernel and use no workspace; the other
+ * cases write split partials to the workspace and merge them in a second
+ * launch.
  * Ordering: like every kernel of the library this one is launched with
  * programmatic dependent launch; with FP8 rows it reads q, cu_q, q_pos and
- * seq_lens before waiting for the kernel enqueued just before it, so these
- * must not be written by a kernel that lets its successor start early and
- * runs immediately before this call (the library's own kernels never write
- * them; data written by a copy or by earlier work is safe).
+ * seq_lens before waiting for the kernels enqueued before it.  A chain of
+ * launches that each let their successor start early can have several of
+ * them running at once, so these inputs must not be written by any such
+ * early-triggering kernel enqueued on the stream since the last ordinary
+ * launch, copy or event wait (the library's own kernels never write them;
+ * data written by a copy, or by work ordered before that point, is safe).
  */
 size_t csa_sparse_mqa_workspace_size(int32_t num_q, int32_t heads, int32_t window,
                                      int32_t decode);

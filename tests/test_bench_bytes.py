@@ -10,23 +10,26 @@ from compressed_sparse_attention_12_b200 import synth  # noqa: E402
 
 
 def test_indexer_bytes_decode_128k():
-    # 32 rows x 32768 visible keys of (128 FP8 codes + 4 B scale) + a 4 B logit
-    # each, plus 64 query heads of (128 + 4) B codes and a 4 B weight per row
+    # 32 requests x 32768 keys of (128 FP8 codes + 4 B scale), plus 64 query
+    # heads of (128 + 4) B codes and a 4 B weight per row; the 4 B logits are
+    # counted apart
     w = synth.workload("decode_128k")
-    assert bench.indexer_alg_bytes(w) == 32 * 32768 * (132 + 4) + 32 * 64 * (132 + 4)
+    assert bench.indexer_alg_bytes(w) == 32 * 32768 * 132 + 32 * 64 * (132 + 4)
+    assert bench.indexer_logit_bytes(w) == 32 * 32768 * 4
 
 
 def test_indexer_bytes_decode_1m_fp4():
     # FP4 8x64: a key is 32 code bytes + 4 block scales + a 4 B row scale
     w = synth.workload("decode_1m")
     assert bench.index_bytes_per_key(w) == 40
-    assert bench.indexer_alg_bytes(w) == 8 * 262144 * (40 + 4) + 8 * 8 * (40 + 4)
+    assert bench.indexer_alg_bytes(w) == 8 * 262144 * 40 + 8 * 8 * (40 + 4)
 
 
 def test_indexer_bytes_dsa_counts_every_raw_key():
     # ratio 1: query at position L-1 sees L keys
     w = synth.workload("dsa_128k")
-    assert bench.indexer_alg_bytes(w, 1) == 32 * 131072 * (132 + 4) + 32 * 64 * (132 + 4)
+    assert bench.indexer_alg_bytes(w, 1) == 32 * 131072 * 132 + 32 * 64 * (132 + 4)
+    assert bench.indexer_logit_bytes(w, 1) == 32 * 131072 * 4
 
 
 def test_step_bytes_decode_128k():
@@ -52,7 +55,8 @@ def test_prefill_counts_each_key_once_and_is_tensor_bound():
     L = 262144 + 4096
     nv = sum(min(L // 4, (p + 1) // 4) for p in range(L - 4096, L))
     assert bench.indexer_flops(w) == nv * 64 * 128 * 2
-    assert bench.indexer_alg_bytes(w) == (L // 4) * 132 + nv * 4 + 4096 * 64 * 136
+    assert bench.indexer_alg_bytes(w) == (L // 4) * 132 + 4096 * 64 * 136
+    assert bench.indexer_logit_bytes(w) == nv * 4
     line = bench.indexer_roofline(w, 7.8e-3, 6551.4, "measured", None)
     assert line["bound"] == "tensor" and line["unit"] == "TFLOP/s"
     assert abs(line["achieved"] - nv * 64 * 128 * 2 / 7.8e-3 / 1e12) < 1e-6
@@ -63,6 +67,7 @@ def test_decode_roofline_is_hbm_bound():
     w = synth.workload("decode_128k")
     line = bench.indexer_roofline(w, 43.1e-6, 6551.4, "measured", 144419328)
     assert line["bound"] == "hbm" and line["unit"] == "GB/s"
-    assert line["alg_bytes_per_launch"] == 142884864
+    assert line["alg_bytes_per_launch"] == 32 * 32768 * 132 + 32 * 64 * 136
+    assert line["logit_bytes_per_launch"] == 32 * 32768 * 4
     assert line["traffic"] == 144419328
     assert line["intensity_flop_per_byte"] < line["ridge_flop_per_byte"]

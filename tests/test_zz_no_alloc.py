@@ -45,7 +45,11 @@ def test_noalloc_equals_workspace_entry_point_on_consecutive_calls():
     build.build()
     rng = np.random.default_rng(2024)
     cases = [_case(rng, [300, 9000, 70000], [1, 3, 2]),
-             _case(rng, [262144, 511, 40000, 7], [1, 1, 4, 1])]
+             _case(rng, [262144, 511, 40000, 7], [1, 1, 4, 1]),
+             # 4100 rows of short lists: one launch with no scratch, accepted
+             # although a two-stage workspace for them would exceed the array
+             _case(rng, [1000] * 41, [100] * 41)]
+    assert csa.csa_topk512_workspace_size(41 * 100, 1000) > csa.TOPK_NOALLOC_MAX_BYTES
     for c in cases:                     # two calls in a row, different sizes
         st_ref = torch.zeros(1, dtype=torch.int32, device="cuda")
         st_na = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -70,7 +74,9 @@ def test_noalloc_rejects_sizes_beyond_its_array():
     build.build()
     L = csa.lib()
     p = lambda: ctypes.c_void_p(4096)        # never dereferenced: rejected on the host
-    num_q, max_c4 = 4097, 8192               # 4097 * 1 chunk * 512 * 8 B > 16 MiB
+    # rows longer than 49152 keys take the two-stage selection, whose
+    # candidates (512 rows x 8 chunks x (512 x 8 + 8) B) exceed 16 MiB
+    num_q, max_c4 = 512, 65536
     assert csa.csa_topk512_workspace_size(num_q, max_c4) > csa.TOPK_NOALLOC_MAX_BYTES
     r = L.csa_topk512_page_transform_noalloc(p(), max_c4, num_q, p(), 1, p(), None, p(), 128,
                                              128 * 64, 64, max_c4, p(), None, None, None)
