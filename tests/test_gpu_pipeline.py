@@ -64,6 +64,21 @@ def test_step_end_to_end(name, scale):
           f"min {np.min(overlaps):.5f}, identical sets {exact}/{len(ref)}")
     assert np.mean(overlaps) >= 0.98
     assert exact >= 0.5 * len(ref)
+    # every query: the attention on exactly the rows the GPU selected and its
+    # window, decoded from the GPU's own cache bytes, against the oracle's
+    fp8 = w.kv_fmt == "fp8"
+    c4c = batch.c4_cache.cpu().numpy()
+    rwc = batch.raw_cache.cpu().numpy()
+    qf = data["q"].double().numpy()
+    for t in ref:
+        b = int(np.searchsorted(w.cu_q, t, side="right") - 1)
+        sel = phys[t][phys[t] >= 0]
+        win = orc.window_positions(int(w.q_pos[t]), w.window)
+        rsl = orc.raw_slot(batch.pt_host[b], win)
+        rows = np.concatenate([orc.kv_decode_rows(c4c[sel], fp8).reshape(-1, 576),
+                               orc.kv_decode_rows(rwc[rsl], fp8).reshape(-1, 576)])
+        ro, _ = orc.sparse_attention(qf[t], rows, batch.sm_scale)
+        assert (np.abs(out[t] - ro) - bf16_bound(ro, rel=0.0)).max() <= tol, t
 
 
 def _full_index_check(name, sample_q):
@@ -154,12 +169,139 @@ def _full_index_check(name, sample_q):
         assert np.abs(lse.cpu().numpy()[b] - rl).max() <= 2e-2, b
 
 
+def _full_ragged_check(name, sample_q):
+    """Indexer + top-512 at full size for workloads with any mix of request
+    lengths and query rows per request (the ragged serving batch: lengths up to
+    1M, compressed lengths below 512 padded with -1, 1 or 5 query rows per
+    request): logits on oracle-quantised keys to 1e-2 on every visible key of
+    every query row, top-512 bit-exact (with -1 padding) on the oracle's
+    logits in the benchmark's launch shape, attention on sampled queries."""
+    from compressed_sparse_attention_12_b200 import csa, synth
+    w = synth.workload(name)
+    pt = synth.page_table(w)
+    rng = np.random.default_rng(23)
+    bs, Hi, Di, nq = w.bs, w.idx_heads, w.idx_dim, w.num_q
+    c4 = w.c4_lens.astype(np.int64)
+    off = np.concatenate([[0], np.cumsum(c4)])
+    n_keys = int(off[-1])
+    keys = (rng.standard_t(3, (n_keys, Di)) if w.key_dist == "student_t3"
+            else rng.standard_normal((n_keys, Di)))
+    kq = orc.index_quantise(keys, w.idx_fmt)
+    del keys
+    slots = np.concatenate([pt[b, np.arange(c4[b]) // 64].astype(np.int64) * 64 +
+                            np.arange(c4[b]) % 64 for b in range(bs)])
+    n_slots = w.num_pages * 64
+    kc, kb, ks = index_arrays(kq, w.idx_fmt, Di, n_slots, slots)
+    qx = rng.standard_normal((nq, Hi, Di))
+    qq = orc.index_quantise(qx, w.idx_fmt)
+    qc, qb, qs = index_arrays(qq, w.idx_fmt, Di, nq * Hi)
+    ww = rng.uniform(size=(nq, Hi)).astype(np.float32)
+    wf = (ww * (qq["scales"].reshape(nq, Hi) if w.idx_fmt != "bf16" else 1.0)).astype(np.float32)
+    max_c4 = int(c4.max())
+    stride = (max_c4 + 15) // 16 * 16
+    logits = torch.empty((nq, stride), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c4_d, cu_q, q_pos = dev(c4.astype(np.int32)), dev(w.cu_q), dev(w.q_pos)
+    csa.csa_indexer_logits(qc, qb, dev(wf), Hi, Di, csa.FMT[w.idx_fmt], kc, kb, ks, dev(pt), c4_d,
+                           cu_q, q_pos, max_c4, logits, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    got = logits.cpu().numpy()
+    kd = kq["deq"]
+    qd = qq["deq"].reshape(nq, Hi, Di)
+    lg32 = np.zeros((nq, stride), dtype=np.float32)
+    nv = np.zeros(nq, dtype=np.int64)
+    req = np.zeros(nq, dtype=np.int64)
+    for b in range(bs):
+        for t in range(int(w.cu_q[b]), int(w.cu_q[b + 1])):
+            req[t] = b
+            nv[t] = min(int(c4[b]), (int(w.q_pos[t]) + 1) // 4)
+            if nv[t] == 0:
+                continue
+            ref = orc.indexer_logits(qd[t:t + 1], ww[t:t + 1], kd[off[b]:off[b] + c4[b]],
+                                     [nv[t]])[0, :nv[t]]
+            assert rel_close(got[t, :nv[t]], ref, 1e-2).all(), (b, t)
+            lg32[t, :nv[t]] = ref.astype(np.float32)
+    del kd
+    out = torch.empty((nq, 512), dtype=torch.int32, device="cuda")
+    raw = torch.empty((nq, 512), dtype=torch.int32, device="cuda")
+    csa.csa_topk512_page_transform(dev(lg32), c4_d, cu_q, q_pos, dev(pt), n_slots, max_c4, out, raw,
+                                   status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    go, gr = out.cpu().numpy(), raw.cpu().numpy()
+    short = 0
+    for t in range(nq):
+        phys, logical = orc.topk_transform(lg32[t], int(nv[t]), pt[req[t]], n_slots)
+        assert np.array_equal(gr[t], logical) and np.array_equal(go[t], phys), t
+        short += int(nv[t] < 512)
+    if name == "ragged":
+        assert short > 0              # some rows are padded with -1
+    # attention on sampled queries: rows drawn per slot (queries of one request
+    # share the rows of the slots they both select)
+    fp8 = w.kv_fmt == "fp8"
+    rb = 656 if fp8 else 1152
+    c4_cache = torch.zeros((n_slots, rb), dtype=torch.uint8, device="cuda")
+    raw_cache = torch.zeros((w.num_pages * 256, rb), dtype=torch.uint8, device="cuda")
+    q = torch.randn((nq, w.heads, 576), generator=torch.Generator().manual_seed(5)).bfloat16()
+    sm_scale = 1.0 / math.sqrt(576)
+    c4_rows, raw_rows = {}, {}
+
+    def rows_at(table, cache, sl):
+        new = [int(x) for x in sl if int(x) not in table]
+        if new:
+            enc = orc.kv_encode_rows(rng.standard_normal((len(new), 576)), fp8)
+            cache[dev(np.asarray(new, dtype=np.int64))] = dev(enc)
+            for x, e in zip(new, orc.kv_decode_rows(enc, fp8)):
+                table[x] = e
+        return np.array([table[int(x)] for x in sl]).reshape(-1, 576)
+
+    want = {}
+    for t in sample_q:
+        b = int(req[t])
+        sel = go[t][go[t] >= 0]
+        win = orc.window_positions(int(w.q_pos[t]), w.window)
+        rsl = pt[b, win // 256].astype(np.int64) * 256 + win % 256
+        want[t] = (sel, rsl)
+    for t, (sel, rsl) in want.items():
+        rows_at(c4_rows, c4_cache, sel)
+        rows_at(raw_rows, raw_cache, rsl)
+    o = torch.empty((nq, w.heads, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((nq, w.heads), dtype=torch.float32, device="cuda")
+    decode = bool((w.q_lens <= 8).all())
+    fn = csa.csa_sparse_mqa_decode if decode else csa.csa_sparse_mqa_prefill
+    fn(q.cuda(), c4_cache, raw_cache, csa.FMT[w.kv_fmt], out, dev(pt),
+       dev(w.seq_lens.astype(np.int32)), cu_q, q_pos, w.window, sm_scale, o, lse, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    go_, gl = o.float().cpu().numpy(), lse.cpu().numpy()
+    tol = 2e-2 if fp8 else 5e-3
+    for t, (sel, rsl) in want.items():
+        allrows = np.concatenate([rows_at(c4_rows, c4_cache, sel), rows_at(raw_rows, raw_cache, rsl)])
+        ro, rl = orc.sparse_attention(q[t].double().numpy(), allrows, sm_scale)
+        assert (np.abs(go_[t] - ro) - bf16_bound(ro, rel=0.0)).max() <= tol, t
+        assert np.abs(gl[t] - rl).max() <= 2e-2, t
+
+
 def test_full_size_decode_128k():
     _full_index_check("decode_128k", sample_q=[0, 13, 31])
 
 
 def test_full_size_decode_1m():
     _full_index_check("decode_1m", sample_q=[0, 7])
+
+
+def test_full_size_decode_1m_wide():
+    _full_ragged_check("decode_1m_wide", sample_q=[0, 3, 7])
+
+
+def test_full_size_ragged():
+    # queries 0 and 1 belong to the two requests shorter than 512 compressed
+    # rows; the last five are the verify rows of the last (5-row) request
+    from compressed_sparse_attention_12_b200 import synth
+    w = synth.workload("ragged")
+    last = int(w.num_q)
+    _full_ragged_check("ragged", sample_q=[0, 1, 2, 40, last - 5, last - 1])
 
 
 def test_full_size_prefill_sampled():

@@ -371,6 +371,41 @@ def test_indexer_logits(fmt, dim, heads):
             assert np.isnan(got[t, nv:]).all()
 
 
+@pytest.mark.parametrize("fmt,dim,heads", [("fp8", 128, 64), ("fp4", 64, 8), ("bf16", 64, 8)])
+def test_indexer_logits_cuda_core_path(fmt, dim, heads):
+    """Index caches whose slot count is not a multiple of 64 (here 64k + 8)
+    take the CUDA-core indexer (the tensor-core kernel moves whole 64-row
+    pages); same logits as the oracle to 1e-2."""
+    csa = _csa()
+    c = _indexer_case(fmt, dim, heads, seed=7 + dim, c4_lens=[0, 63, 65, 1000, 3000],
+                      q_lens=[1, 2, 1, 5, 1], dist="t3" if fmt == "fp4" else "normal")
+    n_rows = c["n_slots"] + 8
+    kc, kb, ks = index_arrays(c["keys"], fmt, dim, n_rows, c["slots"])
+    qc, qb, qs = index_arrays(c["qq"], fmt, dim, c["nq"] * heads)
+    wf = (c["w"] * (c["qq"]["scales"].reshape(c["nq"], heads) if fmt != "bf16" else 1.0)
+          ).astype(np.float32)
+    max_c4 = int(c["c4"].max())
+    logits = torch.full((c["nq"], max_c4 + 16), float("nan"), dtype=torch.float32, device="cuda")
+    st = zstatus()
+    csa.csa_indexer_logits(qc, qb, dev(wf), heads, dim, FMT[fmt], kc, kb, ks, dev(c["pt"]),
+                           dev(c["c4"].astype(np.int32)), dev(c["cu_q"]), dev(c["q_pos"]), max_c4,
+                           logits, num_slots=n_rows, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    got = logits.cpu().numpy()
+    qd = c["qq"]["deq"].reshape(c["nq"], heads, dim)
+    kd = c["keys"]["deq"]
+    off = np.concatenate([[0], np.cumsum(c["c4"])])
+    for b in range(len(c["c4"])):
+        for t in range(c["cu_q"][b], c["cu_q"][b + 1]):
+            nv = min(int(c["c4"][b]), (int(c["q_pos"][t]) + 1) // 4)
+            if nv:
+                ref = orc.indexer_logits(qd[t:t + 1], c["w"][t:t + 1],
+                                         kd[off[b]:off[b] + c["c4"][b]], [nv])[0, :nv]
+                assert rel_close(got[t, :nv], ref, 1e-2).all(), (b, t)
+            assert np.isnan(got[t, nv:]).all()
+
+
 # ------------------------------------------------------------------ top-512
 
 def _topk_case(case, rng):
