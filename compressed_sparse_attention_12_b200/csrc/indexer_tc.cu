@@ -33,7 +33,12 @@
 
 namespace csa {
 
-constexpr int kTcThreads = 320;   // 10 warps: producer, MMA, two epilogue groups of 4
+// Warps: producer, MMA, then EG epilogue groups of four (EG = 2: 320 threads,
+// two CTAs per SM; EG = 4 for the 256-column accumulators of prefill-shaped
+// launches: 576 threads, one CTA per SM)
+template <int EG>
+__host__ __device__ constexpr int tc_threads() { return 64 + 128 * EG; }
+constexpr int kTcThreads = tc_threads<2>();
 constexpr int kTcTile = 128;      // keys per tile (two 64-row pages)
 
 template <int RB>
@@ -73,12 +78,94 @@ constexpr int kKsRing = 8;     // key-scale tiles in flight per epilogue group
 constexpr int kSfLag = 4;
 constexpr int kSfSlots = kSfLag + 1;
 
-template <int FMT, int RB>
-__global__ void __launch_bounds__(kTcThreads, 2)
+// Query group g of a launch.  Request b's query rows form ceil(rows_b / qg)
+// groups of qg consecutive rows (the last one shorter), numbered after the
+// groups of requests 0..b-1.  Sets *b_out and the group's first row *t0_out
+// (-1 when g is past the last group).  Every lane of the calling warp must be
+// active: the requests are scanned 32 at a time with a warp prefix sum.
+__device__ __forceinline__ void query_group(const int *cu_q, int bs, int qg, int g, int *b_out,
+                                            int *t0_out) {
+    *b_out = 0;
+    *t0_out = -1;
+    if (qg == 1) {                        // one group per row
+        if (g >= cu_q[bs]) return;
+        int lo = 0, hi = bs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (cu_q[mid] <= g) lo = mid; else hi = mid - 1;
+        }
+        *b_out = lo;
+        *t0_out = g;
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    int before = 0;                       // groups of the requests already scanned
+    for (int b0 = 0; b0 < bs; b0 += 32) {
+        const int bb = b0 + lane;
+        int first = 0, ng = 0;
+        if (bb < bs) {
+            first = cu_q[bb];
+            ng = (cu_q[bb + 1] - first + qg - 1) / qg;
+        }
+        int incl = ng;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        const uint32_t hit = __ballot_sync(0xffffffffu, g < before + incl);
+        if (hit) {
+            const int src = __ffs(hit) - 1;
+            const int excl = before + __shfl_sync(0xffffffffu, incl - ng, src);
+            *b_out = b0 + src;
+            *t0_out = __shfl_sync(0xffffffffu, first, src) + (g - excl) * qg;
+            return;
+        }
+        before += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
+// Upper bound of the number of query groups: sum over requests of
+// ceil(rows_b / qg) <= (num_q + bs * (qg - 1)) / qg, and at most num_q.
+static int query_groups_bound(int num_q, int bs, int qg) {
+    if (qg <= 1) return num_q;
+    const long long g = ((long long)num_q + (long long)bs * (qg - 1)) / qg;
+    return (int)(g < num_q ? g : num_q);
+}
+
+// Packed fp32 pair multiply-add: acc += a * b elementwise (one instruction
+// for two lanes of work on sm_100).
+__device__ __forceinline__ void ffma2(float2 &acc, float2 a, float2 b) {
+    uint64_t d;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+        : "=l"(d)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(acc.x), "f"(acc.y));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(d));
+}
+
+// acc += w[j] * ReLU(v[j]) over 16 accumulator columns (part of one query's
+// run of heads) as two pair accumulators, weights read 16 bytes at a time.
+__device__ __forceinline__ void relu_dot16(const uint32_t *v, const float *w, float2 (&acc)[2]) {
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) {
+        const float4 wv = *reinterpret_cast<const float4 *>(w + j);
+        ffma2(acc[0], make_float2(wv.x, wv.y),
+              make_float2(fmaxf(__uint_as_float(v[j]), 0.f), fmaxf(__uint_as_float(v[j + 1]), 0.f)));
+        ffma2(acc[1], make_float2(wv.z, wv.w),
+              make_float2(fmaxf(__uint_as_float(v[j + 2]), 0.f),
+                          fmaxf(__uint_as_float(v[j + 3]), 0.f)));
+    }
+}
+
+template <int FMT, int RB, int EG>
+__global__ void __launch_bounds__(tc_threads<EG>(), EG == 2 ? 2 : 1)
 indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                   const TcParams p, const TcSelect sel) {
     pdl_begin();
     using G = TcGeom<RB>;
+    constexpr int kThreads = tc_threads<EG>();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned carve-up: stages | q tile | w' | nv | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -105,15 +192,10 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // ---- which query group and key tiles (uniform over the CTA)
-    const int t0 = blockIdx.y;
-    int lo = 0, hi = a.bs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.cu_q[mid] <= t0) lo = mid; else hi = mid - 1;
-    }
-    const int b = lo;
-    const int first = a.cu_q[b], last = a.cu_q[b + 1];
-    if (((t0 - first) % p.qg) != 0) return;                 // not a group leader
+    int b, t0;
+    query_group(a.cu_q, a.bs, p.qg, (int)blockIdx.y, &b, &t0);
+    if (t0 < 0) return;                                     // past the last group
+    const int last = a.cu_q[b + 1];
     const int nq = min(p.qg, last - t0);
     const int cap = min(a.max_c4_len, a.pt_stride * kC4Page);
     int nv_max = 0;
@@ -152,14 +234,14 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         }
         for (int i = 0; i < p.nacc; i++) {
             tc::mbar_init(tc::saddr(&tfull[i]), 1);
-            tc::mbar_init(tc::saddr(&tempty[i]), 4);     // the 4 warps of one group
+            tc::mbar_init(tc::saddr(&tempty[i]), 4 * (EG / 2));   // the warps reading it
         }
         tc::mbar_init(tc::saddr(drain), 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
     if (threadIdx.x < 4) nv_s[threadIdx.x] = nv_q[threadIdx.x];
-    for (int u = threadIdx.x; u < 2 * my_tiles; u += kTcThreads) {
+    for (int u = threadIdx.x; u < 2 * my_tiles; u += kThreads) {
         const int pidx = tile_begin * 2 + u;
         int page = -1;
         if (pidx * kC4Page < nv_max && pidx < a.pt_stride) page = pt_row[pidx];
@@ -169,7 +251,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     {
         const uint8_t *qc = reinterpret_cast<const uint8_t *>(a.q_codes);
         const int chunks16 = RB / 16;
-        for (int u = threadIdx.x; u < p.n * chunks16; u += kTcThreads) {
+        for (int u = threadIdx.x; u < p.n * chunks16; u += kThreads) {
             const int n = u / chunks16, c = u % chunks16;
             const int qi = n / p.hi_pad, h = n % p.hi_pad;
             uint4 v = make_uint4(0, 0, 0, 0);
@@ -180,7 +262,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             *reinterpret_cast<uint4 *>(q_buf + chunk * p.n * G::kSpan +
                                        tc::swz(n, byte, G::kSpan)) = v;
         }
-        for (int n = threadIdx.x; n < p.n; n += kTcThreads) {
+        for (int n = threadIdx.x; n < p.n; n += kThreads) {
             const int qi = n / p.hi_pad, h = n % p.hi_pad;
             w_s[n] = (qi < nq && h < a.heads) ? a.q_weights[(int64_t)(t0 + qi) * a.heads + h] : 0.f;
         }
@@ -188,7 +270,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             // scale-factor layout of 128 rows: row n = m0 + 32*m1 keeps its four
             // block scales of K-step ks at byte ks*512 + m0*16 + m1*4
             constexpr int nsf = RB / 8;      // block scales per row (Di/16; a row is Di/2 bytes)
-            for (int u = threadIdx.x; u < 128 * G::kKSteps; u += kTcThreads) {
+            for (int u = threadIdx.x; u < 128 * G::kKSteps; u += kThreads) {
                 const int n = u % 128, ks = u / 128;
                 const int qi = n / p.hi_pad, h = n % p.hi_pad;
                 uint32_t wv = 0;
@@ -383,13 +465,19 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             tc::mbar_wait(tc::saddr(drain), 0, nullptr);
         }
     } else {
-        // ---------------- epilogue: group eg = (warp-2)/4 takes tiles i with i%2 == eg
+        // ---------------- epilogue: group eg = (warp-2)/4 takes the tiles of
+        // parity eg & 1; with four groups, eg >> 1 picks which half of the
+        // group's query rows (and so of the accumulator columns) it reduces
         const int eg = (warp - 2) >> 2;
+        const int par = eg & 1;
+        const int qh = EG == 4 ? p.qg / 2 : p.qg;          // query rows per group
+        const int x_lo = EG == 4 ? (eg >> 1) * qh : 0;
+        const int c_lo = x_lo * p.hi_pad, c_hi = min(p.n, c_lo + qh * p.hi_pad);
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float *lg = a.logits;
-        // Key scale of this thread's row for the group's j-th tile (i = eg + 2j):
+        // Key scale of this thread's row for the group's j-th tile (i = par + 2j):
         // a per-thread ring of kKsRing cp.async copies keeps the loads of the
         // next tiles in flight while this one is reduced.
         auto key_slot = [&](int i, bool &valid) -> int64_t {
@@ -405,7 +493,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         auto ring_issue = [&](int j) {
             if constexpr (FMT != CSA_FMT_BF16) {
                 bool v;
-                const int64_t slot = key_slot(eg + 2 * j, v);
+                const int64_t slot = key_slot(par + 2 * j, v);
                 if (slot >= 0) tc::cp_async4(tc::saddr(my_ring + (j % kKsRing) * kTcTile),
                                              a.k_scales + slot);
                 tc::cp_async_commit();
@@ -415,9 +503,9 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         // tile j+kKsRing-1 then goes to the slot read one tile earlier
 #pragma unroll 1
         for (int j = 0; j < kKsRing - 1; j++) ring_issue(j);
-        for (int i = eg; i < my_tiles; i += 2) {
+        for (int i = par; i < my_tiles; i += 2) {
             const int acc = i & (p.nacc - 1);     // same parity as i: this group's
-            const int j = (i - eg) >> 1;
+            const int j = (i - par) >> 1;
             const int sk = (tile_begin + i) * kTcTile + row;
             bool valid;
             const int64_t slot_i = key_slot(i, valid);
@@ -429,35 +517,52 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 kscale = valid ? my_ring[(j % kKsRing) * kTcTile] : 0.0f;
                 ring_issue(j + kKsRing - 1);
             }
-            if (!tc::mbar_wait(tc::saddr(&tfull[acc]), (uint32_t)((i / p.nacc) & 1), abort_flag)) {
+            // the other group's tile is being reduced meanwhile: sleep in the wait
+            if (!tc::mbar_wait_sleep(tc::saddr(&tfull[acc]), (uint32_t)((i / p.nacc) & 1),
+                                     abort_flag)) {
                 if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
                 *abort_flag = 1;
                 break;
             }
             tc::fence_after_sync();
+            // per query row x_lo + x of the group: sum_j w'[c+j] * ReLU(acc[c+j])
+            // over its hi_pad columns (a multiple of 16)
             float out[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t ta = tmem_base + lane_addr + (uint32_t)(acc * p.n);
-            for (int c0 = 0; c0 < p.n; c0 += 32) {
-                // 32 columns per TMEM round trip; sum_j w'[c+j] * ReLU(acc[c+j])
-                // over 16-column groups (a group never straddles two queries:
-                // hi_pad is a multiple of 16)
-                uint32_t v[32];
-                tc::tmem_ld32_nowait(ta + (uint32_t)c0, v);
+            if (p.hi_pad % 32 == 0) {
+                // 16-column TMEM loads, double-buffered: the load of the next
+                // 16 columns is in flight while these are reduced
+                uint32_t va[16], vb[16];
+                tc::tmem_ld16_nowait(ta + (uint32_t)c_lo, va);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int q16 = 0; q16 < 2; q16++) {
-                    const int c = c0 + 16 * q16;
-                    if (c < p.n) {
-                        float sacc = 0.0f;
-#pragma unroll
-                        for (int j = 0; j < 16; j++)
-                            sacc = fmaf(w_s[c + j], fmaxf(__uint_as_float(v[16 * q16 + j]), 0.0f),
-                                        sacc);
-                        const int qi = c / p.hi_pad;
-#pragma unroll
-                        for (int x = 0; x < 4; x++)
-                            if (x == qi) out[x] += sacc;
+                for (int x = 0; x < 4; x++) {
+                    if (x >= qh) break;
+                    const int ce = c_lo + (x + 1) * p.hi_pad;
+                    float2 sx[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    for (int c = ce - p.hi_pad; c < ce; c += 32) {
+                        tc::tmem_ld16_nowait(ta + (uint32_t)(c + 16), vb);
+                        relu_dot16(va, w_s + c, sx);
+                        tc::tmem_wait_ld();
+                        if (c + 32 < c_hi) tc::tmem_ld16_nowait(ta + (uint32_t)(c + 32), va);
+                        relu_dot16(vb, w_s + c + 16, sx);
+                        tc::tmem_wait_ld();
                     }
+                    out[x] = (sx[0].x + sx[1].x) + (sx[0].y + sx[1].y);
+                }
+            } else {
+#pragma unroll
+                for (int x = 0; x < 4; x++) {
+                    if (x >= qh) break;
+                    const int cb = c_lo + x * p.hi_pad, ce = cb + p.hi_pad;
+                    float2 sx[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    for (int c = cb; c < ce; c += 16) {
+                        uint32_t v[16];
+                        tc::tmem_ld16_nowait(ta + (uint32_t)c, v);
+                        tc::tmem_wait_ld();
+                        relu_dot16(v, w_s + c, sx);
+                    }
+                    out[x] = (sx[0].x + sx[1].x) + (sx[0].y + sx[1].y);
                 }
             }
             tc::fence_before_sync();
@@ -466,8 +571,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             if (valid) {
 #pragma unroll
                 for (int x = 0; x < 4; x++)
-                    if (x < nq && sk < nv_s[x])
-                        lg[(int64_t)(t0 + x) * a.logits_stride + sk] = out[x] * kscale;
+                    if (x < qh && x_lo + x < nq && sk < nv_s[x_lo + x])
+                        lg[(int64_t)(t0 + x_lo + x) * a.logits_stride + sk] = out[x] * kscale;
             }
         }
         tc::cp_async_wait<0>();     // no copy into the ring outlives the loop
@@ -479,6 +584,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         __syncwarp();
         tc::tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
     }
+    if constexpr (EG == 2) {    // the fused plans use two epilogue groups
     if (sel.cand_key == nullptr || *abort_flag) return;
     // ---- fused top-512 of this CTA's chunk, per query row of the group: the
     // logits just written (visible to the block after the barrier above, and
@@ -498,6 +604,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         select_chunk<kTcThreads>(skeys, len, k0, sel.cand_key + c * kTopK, sel.cand_idx + c * kTopK,
                                  sel.chunk_info + c, tsh, a.status);
         __syncthreads();
+    }
     }
 }
 
@@ -539,13 +646,13 @@ static bool make_key_map(CUtensorMap *m, const void *codes, int64_t num_slots, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p) {
+static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p, int eg) {
     const size_t ks = rb / 32;
     return 1024 + (size_t)p.stages * kTcTile * rb + (((size_t)p.n * rb + 1023) & ~(size_t)1023) +
            (fp4 ? (p.stages + 1) * ks * 512 + (rb == 32 ? (size_t)kSfSlots * 16 * rb : 0) : 0) +
            256 * 4 + 16 * 4 +
            (2 * p.stages + 2 * p.nacc + 1) * 8 + 32 +
-           (size_t)2 * p.tiles_per_cta * 4 + 16 + (size_t)2 * kKsRing * kTcTile * 4;
+           (size_t)2 * p.tiles_per_cta * 4 + 16 + (size_t)eg * kKsRing * kTcTile * 4;
 }
 
 bool indexer_tc_supported(const IndexerArgs &a) {
@@ -567,6 +674,7 @@ bool indexer_tc_supported(const IndexerArgs &a) {
 struct TcPlan {
     TcParams p;
     int rb, chunks;
+    int eg;            // epilogue groups: 4 where 256-column accumulators split by query rows
     size_t smem;
 };
 
@@ -578,12 +686,18 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     pl.rb = rb;
     p.hi_pad = (a.heads + 15) / 16 * 16;
     // queries of one request share the key tiles: group up to 4 of them
-    // (N <= 128) when requests carry several query rows
-    p.qg = a.num_q <= a.bs ? 1 : 128 / p.hi_pad;
+    // (N <= 128) when requests carry several query rows, N <= 256 when they
+    // carry many (a prefill chunk: each key tile read from L2 then feeds
+    // twice the MMA work; the two accumulators fill TMEM, one CTA per SM)
+    const int n_max = (!fuse && !fp4 && a.num_q >= 8 * a.bs) ? 256 : 128;
+    p.qg = a.num_q <= a.bs ? 1 : n_max / p.hi_pad;
     if (p.qg < 1) p.qg = 1;
     if (p.qg > 4) p.qg = 4;
     if (fp4 && p.qg * p.hi_pad > 64) p.qg = p.hi_pad >= 64 ? 1 : 64 / p.hi_pad;
     p.n = p.qg * p.hi_pad;
+    // four epilogue groups (two per accumulator, each reducing half of the
+    // query rows) for the wide accumulators
+    pl.eg = (p.n > 128 && p.qg % 2 == 0) ? 4 : 2;
     // as many accumulators in flight (up to 8) as keep the CTA within 256 TMEM
     // columns (two CTAs per SM): the MMA of tile i waits for the epilogue of
     // tile i - nacc, so a deeper ring hides the hand-off latency of small tiles
@@ -597,8 +711,9 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     p.num_pages = (int)(a.num_slots / kC4Page);
     // 64-80 KB of key tiles in flight per CTA, two CTAs per SM
     p.stages = rb == 256 ? 3 : rb == 128 ? 5 : rb == 64 ? 8 : 16;
+    if (p.tmem_cols > 256) p.stages = p.n * rb > 16384 ? 2 * p.stages - 1 : 2 * p.stages;  // one CTA per SM
     const int tiles_max = (a.max_c4_len + kTcTile - 1) / kTcTile;
-    const int groups = (a.num_q + p.qg - 1) / p.qg;
+    const int groups = query_groups_bound(a.num_q, a.bs, p.qg);
     // one wave: at most (SMs x resident CTAs per SM) CTAs, split evenly over
     // the query groups (a second, nearly empty wave would double the time)
     int sms = 148;
@@ -609,7 +724,7 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     }
     p.tiles_per_cta = fuse ? 64 : tiles_max;          // upper bound for the estimate
     // 228 KB of shared memory per SM, 1 KB of it reserved per resident CTA
-    const size_t smem_est = tc_smem_bytes(rb, fp4, p) + 1024;
+    const size_t smem_est = tc_smem_bytes(rb, fp4, p, pl.eg) + 1024;
     int by_smem = (int)((228 * 1024) / smem_est);
     int ctas_per_sm = 512 / cols;
     if (by_smem < ctas_per_sm) ctas_per_sm = by_smem;
@@ -633,7 +748,7 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     }
     pl.chunks = (tiles_max + p.tiles_per_cta - 1) / p.tiles_per_cta;
     if (pl.chunks < 1) pl.chunks = 1;
-    pl.smem = tc_smem_bytes(rb, fp4, p);
+    pl.smem = tc_smem_bytes(rb, fp4, p, pl.eg);
     return pl;
 }
 
@@ -652,23 +767,29 @@ static cudaError_t launch_tc_plan(const IndexerArgs &a, const TcPlan &pl, const 
     if (!make_key_map(&map, a.k_codes, a.num_slots, pl.rb)) return cudaErrorInvalidValue;
     const TcParams p = pl.p;
     const size_t smem = pl.smem;
-    dim3 grid(pl.chunks, a.num_q);
+    dim3 grid(pl.chunks, query_groups_bound(a.num_q, a.bs, p.qg));
     const bool fp4 = a.fmt == CSA_FMT_FP4;
     const int rb = pl.rb;
-#define CSA_TC(F, R)                                                                        \
+#define CSA_TC_EG(F, R, E)                                                                  \
     do {                                                                                    \
         static int done[64] = {0};                                                          \
-        cudaError_t e = ensure_max_smem((const void *)indexer_tc_kernel<F, R>, 200 * 1024, done); \
+        cudaError_t e = ensure_max_smem((const void *)indexer_tc_kernel<F, R, E>, 227 * 1024, done); \
         if (e != cudaSuccess) return e;                                                     \
-        launch_k(indexer_tc_kernel<F, R>, grid, kTcThreads, smem, s, a, map, p, sel);       \
+        launch_k(indexer_tc_kernel<F, R, E>, grid, tc_threads<E>(), smem, s, a, map, p, sel); \
+    } while (0)
+#define CSA_TC(F, R)                                                                        \
+    do {                                                                                    \
+        if (pl.eg == 4) CSA_TC_EG(F, R, 4);                                                 \
+        else CSA_TC_EG(F, R, 2);                                                            \
     } while (0)
     if (a.fmt == CSA_FMT_FP8 && rb == 128) CSA_TC(CSA_FMT_FP8, 128);
     else if (a.fmt == CSA_FMT_FP8) CSA_TC(CSA_FMT_FP8, 64);
-    else if (fp4 && rb == 64) CSA_TC(CSA_FMT_FP4, 64);
-    else if (fp4) CSA_TC(CSA_FMT_FP4, 32);
+    else if (fp4 && rb == 64) CSA_TC_EG(CSA_FMT_FP4, 64, 2);
+    else if (fp4) CSA_TC_EG(CSA_FMT_FP4, 32, 2);
     else if (rb == 128) CSA_TC(CSA_FMT_BF16, 128);
     else CSA_TC(CSA_FMT_BF16, 256);
 #undef CSA_TC
+#undef CSA_TC_EG
     return cudaGetLastError();
 }
 

@@ -304,6 +304,51 @@ def test_full_size_ragged():
     _full_ragged_check("ragged", sample_q=[0, 1, 2, 40, last - 5, last - 1])
 
 
+def test_full_size_prefill_indexer_shared_codes():
+    """The indexer in the prefill launch shape (one request, 4096 causal query
+    rows seeing 65536-66560 keys, query rows grouped four to a tile column
+    block) on keys and queries quantised by the oracle: sampled rows against
+    the oracle's logits at 1e-2 relative, covering every row position inside a
+    query group and both ends of the chunk."""
+    from compressed_sparse_attention_12_b200 import csa, synth
+    w = synth.workload("prefill")
+    assert w.bs == 1
+    pt = synth.page_table(w)
+    rng = np.random.default_rng(29)
+    n = int(w.c4_lens[0])
+    nq, Hi, Di = int(w.num_q), w.idx_heads, w.idx_dim
+    keys = rng.standard_normal((n, Di))
+    kq = orc.index_quantise(keys, w.idx_fmt)
+    s = np.arange(n)
+    slots = pt[0, s // 64].astype(np.int64) * 64 + s % 64
+    n_slots = w.num_pages * 64
+    kc, kb, ks = index_arrays(kq, w.idx_fmt, Di, n_slots, slots)
+    qx = rng.standard_normal((nq, Hi, Di))
+    qq = orc.index_quantise(qx, w.idx_fmt)
+    qc, qb, qs = index_arrays(qq, w.idx_fmt, Di, nq * Hi)
+    ww = rng.uniform(size=(nq, Hi)).astype(np.float32)
+    wf = (ww * qq["scales"].reshape(nq, Hi)).astype(np.float32)
+    stride = (n + 15) // 16 * 16
+    logits = torch.full((nq, stride), float("nan"), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa.csa_indexer_logits(qc, qb, dev(wf), Hi, Di, csa.FMT[w.idx_fmt], kc, kb, ks, dev(pt),
+                           dev(w.c4_lens.astype(np.int32)), dev(w.cu_q), dev(w.q_pos), n, logits,
+                           status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    sample = [0, 1, 2, 3, 4, 5, 6, 7, 1029, 2046, 2047, 4092, 4093, 4094, 4095]
+    got = logits[sample].cpu().numpy()
+    kd = kq["deq"]
+    qd = qq["deq"].reshape(nq, Hi, Di)
+    for i, t in enumerate(sample):
+        nv = min(n, orc.n_visible(int(w.q_pos[t])))
+        assert 65536 <= nv <= n, (t, nv)
+        ref = orc.indexer_logits(qd[t:t + 1], ww[t:t + 1], kd[:nv], [nv])[0]
+        assert rel_close(got[i, :nv], ref, 1e-2).all(), t
+        # keys past the causal limit are not written
+        assert np.isnan(got[i, nv:]).all(), t
+
+
 def test_full_size_prefill_sampled():
     """The 4096-token prefill on a 262144-token context at full size in the
     benchmark's separate form (plain indexer, two-stage top-k over rows of
