@@ -32,6 +32,16 @@ constexpr int kBf16RowBytes = 1152;
 // this one depends on have completed and their writes are visible.  Nothing
 // global is read before the wait.  Both instructions are no-ops when the
 // kernel was launched without the programmatic-serialization attribute.
+// The two halves of pdl_begin, for kernels that read caller inputs (request
+// offsets, lengths, positions) before waiting on the preceding kernel.
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void pdl_begin() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");

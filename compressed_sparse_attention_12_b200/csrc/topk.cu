@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include <atomic>
+#include <cstdint>
 
 #include "topk.cuh"
 
@@ -367,33 +368,342 @@ topk_reg_kernel(const float *__restrict__ logits, int64_t stride, const int32_t 
     }
 }
 
+// ------------------------------------------------------------------ bound-first selection
+//
+// For a few long rows (decode batches): three launches spread over every SM
+// instead of one CTA per row.
+//   A (grid chunks x rows): the row's keys fall into G groups of g = 2^s
+//     consecutive keys (g the largest power of two with n/g >= 1024, so
+//     1024 <= G <= 2048 once n >= 1024; g = 1 below); each CTA writes the
+//     maxima of its chunk's groups.
+//   B (same grid): every CTA takes L, the lower edge of the radix bin that
+//     holds the K-th largest of the row's G group maxima (K = min(512, n);
+//     L = 0 when n <= K).  K groups hold a key >= L, so L is at most the
+//     row's K-th largest key: every key of the top K is >= L.  The CTA writes
+//     its chunk's keys >= L, in index order, to the chunk's own region of the
+//     row's candidate buffer and records how many there are.
+//   C (one CTA per row): gathers the chunk segments in chunk order (so in
+//     index order) into shared memory -- or, when they do not fit, into a
+//     second buffer in the workspace -- and selects the top K among them as
+//     the one-launch kernels do, with the page transform and -1 padding.
+// Each kernel looks up its row (caller inputs only) before it waits on the
+// preceding kernel.
+constexpr int kTbThreads = 512;
+constexpr int kTbChunk = 4096;         // keys per CTA in launches A and B
+constexpr int kTbMaxGroups = 2048;
+constexpr int kTbCap = 16384;          // candidates selected from shared memory in launch C
+constexpr int kTbMaxRows = 64;         // with more rows the per-row launches fill the GPU
+constexpr int kTbMinLen = 49152;       // shorter rows: one CTA per row (registers or shared memory)
+
+// log2 of the group size for a row of n keys
+__device__ __forceinline__ int tb_group_shift(int n) {
+    return n < 2048 ? 0 : 31 - __clz(n / 1024);
+}
+
+__global__ void __launch_bounds__(kTbThreads)
+topk_tb_groupmax_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens,
+                        int bs, const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
+                        int pt_stride, uint32_t *gmax, int32_t *status, int ratio) {
+    pdl_trigger();
+    __shared__ TkShared sh;
+    __shared__ uint32_t sgm[kTbChunk];
+    const int t = blockIdx.y, c = blockIdx.x;
+    const RowInfo ri = row_info<kTbThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride,
+                                            status, c == 0, sh, ratio);
+    const int n = ri.n_vis, lo = c * kTbChunk;
+    if (lo >= n) {
+        pdl_wait();
+        return;
+    }
+    const int len = min(kTbChunk, n - lo);
+    const int sh_g = tb_group_shift(n);
+    const int ngr = (len + (1 << sh_g) - 1) >> sh_g;      // kTbChunk is a multiple of the group size
+    for (int j = threadIdx.x; j < ngr; j += kTbThreads) sgm[j] = 0u;
+    __syncthreads();
+    pdl_wait();
+    const float *row = logits + (int64_t)t * stride + lo;
+    const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+    for (int base = 0; base < len; base += 4 * kTbThreads) {   // same trip count in every lane
+        const int i = base + 4 * (int)threadIdx.x;
+        uint32_t k[4];
+        if (vec && i + 4 <= len) {
+            const float4 x = *reinterpret_cast<const float4 *>(row + i);
+            k[0] = order_key(x.x, status);
+            k[1] = order_key(x.y, status);
+            k[2] = order_key(x.z, status);
+            k[3] = order_key(x.w, status);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; e++) k[e] = i + e < len ? order_key(row[i + e], status) : 0u;
+        }
+        if (sh_g >= 2) {
+            // the four keys share a group (absent ones, 0, are the smallest
+            // key); the g/4 lanes of one group combine first, aligned runs of
+            // lanes holding consecutive keys, and one of them updates the slot
+            uint32_t m = max(max(k[0], k[1]), max(k[2], k[3]));
+            const int lanes = min(1 << (sh_g - 2), 32);
+            for (int o = 1; o < lanes; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((threadIdx.x & (lanes - 1)) == 0 && i < len) atomicMax(&sgm[i >> sh_g], m);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                if (i + e < len) atomicMax(&sgm[(i + e) >> sh_g], k[e]);
+        }
+    }
+    __syncthreads();
+    uint32_t *g = gmax + (int64_t)t * kTbMaxGroups + (lo >> sh_g);
+    for (int j = threadIdx.x; j < ngr; j += kTbThreads) g[j] = sgm[j];
+}
+
+__global__ void __launch_bounds__(kTbThreads)
+topk_tb_gather_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens,
+                      int bs, const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
+                      int pt_stride, const uint32_t *gmax, uint32_t *counts, int mc,
+                      uint32_t *cand_key, int32_t *cand_idx, int64_t cs, int32_t *status,
+                      int ratio) {
+    pdl_trigger();
+    __shared__ TkShared sh;
+    __shared__ __align__(16) uint32_t skeys[kTbChunk];
+    __shared__ uint32_t sg[kTbMaxGroups];
+    const int t = blockIdx.y, c = blockIdx.x;
+    const RowInfo ri = row_info<kTbThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride,
+                                            status, false, sh, ratio);
+    pdl_wait();
+    const int n = ri.n_vis, lo = c * kTbChunk;
+    if (lo >= n) return;
+    const int len = min(kTbChunk, n - lo);
+    const int K = min(kTopK, n);
+    uint32_t L = 0;
+    if (n > K) {
+        const int sh_g = tb_group_shift(n);
+        const int G = (n + (1 << sh_g) - 1) >> sh_g;      // >= K (G = n below 2048 keys)
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+        for (int j = threadIdx.x; j < G; j += kTbThreads) {
+            const uint32_t v = gmax[(int64_t)t * kTbMaxGroups + j];
+            sg[j] = v;
+            kmin = min(kmin, v);
+            kmax = max(kmax, v);
+        }
+        block_minmax<kTbThreads>(kmin, kmax, sh);          // its barrier also publishes sg
+        // one radix pass: the lower edge of the bin holding the K-th largest
+        // maximum is below it, so still a bound of the row's K-th key
+        int need_eq;
+        radix_threshold<kTbThreads>(sg, G, K, kmin, kmax, sh, &L, &need_eq, true);
+    }
+    stage_row_keys<kTbThreads>(skeys, logits + (int64_t)t * stride + lo, len);
+    __syncthreads();
+    for (int i = threadIdx.x; i < len; i += kTbThreads)
+        skeys[i] = order_key(__uint_as_float(skeys[i]), status);
+    __syncthreads();
+    uint32_t *ok = cand_key + (int64_t)t * cs + lo;
+    int32_t *oi = cand_idx + (int64_t)t * cs + lo;
+    const int kept = ordered_compact<kTbThreads>(skeys, len, L, len, sh, [&](int pos, int i, uint32_t k) {
+        ok[pos] = k;
+        oi[pos] = lo + i;
+    });
+    if (threadIdx.x == 0) counts[(int64_t)t * mc + c] = (uint32_t)kept;
+}
+
+__global__ void __launch_bounds__(kTkRowThreads, 1)
+topk_tb_final_kernel(const int32_t *c4_lens, int bs, const int32_t *cu_q, const int32_t *q_pos,
+                     int max_c4_len, const int32_t *page_table, int pt_stride, int64_t num_slots,
+                     const uint32_t *counts, int mc, const uint32_t *cand_key,
+                     const int32_t *cand_idx, uint32_t *ord_key, int32_t *ord_idx, int64_t cs,
+                     int32_t *out_phys, int32_t *out_raw, int32_t *status, int ratio) {
+    pdl_trigger();
+    extern __shared__ __align__(16) uint8_t tbc_smem[];
+    TkRowShared &sh = *reinterpret_cast<TkRowShared *>(tbc_smem);
+    uint32_t *skeys = reinterpret_cast<uint32_t *>(tbc_smem + kTkRowKeysOffset);
+    int32_t *sidx = reinterpret_cast<int32_t *>(skeys + kTbCap);
+    __shared__ uint32_t c_pre[kTkRowThreads];
+    const int t = blockIdx.x;
+    const RowInfo ri = row_info<kTkRowThreads>(t, cu_q, bs, q_pos, c4_lens, max_c4_len,
+                                               pt_stride, status, false, sh, ratio);
+    pdl_wait();
+    const int n = ri.n_vis;
+    const int K = min(kTopK, n);
+    int32_t *op = out_phys + (int64_t)t * kTopK;
+    int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
+    if (n > 0) {
+        const int nch = (n + kTbChunk - 1) / kTbChunk;     // <= kTkRowThreads (host check)
+        const uint32_t cc = (int)threadIdx.x < nch ? counts[(int64_t)t * mc + threadIdx.x] : 0u;
+        uint32_t m;
+        const uint32_t pre = block_excl_scan<kTkRowThreads>(cc, &m, sh);
+        if ((int)threadIdx.x < nch) c_pre[threadIdx.x] = pre;
+        __syncthreads();
+        const bool in_smem = m <= (uint32_t)kTbCap;
+        uint32_t *dk = in_smem ? skeys : ord_key + (int64_t)t * cs;
+        int32_t *di = in_smem ? sidx : ord_idx + (int64_t)t * cs;
+        const uint32_t *sk = cand_key + (int64_t)t * cs;
+        const int32_t *si = cand_idx + (int64_t)t * cs;
+        // position p of the gathered list lies in the last chunk c with
+        // c_pre[c] <= p (a binary search over the chunk table), so all loads
+        // of a thread are independent
+        for (uint32_t p = threadIdx.x; p < m; p += kTkRowThreads) {
+            int lo_c = 0, hi_c = nch - 1;
+            while (lo_c < hi_c) {
+                const int mid = (lo_c + hi_c + 1) >> 1;
+                if (c_pre[mid] <= p) lo_c = mid; else hi_c = mid - 1;
+            }
+            const uint32_t src = (uint32_t)lo_c * kTbChunk + (p - c_pre[lo_c]);
+            dk[p] = sk[src];
+            di[p] = si[src];
+        }
+        __syncthreads();
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+        for (uint32_t i = threadIdx.x; i < m; i += kTkRowThreads) {
+            kmin = min(kmin, dk[i]);
+            kmax = max(kmax, dk[i]);
+        }
+        block_minmax<kTkRowThreads>(kmin, kmax, sh);
+        uint32_t T = 0;
+        int need_eq = (int)m;
+        if ((int)m > K) radix_threshold<kTkRowThreads>(dk, (int)m, K, kmin, kmax, sh, &T, &need_eq);
+        const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
+        ordered_compact<kTkRowThreads>(dk, (int)m, T, need_eq, sh, [&](int pos, int i, uint32_t) {
+            const int32_t s = di[i];
+            const int32_t page = pt_row[s / kC4Page];
+            const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
+            int32_t phys = (int32_t)slot;
+            if (page < 0 || slot >= num_slots) {
+                report(status, CSA_ERR_BOUNDS);
+                phys = -1;
+            }
+            op[pos] = phys;
+            if (orw) orw[pos] = s;
+        });
+    }
+    for (int p = max(K, 0) + threadIdx.x; p < kTopK; p += kTkRowThreads) {
+        op[p] = -1;
+        if (orw) orw[p] = -1;
+    }
+}
+
+// Workspace of the bound-first selection, per row: group maxima, one
+// candidate count per chunk, the candidates by chunk region (keys, indices)
+// and the gathered overflow copy.
+struct TbLayout {
+    int64_t cs;          // candidates per row (max_c4_len rounded up to 4)
+    int mc;              // chunks per row
+    size_t gmax, counts, ck, ci, ok2, oi2, bytes;
+};
+
+static size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+static TbLayout tb_layout(int num_q, int max_c4_len) {
+    TbLayout l;
+    l.cs = ((int64_t)max_c4_len + 3) & ~(int64_t)3;
+    l.mc = (max_c4_len + kTbChunk - 1) / kTbChunk;
+    const size_t q = (size_t)num_q;
+    l.gmax = 0;
+    l.counts = align16(l.gmax + q * kTbMaxGroups * 4);
+    l.ck = align16(l.counts + q * l.mc * 4);
+    l.ci = align16(l.ck + q * l.cs * 4);
+    l.ok2 = align16(l.ci + q * l.cs * 4);
+    l.oi2 = align16(l.ok2 + q * l.cs * 4);
+    l.bytes = align16(l.oi2 + q * l.cs * 4);
+    return l;
+}
+
+static size_t tb_bytes(int num_q, int max_c4_len) { return tb_layout(num_q, max_c4_len).bytes; }
+
+static bool tb_applies(int num_q, int max_c4_len) {
+    return num_q <= kTbMaxRows && max_c4_len > kTbMinLen &&
+           max_c4_len <= kTkRowThreads * kTbChunk;
+}
+
+static cudaError_t launch_topk_bound_first(const TopkArgs &a, cudaStream_t s) {
+    const TbLayout l = tb_layout(a.num_q, a.max_c4_len);
+    uint8_t *w = (uint8_t *)a.workspace;
+    uint32_t *gmax = (uint32_t *)(w + l.gmax);
+    uint32_t *counts = (uint32_t *)(w + l.counts);
+    uint32_t *ck = (uint32_t *)(w + l.ck);
+    int32_t *ci = (int32_t *)(w + l.ci);
+    uint32_t *ok2 = (uint32_t *)(w + l.ok2);
+    int32_t *oi2 = (int32_t *)(w + l.oi2);
+    dim3 g(l.mc, a.num_q);
+    launch_k(topk_tb_groupmax_kernel, g, kTbThreads, 0, s, a.logits, a.logits_stride,
+             a.c4_seq_lens, a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.pt_stride, gmax, a.status,
+             a.ratio);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    launch_k(topk_tb_gather_kernel, g, kTbThreads, 0, s, a.logits, a.logits_stride,
+             a.c4_seq_lens, a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.pt_stride,
+             (const uint32_t *)gmax, counts, l.mc, ck, ci, l.cs, a.status, a.ratio);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t smem = kTkRowKeysOffset + (size_t)kTbCap * 8;
+    static int done[64] = {0};
+    e = ensure_max_smem((const void *)topk_tb_final_kernel, (int)smem, done);
+    if (e != cudaSuccess) return e;
+    launch_k(topk_tb_final_kernel, a.num_q, kTkRowThreads, smem, s, a.c4_seq_lens, a.bs, a.cu_q,
+             a.q_pos, a.max_c4_len, a.page_table, a.pt_stride, a.num_slots,
+             (const uint32_t *)counts, l.mc, (const uint32_t *)ck, (const int32_t *)ci, ok2, oi2,
+             l.cs, a.out_phys, a.out_raw, a.status, a.ratio);
+    return cudaGetLastError();
+}
+
 static int topk_max_chunks(int max_c4_len) {
     return max_c4_len <= 0 ? 1 : (max_c4_len + kTkChunk - 1) / kTkChunk;
 }
 
-// Workspace: candidate keys, candidate indices (num_q x chunks x 512 each),
-// then one (512th key, largest key) pair per chunk.
-size_t topk_workspace_bytes(int num_q, int max_c4_len) {
+// Workspace of the two-stage selection: candidate keys, candidate indices
+// (num_q x chunks x 512 each), then one (512th key, largest key) pair per chunk.
+static size_t two_stage_bytes(int num_q, int max_c4_len) {
     const size_t chunks = (size_t)num_q * topk_max_chunks(max_c4_len);
     return chunks * kTopK * 8 + chunks * sizeof(uint2);
 }
 
-// Scratch the selection actually uses: none for rows of at most kTkRowMax
-// logits (one launch, the row in registers or shared memory), the two-stage
-// candidate buffer for longer rows.
-size_t topk_scratch_bytes(int num_q, int max_c4_len) {
-    return max_c4_len <= kTkRowMax ? 0 : topk_workspace_bytes(num_q, max_c4_len);
+// Which selection runs for these sizes: the bound-first launches for a few
+// long rows (when their workspace fits `limit`), else one CTA per row for rows
+// of at most kTkRowMax keys, else the two-stage merge.
+enum TopkKind { kTopkReg, kTopkRow, kTopkBound, kTopkTwoStage };
+
+static TopkKind topk_kind(int num_q, int max_c4_len, size_t limit) {
+    if (tb_applies(num_q, max_c4_len) && tb_bytes(num_q, max_c4_len) <= limit) return kTopkBound;
+    if (max_c4_len <= kTkRegMax) return kTopkReg;
+    if (max_c4_len <= kTkRowMax) return kTopkRow;
+    return kTopkTwoStage;
 }
 
+// Workspace that covers every path launch_topk512 may take for these sizes.
+size_t topk_workspace_bytes(int num_q, int max_c4_len) {
+    size_t b = two_stage_bytes(num_q, max_c4_len);
+    if (topk_kind(num_q, max_c4_len, SIZE_MAX) == kTopkBound) {
+        const size_t tb = tb_bytes(num_q, max_c4_len);
+        if (tb > b) b = tb;
+    }
+    return b;
+}
+
+// Scratch the selection uses when it must fit CSA_TOPK_NOALLOC_MAX_BYTES:
+// the bound-first buffers where they fit, none for rows of at most kTkRowMax
+// logits otherwise (one launch), the two-stage candidate buffer for longer rows.
+size_t topk_scratch_bytes(int num_q, int max_c4_len) {
+    switch (topk_kind(num_q, max_c4_len, (size_t)CSA_TOPK_NOALLOC_MAX_BYTES)) {
+    case kTopkBound: return tb_bytes(num_q, max_c4_len);
+    case kTopkTwoStage: return two_stage_bytes(num_q, max_c4_len);
+    default: return 0;
+    }
+}
+
+static cudaError_t launch_topk512_limited(const TopkArgs &a, cudaStream_t s, size_t limit);
+
 cudaError_t launch_topk512(const TopkArgs &a, cudaStream_t s) {
+    return launch_topk512_limited(a, s, SIZE_MAX);
+}
+
+static cudaError_t launch_topk512_limited(const TopkArgs &a, cudaStream_t s, size_t limit) {
     if (a.num_q == 0) return cudaSuccess;
-    if (a.max_c4_len <= kTkRegMax) {
+    const TopkKind kind = topk_kind(a.num_q, a.max_c4_len, limit);
+    if (kind == kTopkBound) return launch_topk_bound_first(a, s);
+    if (kind == kTopkReg) {
         launch_k(topk_reg_kernel, a.num_q, kTkRowThreads, 0, s, a.logits, a.logits_stride,
                  a.c4_seq_lens, a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.page_table, a.pt_stride,
                  a.num_slots, a.out_phys, a.out_raw, a.status, a.ratio);
         return cudaGetLastError();
     }
-    if (a.max_c4_len <= kTkRowMax) {
+    if (kind == kTopkRow) {
         const size_t smem = kTkRowKeysOffset + (size_t)((a.max_c4_len + 3) & ~3) * 4;
         static int done_row[64] = {0};
         cudaError_t e = ensure_max_smem((const void *)topk_row_kernel,
@@ -461,7 +771,7 @@ cudaError_t launch_topk512_noalloc(const TopkArgs &a, cudaStream_t s) {
     }
     TopkArgs b = a;
     b.workspace = ptr;
-    return launch_topk512(b, s);
+    return launch_topk512_limited(b, s, (size_t)CSA_TOPK_NOALLOC_MAX_BYTES);
 }
 
 }  // namespace csa

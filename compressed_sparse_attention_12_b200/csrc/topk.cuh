@@ -92,15 +92,18 @@ __device__ __forceinline__ void block_minmax(uint32_t &lo, uint32_t &hi, TkShare
 // and exponent (the usual case for one row of logits) already spread over the
 // bins of the first pass; two passes resolve a range of up to 24 bits.  keys may
 // point to shared or global memory.
+// With one_pass the result is only the lower edge of the top digit's bin: a
+// lower bound of the K-th largest key.
 template <int NT>
 __device__ void radix_threshold(const uint32_t *keys, int n, int K, uint32_t kmin, uint32_t kmax,
-                                TkSharedT<NT> &sh, uint32_t *T_out, int *need_eq_out) {
+                                TkSharedT<NT> &sh, uint32_t *T_out, int *need_eq_out,
+                                bool one_pass = false) {
     const uint32_t range = kmax - kmin;
     const int B = range == 0 ? 0 : 32 - __clz(range);
     uint32_t prefix = 0;            // resolved high bits of d
     int remaining = K;
 #pragma unroll 1
-    for (int done = 0; done < B;) {
+    for (int done = 0; done < B && !(one_pass && done > 0);) {
         const int width = min(12, B - done);
         const int shift = B - done - width;
         const int hi = shift + width;            // bits at and above hi are resolved

@@ -217,6 +217,14 @@ csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scal
  *   workspace      >= csa_topk512_workspace_size(num_q, max_c4_len) bytes
  *                  (always checked; written only when max_c4_len > 49152, the
  *                  rows shorter than that being selected in one launch)
+ * Rows longer than 49152 keys are selected in several launches: with at most
+ * 64 rows, a bound-first selection spread over every SM (the maxima of about
+ * 1024-2048 groups of consecutive keys give a lower bound of the 512th key,
+ * only the keys above it are kept, then one CTA per row selects among them);
+ * with more rows, a per-chunk top-512 and a per-row merge.  The kernels of
+ * this step read cu_q, q_pos and c4_seq_lens before waiting for the kernels
+ * enqueued before them: the ordering rule of csa_sparse_mqa_decode applies to
+ * those three inputs.
  */
 size_t csa_topk512_workspace_size(int32_t num_q, int32_t max_c4_len);
 csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stride,
@@ -245,8 +253,9 @@ csa_status_t csa_topk512_page_transform(const float *logits, int64_t logits_stri
  * on a device, do not call this entry point again in the same process (load
  * the library in a fresh process).  Rows of at most 49152 compressed keys are
  * selected in one launch that needs no scratch, so any number of them is
- * accepted; for longer rows calls return CSA_ERR_WORKSPACE without launching
- * when csa_topk512_workspace_size(num_q, max_c4_len) exceeds the maximum.
+ * accepted; longer rows use the bound-first selection when its buffers fit
+ * the array, else the per-chunk selection and merge, and calls return
+ * CSA_ERR_WORKSPACE without launching when that one does not fit either.
  * Every call shares the one array (its contents persist between calls and
  * nothing in it needs to start at zero), so calls that overlap on the GPU --
  * on different streams, or from several threads -- race and must be ordered

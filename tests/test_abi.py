@@ -52,7 +52,12 @@ def test_workspace_sizes(L):
     # (512th key, largest key) pair
     assert csa.csa_topk512_workspace_size(3, 8192) == 3 * 1 * (512 * 8 + 8)
     assert csa.csa_topk512_workspace_size(3, 8193) == 3 * 2 * (512 * 8 + 8)
-    assert csa.csa_topk512_workspace_size(8, 262144) == 8 * 32 * (512 * 8 + 8)
+    # up to 64 rows longer than 49152 logits take the bound-first selection:
+    # per row 2048 group maxima, one count per 4096-logit chunk, and two
+    # (key, index) buffers as long as the row
+    assert csa.csa_topk512_workspace_size(8, 262144) == (8 * 2048 * 4 + 8 * 64 * 4 +
+                                                         4 * 8 * 262144 * 4)
+    assert csa.csa_topk512_workspace_size(65, 262144) == 65 * 32 * (512 * 8 + 8)
     assert csa.csa_sparse_mqa_workspace_size(4096, 64, 128, 0) == 0
     assert csa.csa_sparse_mqa_workspace_size(32, 64, 128, 1) > 0
 
