@@ -57,6 +57,15 @@ def parse():
     p.add_argument("--profile", action="store_true",
                    help="profiling run: no CPU baseline or end-to-end leg; the drawn float "
                         "inputs are freed once the caches are built")
+    p.add_argument("--scale", type=float, default=1.0,
+                   help="shrink the workload's context lengths by this factor (small cases "
+                        "for profiler captures; the benchmark line is taken at 1)")
+    p.add_argument("--traffic-record", metavar="CSV",
+                   help="write profiles/indexer_tc_<workload>.json from an ncu CSV log of "
+                        "dram__bytes_read.sum and dram__bytes_write.sum for indexer_tc_kernel "
+                        "launches of this workload, then exit")
+    p.add_argument("--traffic-command", default="",
+                   help="the command line that produced --traffic-record's log (stored with it)")
     return p.parse_args()
 
 
@@ -89,6 +98,47 @@ def profiled_traffic(w):
     return int(rec["traffic_bytes_per_launch"])
 
 
+_BYTE_UNITS = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6,
+               "GB": 1e9, "B": 1}
+
+
+def write_traffic_record(csv_path, workload, command):
+    """profiles/indexer_tc_<workload>.json: mean DRAM bytes (read + write) per
+    indexer_tc_kernel launch in an ncu CSV log, with the indexer sources' hash."""
+    import csv
+    per = {}
+    with open(csv_path) as fh:
+        rows = [r for r in csv.reader(fh)]
+    head = None
+    for r in rows:
+        if "Metric Name" in r and "Kernel Name" in r:
+            head = r
+            continue
+        if head is None or len(r) != len(head):
+            continue
+        d = dict(zip(head, r))
+        if "indexer_tc_kernel" not in d["Kernel Name"]:
+            continue
+        name = d["Metric Name"]
+        if name not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        v = float(d["Metric Value"].replace(",", "")) * _BYTE_UNITS[d.get("Metric Unit", "byte")]
+        per.setdefault(d["ID"], {})[name] = v
+    launches = [x for x in per.values() if len(x) == 2]
+    if not launches:
+        raise SystemExit(f"no indexer_tc_kernel launch with both DRAM metrics in {csv_path}")
+    traffic = sum(x["dram__bytes_read.sum"] + x["dram__bytes_write.sum"] for x in launches)
+    rec = {"kernel": "indexer_tc_kernel", "workload": workload,
+           "traffic_bytes_per_launch": int(round(traffic / len(launches))),
+           "launches": len(launches), "source_sha256": indexer_source_hash(),
+           "command": command}
+    out = os.path.join(ROOT, "profiles", f"indexer_tc_{workload.replace('_', '')}.json")
+    with open(out, "w") as fh:
+        json.dump(rec, fh, indent=1)
+        fh.write("\n")
+    print(out, rec["traffic_bytes_per_launch"])
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -99,7 +149,8 @@ def peaks():
 
 
 def workload_config(w):
-    return {"workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
+    extra = {} if SCALE == 1.0 else {"scale": SCALE}
+    return {**extra, "workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
             "c4_seq_len": int(w.c4_lens.max()), "query_tokens": w.num_q,
             "indexer": f"{w.idx_fmt} {w.idx_heads}x{w.idx_dim}", "heads": w.heads,
             "kv": w.kv_fmt, "window": w.window, "topk": w.topk, "page_size": 256,
@@ -243,11 +294,14 @@ class Clocks:
                 "samples": len(sm)}
 
 
+SCALE = 1.0         # --scale
+
+
 def rank_workload(name, rank):
     """Each rank times its own batch: same shapes, seed offset by the rank
     (requests are independent, so the path shards with no data exchange)."""
     from compressed_sparse_attention_12_b200 import synth
-    w = synth.workload(name)
+    w = synth.workload(name, SCALE)
     w.seed += 1000 * rank
     return w
 
@@ -480,7 +534,8 @@ def run_reference(args):
 def hca_workload_config(w):
     from compressed_sparse_attention_12_b200 import synth
     new = synth.hca_plan(w)[1]
-    return {"workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
+    extra = {} if SCALE == 1.0 else {"scale": SCALE}
+    return {**extra, "workload": w.name, "batch": w.bs, "raw_seq_len": int(w.seq_lens.max()),
             "hca_seq_len": int((w.seq_lens // 128).max()), "query_tokens": w.num_q,
             "heads": w.heads, "kv": w.kv_fmt, "window": w.window, "ratio": 128,
             "page_size": 256, "compressed_rows_this_step": int(new.sum() // 128),
@@ -871,6 +926,11 @@ def extra_line(o):
 
 def main():
     args = parse()
+    if args.traffic_record:
+        write_traffic_record(args.traffic_record, args.workload, args.traffic_command)
+        return
+    global SCALE
+    SCALE = args.scale
     if args.impl == "reference":
         run_reference(args)
         return
