@@ -18,14 +18,24 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 CSA_OK, CSA_ERR_INVALID, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA = 0, 1, 2, 3
 CSA_ERR_TIMEOUT, CSA_ERR_BOUNDS, CSA_ERR_NAN, CSA_ERR_WORKSPACE = 4, 5, 6, 7
-CSA_FMT_BF16, CSA_FMT_FP8, CSA_FMT_FP4, CSA_FMT_F32 = 0, 1, 2, 3
+CSA_FMT_BF16, CSA_FMT_FP8, CSA_FMT_FP4, CSA_FMT_F32, CSA_FMT_FP4_PAGE = 0, 1, 2, 3, 4
 CSA_OUT_KV_BF16, CSA_OUT_KV_FP8 = 0, 1
-CSA_OUT_INDEX_BF16, CSA_OUT_INDEX_FP8, CSA_OUT_INDEX_FP4 = 2, 3, 4
+CSA_OUT_INDEX_BF16, CSA_OUT_INDEX_FP8, CSA_OUT_INDEX_FP4, CSA_OUT_INDEX_FP4_PAGE = 2, 3, 4, 5
 TOPK, PAGE_SIZE, C4_PAGE_SIZE, KV_DIM, KV_LATENT = 512, 256, 64, 576, 512
 TOPK_NOALLOC_MAX_BYTES = 16 << 20
 HCA_RATIO, HCA_PAGE_SIZE, HCA_MAX_ROWS = 128, 2, 16 * 48 * 32
 
-FMT = {"bf16": CSA_FMT_BF16, "fp8": CSA_FMT_FP8, "fp4": CSA_FMT_FP4}
+FMT = {"bf16": CSA_FMT_BF16, "fp8": CSA_FMT_FP8, "fp4": CSA_FMT_FP4, "fp4p": CSA_FMT_FP4_PAGE}
+
+
+def index_record_bytes(dim: int) -> int:
+    """Bytes of one CSA_FMT_FP4_PAGE record (the 64 keys of one page)."""
+    return 36 * dim + 256
+
+
+def _slots(fmt, codes):
+    """Index slots held by a key array: one per row, 64 per paged FP4 record."""
+    return codes.shape[0] * C4_PAGE_SIZE if fmt == CSA_FMT_FP4_PAGE else codes.shape[0]
 
 
 class CsaError(RuntimeError):
@@ -158,7 +168,8 @@ def csa_c4_compress(x, gate, bias, cu_x, start_pos, max_rows_per_req, page_table
         _ptr(x), _ptr(gate), _ptr(bias), x.shape[1], bs, _ptr(cu_x), x.shape[0], _ptr(start_pos),
         int(max_rows_per_req), _ptr(page_table), page_table.shape[1], out_kind, _ptr(out),
         _ptr(out_block_scales), _ptr(out_scales),
-        out.shape[0] if num_slots is None else int(num_slots), _ptr(status), _stream(stream)))
+        _slots(CSA_FMT_FP4_PAGE if out_kind == CSA_OUT_INDEX_FP4_PAGE else -1, out)
+        if num_slots is None else int(num_slots), _ptr(status), _stream(stream)))
 
 
 def csa_hadamard_quant(x, fmt, codes, block_scales=None, scales=None, row_map=None,
@@ -166,7 +177,7 @@ def csa_hadamard_quant(x, fmt, codes, block_scales=None, scales=None, row_map=No
     dim = x.shape[-1]
     rows = x.numel() // dim
     x_dtype = CSA_FMT_BF16 if x.dtype == torch.bfloat16 else CSA_FMT_F32
-    n_out = codes.shape[0] if row_map is not None else rows
+    n_out = _slots(fmt, codes) if row_map is not None else rows
     _check("csa_hadamard_quant", lib().csa_hadamard_quant(
         _ptr(x), x_dtype, rows, dim, fmt, _ptr(row_map), n_out, _ptr(codes), _ptr(block_scales),
         _ptr(scales), _ptr(w_in), _ptr(w_out), _ptr(status), _stream(stream)))
@@ -178,7 +189,7 @@ def csa_index_quant(x, fmt, codes, block_scales=None, scales=None, row_map=None,
     dim = x.shape[-1]
     rows = x.numel() // dim
     x_dtype = CSA_FMT_BF16 if x.dtype == torch.bfloat16 else CSA_FMT_F32
-    n_out = codes.shape[0] if row_map is not None else rows
+    n_out = _slots(fmt, codes) if row_map is not None else rows
     _check("csa_index_quant", lib().csa_index_quant(
         _ptr(x), x_dtype, rows, dim, fmt, _ptr(row_map), n_out, _ptr(codes), _ptr(block_scales),
         _ptr(scales), _ptr(w_in), _ptr(w_out), _ptr(status), _stream(stream)))
@@ -192,7 +203,7 @@ def csa_rope_hadamard_quant(x, freqs_cis, rope_dim, positions, rows_per_pos, fmt
     dim = x.shape[-1]
     rows = x.numel() // dim
     x_dtype = CSA_FMT_BF16 if x.dtype == torch.bfloat16 else CSA_FMT_F32
-    n_out = codes.shape[0] if row_map is not None else rows
+    n_out = _slots(fmt, codes) if row_map is not None else rows
     _check("csa_rope_hadamard_quant", lib().csa_rope_hadamard_quant(
         _ptr(x), x_dtype, rows, dim, _ptr(freqs_cis), int(rope_dim), freqs_cis.shape[0],
         _ptr(positions), int(rows_per_pos), fmt, _ptr(row_map), n_out, _ptr(codes),
@@ -210,7 +221,8 @@ def csa_c4_compress_index_rope(x, gate, bias, cu_x, start_pos, max_rows_per_req,
         _ptr(x), _ptr(gate), _ptr(bias), x.shape[1], bs, _ptr(cu_x), x.shape[0], _ptr(start_pos),
         int(max_rows_per_req), _ptr(page_table), page_table.shape[1], out_kind, _ptr(freqs_cis),
         int(rope_dim), freqs_cis.shape[0], _ptr(out), _ptr(out_block_scales), _ptr(out_scales),
-        out.shape[0] if num_slots is None else int(num_slots), _ptr(status), _stream(stream)))
+        _slots(CSA_FMT_FP4_PAGE if out_kind == CSA_OUT_INDEX_FP4_PAGE else -1, out)
+        if num_slots is None else int(num_slots), _ptr(status), _stream(stream)))
 
 
 def csa_dsa_indexer_logits(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, fmt, k_codes,
@@ -221,7 +233,7 @@ def csa_dsa_indexer_logits(q_codes, q_block_scales, q_weights, idx_heads, idx_di
     _check("csa_dsa_indexer_logits", lib().csa_dsa_indexer_logits(
         _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
         _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
-        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        _slots(fmt, k_codes) if num_slots is None else int(num_slots), _ptr(page_table),
         page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos),
         int(max_seq_len), _ptr(logits), logits.shape[1], _ptr(status), _stream(stream)))
 
@@ -248,7 +260,7 @@ def csa_indexer_logits(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, f
     _check("csa_indexer_logits", lib().csa_indexer_logits(
         _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
         _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
-        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        _slots(fmt, k_codes) if num_slots is None else int(num_slots), _ptr(page_table),
         page_table.shape[1], _ptr(c4_seq_lens), c4_seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos),
         int(max_c4_len), _ptr(logits), logits.shape[1], _ptr(status), _stream(stream)))
 
@@ -301,7 +313,7 @@ def csa_indexer_topk512(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, 
     _check("csa_indexer_topk512", lib().csa_indexer_topk512(
         _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
         _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
-        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        _slots(fmt, k_codes) if num_slots is None else int(num_slots), _ptr(page_table),
         page_table.shape[1], _ptr(c4_seq_lens), bs, _ptr(cu_q), _ptr(q_pos), int(max_c4_len),
         int(c4_page_size), _ptr(logits), logits.shape[1], _ptr(out_indices), _ptr(raw_indices),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)))
@@ -315,7 +327,7 @@ def csa_indexer_select(q_codes, q_block_scales, q_weights, idx_heads, idx_dim, f
     _check("csa_indexer_select", lib().csa_indexer_select(
         _ptr(q_codes), _ptr(q_block_scales), _ptr(q_weights), num_q, idx_heads, idx_dim, fmt,
         _ptr(k_codes), _ptr(k_block_scales), _ptr(k_scales),
-        k_codes.shape[0] if num_slots is None else int(num_slots), _ptr(page_table),
+        _slots(fmt, k_codes) if num_slots is None else int(num_slots), _ptr(page_table),
         page_table.shape[1], _ptr(c4_seq_lens), c4_seq_lens.shape[0], _ptr(cu_q), _ptr(q_pos),
         int(max_c4_len), _ptr(logits), logits.shape[1], _ptr(workspace), workspace.numel(),
         _ptr(status), _stream(stream)))

@@ -133,6 +133,22 @@ __device__ __forceinline__ float quant_index_row(const float (&v)[E], int lane, 
     for (int i = 0; i < E; i++)
         q[i] = dq > 0.0f ? __fdiv_rn(v[i], dq) : (signbit(v[i]) ? -0.0f : 0.0f);
     const uint32_t packed = f32x8_to_e2m1x8(q);
+    if (fmt == CSA_FMT_FP4_PAGE) {
+        // the slot's 8-key group inside its page's record: codes in 8-key x
+        // 16-byte blocks, then the group's block scales, then its row scales
+        constexpr int Gb = 4 * D + D / 2 + 32;
+        const int r = (int)(orow & 63), i = r & 7;
+        uint8_t *grp = codes + (orow >> 6) * (8 * Gb) + (r >> 3) * Gb;
+        const int b = lane * (E / 2);          // this lane's first code byte (E/2 bytes, one block)
+        uint8_t *o = grp + (b >> 4) * 128 + i * 16 + (b & 15);
+        if (E == 4)
+            *reinterpret_cast<uint16_t *>(o) = (uint16_t)(packed & 0xFFFF);
+        else
+            *o = (uint8_t)(packed & 0xFF);
+        if ((lane % (16 / E)) == 0) grp[4 * D + i * (D / 16) + lane / (16 / E)] = sb;
+        if (lane == 0) *reinterpret_cast<float *>(grp + 4 * D + D / 2 + 4 * i) = st;
+        return st;
+    }
     uint8_t *o = codes + orow * (D / 2) + lane * (E / 2);
     if (E == 4)
         *reinterpret_cast<uint16_t *>(o) = (uint16_t)(packed & 0xFFFF);
@@ -471,9 +487,10 @@ cudaError_t launch_c4_compress(const float *x, const float *gate, const float *b
                                                           max_rows, page_table, pt_stride, fmt,
                                                           (uint8_t *)out, num_slots, status);
     } else {
-        const int fmt = out_kind == CSA_OUT_INDEX_FP8   ? CSA_FMT_FP8
-                        : out_kind == CSA_OUT_INDEX_FP4 ? CSA_FMT_FP4
-                                                        : CSA_FMT_BF16;
+        const int fmt = out_kind == CSA_OUT_INDEX_FP8        ? CSA_FMT_FP8
+                        : out_kind == CSA_OUT_INDEX_FP4      ? CSA_FMT_FP4
+                        : out_kind == CSA_OUT_INDEX_FP4_PAGE ? CSA_FMT_FP4_PAGE
+                                                             : CSA_FMT_BF16;
         dim3 grid((max_blocks + 7) / 8, bs);
         if (dim == 64)
             launch_k(compress_index_kernel<2>, grid, 256, 0, s, 

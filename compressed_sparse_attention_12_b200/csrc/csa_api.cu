@@ -12,8 +12,18 @@ csa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
 bool index_fmt_ok(int32_t fmt) {
-    return fmt == CSA_FMT_BF16 || fmt == CSA_FMT_FP8 || fmt == CSA_FMT_FP4;
+    return fmt == CSA_FMT_BF16 || fmt == CSA_FMT_FP8 || fmt == CSA_FMT_FP4 ||
+           fmt == CSA_FMT_FP4_PAGE;
 }
+
+// Paged FP4 keys are read by bulk copies of whole 64-key page records.
+bool paged_keys_ok(int32_t fmt, const void *k_codes, int64_t num_slots) {
+    return fmt != CSA_FMT_FP4_PAGE ||
+           ((reinterpret_cast<uintptr_t>(k_codes) % 16) == 0 && num_slots % CSA_C4_PAGE_SIZE == 0);
+}
+
+// Formats whose queries carry FP4 block scales.
+bool fp4_query(int32_t fmt) { return fmt == CSA_FMT_FP4 || fmt == CSA_FMT_FP4_PAGE; }
 
 bool kv_fmt_ok(int32_t fmt) { return fmt == CSA_FMT_BF16 || fmt == CSA_FMT_FP8; }
 
@@ -23,7 +33,7 @@ bool index_arrays_ok(int32_t fmt, const void *codes, const void *block_scales,
     if (!codes) return false;
     if (fmt == CSA_FMT_FP8 && !scales) return false;
     if (fmt == CSA_FMT_FP4 && (!scales || !block_scales)) return false;
-    return true;
+    return true;       // CSA_FMT_FP4_PAGE: codes, block and row scales in one record array
 }
 
 }  // namespace
@@ -76,7 +86,7 @@ static csa_status_t c4_compress(const float *x, const float *gate, const float *
         return CSA_ERR_INVALID;
     const bool kv = out_kind == CSA_OUT_KV_BF16 || out_kind == CSA_OUT_KV_FP8;
     const bool idx = out_kind == CSA_OUT_INDEX_BF16 || out_kind == CSA_OUT_INDEX_FP8 ||
-                     out_kind == CSA_OUT_INDEX_FP4;
+                     out_kind == CSA_OUT_INDEX_FP4 || out_kind == CSA_OUT_INDEX_FP4_PAGE;
     if (!kv && !idx) return CSA_ERR_UNSUPPORTED;
     if (kv && dim != CSA_KV_DIM) return CSA_ERR_UNSUPPORTED;
     if (idx && dim != 64 && dim != 128) return CSA_ERR_UNSUPPORTED;
@@ -113,7 +123,7 @@ csa_status_t csa_c4_compress_index_rope(const float *x, const float *gate, const
                                         float *out_scales, int64_t num_slots, int32_t *status,
                                         void *stream) {
     if (out_kind != CSA_OUT_INDEX_BF16 && out_kind != CSA_OUT_INDEX_FP8 &&
-        out_kind != CSA_OUT_INDEX_FP4)
+        out_kind != CSA_OUT_INDEX_FP4 && out_kind != CSA_OUT_INDEX_FP4_PAGE)
         return CSA_ERR_UNSUPPORTED;
     if (!rope_ok(freqs_cis, rope_dim, max_pos, dim)) return CSA_ERR_INVALID;
     csa::RopeArgs rope;
@@ -214,8 +224,9 @@ static csa_status_t indexer_logits(const void *q_codes, const uint8_t *q_block_s
     if (num_q == 0 || max_c4_len == 0) return CSA_OK;
     if (bs < 1 || !q_codes || !q_weights || !page_table || !c4_seq_lens || !cu_q || !logits)
         return CSA_ERR_INVALID;
-    if (fmt == CSA_FMT_FP4 && !q_block_scales) return CSA_ERR_INVALID;
+    if (fp4_query(fmt) && !q_block_scales) return CSA_ERR_INVALID;
     if (!index_arrays_ok(fmt, k_codes, k_block_scales, k_scales)) return CSA_ERR_INVALID;
+    if (!paged_keys_ok(fmt, k_codes, num_slots)) return CSA_ERR_UNSUPPORTED;
     if (logits_stride < max_c4_len) return CSA_ERR_INVALID;
     if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
     csa::IndexerArgs a{q_codes, q_block_scales, q_weights, num_q, idx_heads, idx_dim, fmt,
@@ -359,8 +370,9 @@ csa_status_t csa_indexer_topk512(const void *q_codes, const uint8_t *q_block_sca
     cudaStream_t s = as_stream(stream);
     if (max_c4_len == 0) return cuda_status(csa::launch_topk512(t, s));   // -1 padding only
     if (!q_codes || !q_weights || !logits || logits_stride < max_c4_len) return CSA_ERR_INVALID;
-    if (fmt == CSA_FMT_FP4 && !q_block_scales) return CSA_ERR_INVALID;
+    if (fp4_query(fmt) && !q_block_scales) return CSA_ERR_INVALID;
     if (!index_arrays_ok(fmt, k_codes, k_block_scales, k_scales)) return CSA_ERR_INVALID;
+    if (!paged_keys_ok(fmt, k_codes, num_slots)) return CSA_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < csa_indexer_topk512_workspace_size(
                                             num_q, bs, idx_heads, idx_dim, fmt, max_c4_len))
         return CSA_ERR_WORKSPACE;
@@ -391,8 +403,9 @@ csa_status_t csa_indexer_select(const void *q_codes, const uint8_t *q_block_scal
     if (bs < 1 || !q_codes || !q_weights || !page_table || !c4_seq_lens || !cu_q || !logits ||
         logits_stride < max_c4_len)
         return CSA_ERR_INVALID;
-    if (fmt == CSA_FMT_FP4 && !q_block_scales) return CSA_ERR_INVALID;
+    if (fp4_query(fmt) && !q_block_scales) return CSA_ERR_INVALID;
     if (!index_arrays_ok(fmt, k_codes, k_block_scales, k_scales)) return CSA_ERR_INVALID;
+    if (!paged_keys_ok(fmt, k_codes, num_slots)) return CSA_ERR_UNSUPPORTED;
     if (num_q > 65535) return CSA_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < csa_indexer_topk512_workspace_size(
                                             num_q, bs, idx_heads, idx_dim, fmt, max_c4_len))

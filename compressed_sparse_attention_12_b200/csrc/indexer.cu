@@ -134,6 +134,7 @@ cudaError_t launch_indexer_tc(const IndexerArgs &a, cudaStream_t s);
 cudaError_t launch_indexer(const IndexerArgs &a, cudaStream_t s) {
     if (a.num_q == 0 || a.max_c4_len == 0) return cudaSuccess;
     if (indexer_tc_supported(a)) return launch_indexer_tc(a, s);
+    if (a.fmt == CSA_FMT_FP4_PAGE) return cudaErrorNotSupported;     // records: tensor-core path only
     dim3 grid((a.max_c4_len + kIdxThreads - 1) / kIdxThreads, a.num_q);
     const size_t smem = (size_t)a.heads * (a.dim + 1) * sizeof(float);
 #define CSA_IDX(F, D)                                                                    \

@@ -170,10 +170,17 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     // 1024-byte aligned carve-up: stages | q tile | w' | nv | barriers
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    constexpr bool kFp4 = FMT == CSA_FMT_FP4;
-    constexpr bool kSfStaged = kFp4 && RB == 32;
+    // paged FP4 keys: one record per 64-key page, 8 groups of 8 keys, each
+    // group's codes (8-key x 16-byte blocks), block scales and row scales
+    // side by side; a tile is two records copied whole
+    constexpr bool kPaged = FMT == CSA_FMT_FP4_PAGE;
+    constexpr bool kFp4 = FMT == CSA_FMT_FP4 || kPaged;
+    constexpr bool kSfStaged = kFp4 && RB == 32 && !kPaged;
+    constexpr int kGb = 9 * RB + 32;                     // bytes of an 8-key group (4.5 Di + 32)
+    constexpr int kRec = 8 * kGb;                        // bytes of a page record (36 Di + 256)
+    constexpr int kStage = kPaged ? 2 * kRec : G::kStageBytes;
     uint8_t *stage_buf = base;
-    uint8_t *q_buf = stage_buf + p.stages * G::kStageBytes;
+    uint8_t *q_buf = stage_buf + p.stages * kStage;
     uint8_t *sfa_buf = q_buf + ((p.n * RB + 1023) & ~1023);            // [stages][ksteps][512]
     uint8_t *sfb_buf = sfa_buf + (kFp4 ? p.stages * G::kKSteps * 512 : 0);  // [ksteps][512]
     uint8_t *sf_stage = sfb_buf + (kFp4 ? G::kKSteps * 512 : 0);    // [kSfSlots][16 * RB]
@@ -182,7 +189,8 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
     uint64_t *bars = reinterpret_cast<uint64_t *>(nv_s + 16);
     uint64_t *full = bars, *empty = bars + p.stages, *tfull = bars + 2 * p.stages;
     uint64_t *tempty = tfull + p.nacc, *drain = tempty + p.nacc;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *sfull = drain + 1;                         // paged: the record copies per stage
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfull + p.stages);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *pg_s = const_cast<int *>(abort_flag) + 4;     // page ids of this CTA's tiles (-1: none)
     // per epilogue group, kKsRing tiles of key scales in flight (cp.async ring)
@@ -230,7 +238,10 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             // second one once they are in place (gathered ones add and
             // complete their own pending arrivals)
             tc::mbar_init(tc::saddr(&full[s]), kSfStaged ? 2 : 1);
-            tc::mbar_init(tc::saddr(&empty[s]), 1);
+            // paged: the stage (which holds the row scales) is released by the
+            // epilogue warps that read them, not by the MMA
+            tc::mbar_init(tc::saddr(&empty[s]), kPaged ? 4 * (EG / 2) : 1);
+            if constexpr (kPaged) tc::mbar_init(tc::saddr(&sfull[s]), 1);
         }
         for (int i = 0; i < p.nacc; i++) {
             tc::mbar_init(tc::saddr(&tfull[i]), 1);
@@ -320,6 +331,45 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(tc::saddr(&full[j % p.stages]));
             }
+            if constexpr (kPaged) {
+                // tile j's records have landed (every lane observes the copy);
+                // move their block scales into the scale layout of stage j
+                const int s = j % p.stages;
+                const bool got = tc::mbar_wait(tc::saddr(&sfull[s]),
+                                               (uint32_t)((j / p.stages) & 1), abort_flag);
+                if (!__all_sync(0xffffffffu, got)) {              // uniform over the warp
+                    if (lane == 0) {
+                        if (!*abort_flag) report(a.status, CSA_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    return;
+                }
+                constexpr int nsf = RB / 8;                   // block scales per key
+                constexpr int kCpg = RB / 16;                 // 16-byte scale chunks per group
+                constexpr int KS = G::kKSteps;
+                const uint8_t *stg = stage_buf + s * kStage;
+                uint8_t *dst = sfa_buf + s * KS * 512;
+#pragma unroll
+                for (int q = lane; q < 16 * kCpg; q += 32) {
+                    const int half = q / (8 * kCpg), c = q % (8 * kCpg);
+                    const int g = c / kCpg, cg = c % kCpg;
+                    const int32_t page = pg_s[j * 2 + half];
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (page >= 0 && page < p.num_pages)
+                        v = *reinterpret_cast<const uint4 *>(stg + half * kRec + g * kGb + 8 * RB +
+                                                             cg * 16);
+                    const int m0 = half * 64 + g * 8 + cg * (16 / nsf);
+#pragma unroll
+                    for (int w = 0; w < 4; w++) {
+                        const int m = m0 + w / KS, ks = w % KS;
+                        const uint32_t x = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+                        *reinterpret_cast<uint32_t *>(dst + ks * 512 + (m & 31) * 16 + (m >> 5) * 4) = x;
+                    }
+                }
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(tc::saddr(&full[s]));
+            }
         };
         for (int i = 0; i < my_tiles; i++) {
             const int s = i % p.stages;
@@ -334,7 +384,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            if constexpr (kFp4 && !kSfStaged) {
+            if constexpr (kFp4 && !kSfStaged && !kPaged) {
                 // key m = lane + 32*m1 of the tile: its block scales of K-step ks go
                 // to byte (s*ksteps + ks)*512 + lane*16 + m1*4 by 4-byte cp.async;
                 // each lane's copies hold the stage's phase open until they land
@@ -361,7 +411,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 tc::cp_async_mbar_arrive(tc::saddr(&full[s]));
                 __syncwarp();
             }
-            if constexpr (kSfStaged) {
+            if constexpr (kSfStaged && !kPaged) {
                 // the tile's block scales: 16-byte chunks of each page's
                 // contiguous 64 x Di/16 bytes into staging slot i % kSfSlots
                 constexpr int nsf = RB / 8;               // Di/16 block scales per key
@@ -378,29 +428,37 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 tc::cp_async_commit();
             }
             if (lane == 0) {
-                tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
+                if constexpr (kPaged) tc::mbar_expect_tx(tc::saddr(&sfull[s]), kStage);
+                else tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
 #pragma unroll
                 for (int half = 0; half < 2; half++) {
                     int page = pg_s[i * 2 + half];
                     if (page < 0 || page >= p.num_pages) page = 0;   // epilogue reports visible keys
+                    if constexpr (kPaged) {
+                        // one copy per page: the whole record, one TMA box of
+                        // kRec/256 rows of 256 bytes (no swizzle)
+                        tc::tma_load_2d(tc::saddr(stage_buf + s * kStage + half * kRec), &kmap, 0,
+                                        page * (kRec / 256), tc::saddr(&sfull[s]));
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < G::kChunks; c++)
-                        tc::tma_load_2d(tc::saddr(stage_buf + s * G::kStageBytes +
-                                                  c * kTcTile * G::kSpan + half * 64 * G::kSpan),
-                                        &kmap, c * G::kSpan, page * kC4Page,
-                                        tc::saddr(&full[s]));
+                        for (int c = 0; c < G::kChunks; c++)
+                            tc::tma_load_2d(tc::saddr(stage_buf + s * kStage +
+                                                      c * kTcTile * G::kSpan + half * 64 * G::kSpan),
+                                            &kmap, c * G::kSpan, page * kC4Page,
+                                            tc::saddr(&full[s]));
+                    }
                 }
             }
             issued++;
-            if constexpr (kSfStaged) {
+            if constexpr (kSfStaged || kPaged) {
                 if (i >= kSfLag) {
-                    tc::cp_async_wait<kSfLag>();
+                    if constexpr (kSfStaged) tc::cp_async_wait<kSfLag>();
                     sf_place(i - kSfLag);
                 }
             }
         }
-        if constexpr (kSfStaged) {
-            tc::cp_async_wait<0>();
+        if constexpr (kSfStaged || kPaged) {
+            if constexpr (kSfStaged) tc::cp_async_wait<0>();
             for (int j = max(0, issued - kSfLag); j < issued; j++) sf_place(j);
         }
         // before leaving, every load issued must have landed
@@ -437,7 +495,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 tc::fence_after_sync();
                 if constexpr (kFp4) tc::fence_proxy_async();   // cp.async-written scales -> tcgen05.cp
                 const uint32_t d = tmem_base + (uint32_t)(acc * p.n);
-                const uint32_t sa = tc::saddr(stage_buf + s * G::kStageBytes);
+                const uint32_t sa = tc::saddr(stage_buf + s * kStage);
                 const uint32_t sb = tc::saddr(q_buf);
                 const uint32_t sfa = tmem_base + sfa_col + (uint32_t)(acc * 4 * G::kKSteps);
                 if constexpr (kFp4) {
@@ -450,14 +508,17 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
                 for (int k = 0; k < G::kKSteps; k++) {
                     const int c = (k * 32) / G::kSpan, off = (k * 32) % G::kSpan;
-                    const uint64_t ad = tc::kmajor_desc(sa + c * kTcTile * G::kSpan + off, G::kSpan);
+                    // paged keys: unswizzled, two 16-byte core matrices per K-step
+                    const uint64_t ad = kPaged ? tc::kmajor_plain_desc(sa + k * 256, 128, kGb)
+                                               : tc::kmajor_desc(sa + c * kTcTile * G::kSpan + off,
+                                                                 G::kSpan);
                     const uint64_t bd = tc::kmajor_desc(sb + c * p.n * G::kSpan + off, G::kSpan);
                     if constexpr (FMT == CSA_FMT_FP8) tc::mma_f8f6f4(d, ad, bd, idesc, k > 0);
                     else if constexpr (FMT == CSA_FMT_BF16) tc::mma_f16(d, ad, bd, idesc, k > 0);
                     else tc::mma_mxf4nvf4(d, ad, bd, idesc, sfa + 4 * k, tmem_base + sfb_col + 4 * k,
                                           k > 0);
                 }
-                tc::mma_commit(tc::saddr(&empty[s]));
+                if constexpr (!kPaged) tc::mma_commit(tc::saddr(&empty[s]));
                 tc::mma_commit(tc::saddr(&tfull[acc]));
             }
             // drain: every MMA issued has completed before TMEM is released
@@ -491,7 +552,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
         };
         float *my_ring = ks_ring + eg * kKsRing * kTcTile + row;
         auto ring_issue = [&](int j) {
-            if constexpr (FMT != CSA_FMT_BF16) {
+            if constexpr (FMT != CSA_FMT_BF16 && !kPaged) {   // paged: the scales come with the tile
                 bool v;
                 const int64_t slot = key_slot(par + 2 * j, v);
                 if (slot >= 0) tc::cp_async4(tc::saddr(my_ring + (j % kKsRing) * kTcTile),
@@ -512,7 +573,7 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
             (void)slot_i;
             if (!valid && sk < nv_max) report(a.status, CSA_ERR_BOUNDS);
             float kscale = 1.0f;
-            if constexpr (FMT != CSA_FMT_BF16) {
+            if constexpr (FMT != CSA_FMT_BF16 && !kPaged) {
                 tc::cp_async_wait<kKsRing - 2>();
                 kscale = valid ? my_ring[(j % kKsRing) * kTcTile] : 0.0f;
                 ring_issue(j + kKsRing - 1);
@@ -525,6 +586,19 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 break;
             }
             tc::fence_after_sync();
+            if constexpr (kPaged) {
+                // the key's row scale from the tile's records (their copy has
+                // completed: observed again here), then the stage is free
+                const int s = i % p.stages;
+                tc::mbar_wait(tc::saddr(&sfull[s]), (uint32_t)((i / p.stages) & 1), abort_flag);
+                const int r = row & 63;
+                kscale = valid ? *reinterpret_cast<const float *>(
+                                     stage_buf + s * kStage + (row >> 6) * kRec + (r >> 3) * kGb +
+                                     9 * RB + (r & 7) * 4)
+                               : 0.0f;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(tc::saddr(&empty[s]));
+            }
             // per query row x_lo + x of the group: sum_j w'[c+j] * ReLU(acc[c+j])
             // over its hi_pad columns (a multiple of 16)
             float out[4] = {0.f, 0.f, 0.f, 0.f};
@@ -628,6 +702,20 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// Tensor map over paged FP4 records as rows of 256 bytes (a record of
+// rec_bytes = 256 * r is one box of r rows, unswizzled).
+static bool make_record_map(CUtensorMap *m, const void *codes, int64_t num_pages, int rec_bytes) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {256, (cuuint64_t)(num_pages * (rec_bytes / 256))};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {256, (cuuint32_t)(rec_bytes / 256)};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tensor map over the index-key codes as a [num_slots, row_bytes] byte matrix,
 // 64-row boxes of one swizzle span.
 static bool make_key_map(CUtensorMap *m, const void *codes, int64_t num_slots, int row_bytes) {
@@ -646,21 +734,26 @@ static bool make_key_map(CUtensorMap *m, const void *codes, int64_t num_slots, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t tc_smem_bytes(int rb, bool fp4, const TcParams &p, int eg) {
+static size_t tc_smem_bytes(int rb, bool fp4, bool paged, const TcParams &p, int eg) {
     const size_t ks = rb / 32;
-    return 1024 + (size_t)p.stages * kTcTile * rb + (((size_t)p.n * rb + 1023) & ~(size_t)1023) +
-           (fp4 ? (p.stages + 1) * ks * 512 + (rb == 32 ? (size_t)kSfSlots * 16 * rb : 0) : 0) +
+    const size_t stage = paged ? 2 * 8 * (9 * (size_t)rb + 32) : (size_t)kTcTile * rb;
+    return 1024 + (size_t)p.stages * stage + (((size_t)p.n * rb + 1023) & ~(size_t)1023) +
+           (fp4 ? (p.stages + 1) * ks * 512 +
+                      (rb == 32 && !paged ? (size_t)kSfSlots * 16 * rb : 0) : 0) +
            256 * 4 + 16 * 4 +
-           (2 * p.stages + 2 * p.nacc + 1) * 8 + 32 +
+           (3 * p.stages + 2 * p.nacc + 1) * 8 + 32 +
            (size_t)2 * p.tiles_per_cta * 4 + 16 + (size_t)eg * kKsRing * kTcTile * 4;
 }
 
 bool indexer_tc_supported(const IndexerArgs &a) {
     const bool fmt_ok = (a.dim == 64 || a.dim == 128) &&
-                        (a.fmt == CSA_FMT_FP8 || a.fmt == CSA_FMT_BF16 || a.fmt == CSA_FMT_FP4);
-    // FP4 key block scales are copied in 16-byte chunks, query ones four at a time
-    const bool sf_ok = a.fmt != CSA_FMT_FP4 ||
-                       ((reinterpret_cast<uintptr_t>(a.k_block_scales) % 16) == 0 &&
+                        (a.fmt == CSA_FMT_FP8 || a.fmt == CSA_FMT_BF16 || a.fmt == CSA_FMT_FP4 ||
+                         a.fmt == CSA_FMT_FP4_PAGE);
+    // FP4 key block scales are copied in 16-byte chunks (paged: inside the
+    // 16-byte aligned records), query ones four at a time
+    const bool sf_ok = (a.fmt != CSA_FMT_FP4 ||
+                        (reinterpret_cast<uintptr_t>(a.k_block_scales) % 16) == 0) &&
+                       ((a.fmt != CSA_FMT_FP4 && a.fmt != CSA_FMT_FP4_PAGE) ||
                         (reinterpret_cast<uintptr_t>(a.q_block_scales) % 4) == 0);
     return fmt_ok && sf_ok && a.heads <= 128 && (a.num_slots % kC4Page) == 0 &&
            a.num_slots >= kC4Page && (reinterpret_cast<uintptr_t>(a.k_codes) % 16) == 0 &&
@@ -681,7 +774,8 @@ struct TcPlan {
 static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     TcPlan pl;
     TcParams &p = pl.p;
-    const bool fp4 = a.fmt == CSA_FMT_FP4;
+    const bool paged = a.fmt == CSA_FMT_FP4_PAGE;
+    const bool fp4 = a.fmt == CSA_FMT_FP4 || paged;
     const int rb = a.fmt == CSA_FMT_FP8 ? a.dim : fp4 ? a.dim / 2 : 2 * a.dim;
     pl.rb = rb;
     p.hi_pad = (a.heads + 15) / 16 * 16;
@@ -724,7 +818,7 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     }
     p.tiles_per_cta = fuse ? 64 : tiles_max;          // upper bound for the estimate
     // 228 KB of shared memory per SM, 1 KB of it reserved per resident CTA
-    const size_t smem_est = tc_smem_bytes(rb, fp4, p, pl.eg) + 1024;
+    const size_t smem_est = tc_smem_bytes(rb, fp4, paged, p, pl.eg) + 1024;
     int by_smem = (int)((228 * 1024) / smem_est);
     int ctas_per_sm = 512 / cols;
     if (by_smem < ctas_per_sm) ctas_per_sm = by_smem;
@@ -748,7 +842,7 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     }
     pl.chunks = (tiles_max + p.tiles_per_cta - 1) / p.tiles_per_cta;
     if (pl.chunks < 1) pl.chunks = 1;
-    pl.smem = tc_smem_bytes(rb, fp4, p, pl.eg);
+    pl.smem = tc_smem_bytes(rb, fp4, paged, p, pl.eg);
     return pl;
 }
 
@@ -763,12 +857,18 @@ bool indexer_topk_fuses(const IndexerArgs &a) {
 
 static cudaError_t launch_tc_plan(const IndexerArgs &a, const TcPlan &pl, const TcSelect &sel,
                                   cudaStream_t s) {
-    CUtensorMap map;
-    if (!make_key_map(&map, a.k_codes, a.num_slots, pl.rb)) return cudaErrorInvalidValue;
+    CUtensorMap map{};
+    if (a.fmt == CSA_FMT_FP4_PAGE) {
+        if (!make_record_map(&map, a.k_codes, a.num_slots / kC4Page, 72 * pl.rb + 256))
+            return cudaErrorInvalidValue;
+    } else if (!make_key_map(&map, a.k_codes, a.num_slots, pl.rb)) {
+        return cudaErrorInvalidValue;
+    }
     const TcParams p = pl.p;
     const size_t smem = pl.smem;
     dim3 grid(pl.chunks, query_groups_bound(a.num_q, a.bs, p.qg));
     const bool fp4 = a.fmt == CSA_FMT_FP4;
+    const bool paged = a.fmt == CSA_FMT_FP4_PAGE;
     const int rb = pl.rb;
 #define CSA_TC_EG(F, R, E)                                                                  \
     do {                                                                                    \
@@ -784,6 +884,8 @@ static cudaError_t launch_tc_plan(const IndexerArgs &a, const TcPlan &pl, const 
     } while (0)
     if (a.fmt == CSA_FMT_FP8 && rb == 128) CSA_TC(CSA_FMT_FP8, 128);
     else if (a.fmt == CSA_FMT_FP8) CSA_TC(CSA_FMT_FP8, 64);
+    else if (paged && rb == 64) CSA_TC_EG(CSA_FMT_FP4_PAGE, 64, 2);
+    else if (paged) CSA_TC_EG(CSA_FMT_FP4_PAGE, 32, 2);
     else if (fp4 && rb == 64) CSA_TC_EG(CSA_FMT_FP4, 64, 2);
     else if (fp4) CSA_TC_EG(CSA_FMT_FP4, 32, 2);
     else if (rb == 128) CSA_TC(CSA_FMT_BF16, 128);

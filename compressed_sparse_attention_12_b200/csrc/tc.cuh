@@ -294,6 +294,17 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr, int span) {
     return d;
 }
 
+// Shared-memory descriptor of a K-major operand without swizzle: core
+// matrices of 8 rows x 16 bytes (128 contiguous bytes), `lbo` bytes apart
+// along K and `sbo` bytes apart along M (or N).
+__device__ __forceinline__ uint64_t kmajor_plain_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((addr & 0x3FFFF) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
 // Byte offset of (row, byte) inside a tile of `span`-byte rows stored with the
 // `span`-byte swizzle (16-byte chunks XOR-ed with the address bits above 7).
 __device__ __forceinline__ uint32_t swz(int row, int byte, int span) {

@@ -41,7 +41,7 @@ def raw_slots(pt: np.ndarray, b: int, r: np.ndarray) -> np.ndarray:
 
 
 class CsaBatch:
-    def __init__(self, w: Workload, data: dict, device="cuda", sm_scale=None):
+    def __init__(self, w: Workload, data: dict, device="cuda", sm_scale=None, paged_fp4=False):
         self.w = w
         self.device = device
         dev = device
@@ -59,11 +59,19 @@ class CsaBatch:
         self.raw_cache = torch.zeros((self.raw_slots_n, rb), dtype=torch.uint8, device=dev)
         Di, Hi = w.idx_dim, w.idx_heads
         cb = code_bytes(w.idx_fmt, Di)
-        self.k_codes = torch.zeros((self.c4_slots_n, cb), dtype=torch.uint8, device=dev)
-        self.k_bsc = (torch.zeros((self.c4_slots_n, Di // 16), dtype=torch.uint8, device=dev)
-                      if w.idx_fmt == "fp4" else None)
-        self.k_scales = (torch.ones(self.c4_slots_n, dtype=torch.float32, device=dev)
-                         if w.idx_fmt != "bf16" else None)
+        # index keys: structure of arrays (codes, FP4 block scales, row scales);
+        # paged_fp4=True keeps FP4 keys as one CSA_FMT_FP4_PAGE record per page
+        self.key_fmt = csa.CSA_FMT_FP4_PAGE if (paged_fp4 and w.idx_fmt == "fp4") else self.idx_fmt
+        if self.key_fmt == csa.CSA_FMT_FP4_PAGE:
+            self.k_codes = torch.zeros((self.num_pages, csa.index_record_bytes(Di)),
+                                       dtype=torch.uint8, device=dev)
+            self.k_bsc = self.k_scales = None
+        else:
+            self.k_codes = torch.zeros((self.c4_slots_n, cb), dtype=torch.uint8, device=dev)
+            self.k_bsc = (torch.zeros((self.c4_slots_n, Di // 16), dtype=torch.uint8, device=dev)
+                          if w.idx_fmt == "fp4" else None)
+            self.k_scales = (torch.ones(self.c4_slots_n, dtype=torch.float32, device=dev)
+                             if w.idx_fmt != "bf16" else None)
         i32 = lambda a: torch.as_tensor(np.asarray(a, dtype=np.int32), device=dev)
         self.seq_lens = i32(w.seq_lens)
         self.c4_lens = i32(w.c4_lens)
@@ -83,7 +91,7 @@ class CsaBatch:
         if slots.size:
             csa.csa_kv_store(data["kv_c4"].contiguous(), slots_t, self.kv_fmt, self.c4_cache,
                              status=self.status)
-            csa.csa_hadamard_quant(data["idx_k"].contiguous(), self.idx_fmt, self.k_codes,
+            csa.csa_hadamard_quant(data["idx_k"].contiguous(), self.key_fmt, self.k_codes,
                                    self.k_bsc, self.k_scales, row_map=slots_t, status=self.status)
         rreq, rpos = np.asarray(data["raw_req"]), np.asarray(data["raw_pos"])
         rs = pt[rreq, rpos // PAGE].astype(np.int64) * PAGE + rpos % PAGE
@@ -117,7 +125,7 @@ class CsaBatch:
                                    dtype=torch.uint8, device=dev)
         self.fused_ws = torch.empty(
             max(1, csa.csa_indexer_topk512_workspace_size(nq, w.bs, w.idx_heads, w.idx_dim,
-                                                          self.idx_fmt, self.max_c4)),
+                                                          self.key_fmt, self.max_c4)),
             dtype=torch.uint8, device=dev)
         self.decode = bool((w.q_lens <= 8).all())
         self.attn_ws = torch.empty(
@@ -155,6 +163,8 @@ class CsaBatch:
             return
         ik = {"bf16": csa.CSA_OUT_INDEX_BF16, "fp8": csa.CSA_OUT_INDEX_FP8,
               "fp4": csa.CSA_OUT_INDEX_FP4}[w.idx_fmt]
+        if self.key_fmt == csa.CSA_FMT_FP4_PAGE:
+            ik = csa.CSA_OUT_INDEX_FP4_PAGE
         csa.csa_c4_compress(self.raw_idx_k, self.idx_gate, self.idx_bias, self.cu_new,
                             self.start_pos, self.max_new, self.page_table, ik, self.k_codes,
                             self.k_bsc, self.k_scales, status=self.status, stream=stream)
@@ -165,7 +175,7 @@ class CsaBatch:
                                w_in=self.w_head, w_out=self.w_fold, status=self.status,
                                stream=stream)
         csa.csa_indexer_logits(self.q_codes, self.q_bsc, self.w_fold, w.idx_heads, w.idx_dim,
-                               self.idx_fmt, self.k_codes, self.k_bsc, self.k_scales,
+                               self.key_fmt, self.k_codes, self.k_bsc, self.k_scales,
                                self.page_table, self.c4_lens, self.cu_q, self.q_pos, self.max_c4,
                                self.logits, status=self.status, stream=stream)
 
@@ -180,7 +190,7 @@ class CsaBatch:
         w = self.w
         self.quantise_q(stream)
         csa.csa_indexer_topk512(self.q_codes, self.q_bsc, self.w_fold, w.idx_heads, w.idx_dim,
-                                self.idx_fmt, self.k_codes, self.k_bsc, self.k_scales,
+                                self.key_fmt, self.k_codes, self.k_bsc, self.k_scales,
                                 self.page_table, self.c4_lens, self.cu_q, self.q_pos, self.max_c4,
                                 self.logits, self.indices, self.raw_indices, self.fused_ws,
                                 num_slots=self.c4_slots_n, status=self.status, stream=stream)

@@ -59,6 +59,21 @@
  *    CSA_FMT_FP4 : codes = Di/2 bytes, two E2M1 codes per byte (element 2i in
  *                  the low nibble); block_scales = Di/16 unsigned-E4M3 bytes,
  *                  sb = RN(amax_blk/(6*s)); scales[row] fp32 s = amax/2688
+ *    CSA_FMT_FP4_PAGE (index keys only): the FP4 values, codes and scales of
+ *                  the 64 keys of one compressed page (slots 64p .. 64p+63)
+ *                  kept together in one record of R = 36*Di + 256 bytes at
+ *                  byte p*R of the `k_codes` array (2560 bytes for Di = 64,
+ *                  4864 for Di = 128; k_block_scales and k_scales unused).
+ *                  The record is 8 groups of 8 keys, group g (keys 8g..8g+7)
+ *                  at byte g*Gb with Gb = 4.5*Di + 32; for key r (= slot%64,
+ *                  i = r%8) in group g = r/8:
+ *                    code byte b at    g*Gb + (b/16)*128 + i*16 + b%16
+ *                                      (8-key x 16-byte blocks, the tensor
+ *                                      cores' unswizzled operand order)
+ *                    block scale j at  g*Gb + 4*Di + i*Di/16 + j
+ *                    fp32 row scale at g*Gb + 4.5*Di + 4*i
+ *                  so that one copy moves a page and two pages side by side
+ *                  keep one stride between groups.  Queries stay CSA_FMT_FP4.
  *  Every quantised value is rounded to nearest, ties to even, saturating.
  */
 #ifndef CSA_H_
@@ -86,7 +101,8 @@ typedef enum {
     CSA_FMT_BF16 = 0,
     CSA_FMT_FP8 = 1,          /* E4M3 */
     CSA_FMT_FP4 = 2,          /* E2M1 with block-16 unsigned-E4M3 scales */
-    CSA_FMT_F32 = 3           /* input-only: float32 */
+    CSA_FMT_F32 = 3,          /* input-only: float32 */
+    CSA_FMT_FP4_PAGE = 4      /* index keys: FP4 in one record per 64-key page */
 } csa_fmt_t;
 
 /* What csa_c4_compress writes. */
@@ -95,7 +111,8 @@ typedef enum {
     CSA_OUT_KV_FP8 = 1,       /* dim 576, KV row in CSA_FMT_FP8                               */
     CSA_OUT_INDEX_BF16 = 2,   /* dim 64/128, rotated index key, bf16 codes                    */
     CSA_OUT_INDEX_FP8 = 3,    /* dim 64/128, rotated index key, FP8 codes + row scale          */
-    CSA_OUT_INDEX_FP4 = 4     /* dim 64/128, rotated index key, FP4 codes + block/row scales   */
+    CSA_OUT_INDEX_FP4 = 4,    /* dim 64/128, rotated index key, FP4 codes + block/row scales   */
+    CSA_OUT_INDEX_FP4_PAGE = 5 /* dim 64/128, rotated index key into CSA_FMT_FP4_PAGE records  */
 } csa_out_kind_t;
 
 enum { CSA_TOPK = 512, CSA_PAGE_SIZE = 256, CSA_C4_PAGE_SIZE = 64, CSA_C4_RATIO = 4,

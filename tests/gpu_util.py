@@ -15,9 +15,58 @@ def code_bytes(fmt, dim):
     return {"bf16": 2 * dim, "fp8": dim, "fp4": dim // 2}[fmt]
 
 
+def _fp4_page_offsets(dim):
+    """Byte offsets inside a CSA_FMT_FP4_PAGE record (include/csa.h) of each
+    key's code bytes [64, dim/2], block scales [64, dim/16] and row scale
+    bytes [64, 4]."""
+    gb = 4 * dim + dim // 2 + 32
+    r = np.arange(64)[:, None]
+    g, i = r // 8, r % 8
+    b = np.arange(dim // 2)[None, :]
+    codes = g * gb + (b // 16) * 128 + i * 16 + b % 16
+    blocks = g * gb + 4 * dim + i * (dim // 16) + np.arange(dim // 16)[None, :]
+    rows = g * gb + 4 * dim + dim // 2 + 4 * i + np.arange(4)[None, :]
+    return codes, blocks, rows
+
+
+def fp4_page_records(packed, bsc, sc, dim):
+    """FP4 index arrays of n slots (n a multiple of 64) laid out as the
+    paged records of CSA_FMT_FP4_PAGE: per 64-key page, 8 groups of 8 keys,
+    each group's codes (8-key x 16-byte blocks), block scales and fp32 row
+    scales side by side."""
+    packed, bsc = np.asarray(packed, np.uint8), np.asarray(bsc, np.uint8)
+    sc = np.asarray(sc, np.float32)
+    n = packed.shape[0]
+    assert n % 64 == 0
+    pages = n // 64
+    oc, ob, orow = _fp4_page_offsets(dim)
+    rec = np.zeros((pages, 36 * dim + 256), dtype=np.uint8)
+    rec[:, oc] = packed.reshape(pages, 64, dim // 2)
+    rec[:, ob] = bsc.reshape(pages, 64, dim // 16)
+    rec[:, orow] = sc.reshape(pages, 64).view(np.uint8).reshape(pages, 64, 4)
+    return rec
+
+
+def fp4_page_unpack(rec, dim):
+    """Inverse of fp4_page_records: (packed codes, block scales, row scales)
+    per slot."""
+    rec = np.asarray(rec, np.uint8)
+    pages = rec.shape[0]
+    oc, ob, orow = _fp4_page_offsets(dim)
+    packed = rec[:, oc].reshape(pages * 64, dim // 2)
+    bsc = rec[:, ob].reshape(pages * 64, dim // 16)
+    sc = np.ascontiguousarray(rec[:, orow]).view(np.float32).reshape(pages * 64)
+    return packed, bsc, sc
+
+
 def index_arrays(q, fmt, dim, n_rows, rows=None):
     """Oracle index quantisation result `q` (orc.index_quantise) written into
-    [n_rows] library arrays at row indices `rows` (default 0..)."""
+    [n_rows] library arrays at row indices `rows` (default 0..).  "fp4p": the
+    FP4 result as paged records (keys; n_rows a multiple of 64), returned as
+    (records, None, None)."""
+    if fmt == "fp4p":
+        codes, bsc, sc = (t.cpu().numpy() for t in index_arrays(q, "fp4", dim, n_rows, rows))
+        return dev(fp4_page_records(codes, bsc, sc, dim)), None, None
     n = q["deq"].reshape(-1, dim).shape[0]
     rows = np.arange(n) if rows is None else np.asarray(rows)
     codes = np.zeros((n_rows, code_bytes(fmt, dim)), dtype=np.uint8)

@@ -193,3 +193,29 @@ def test_host_validation_of_the_next_rows(L):
     assert r == csa.CSA_ERR_WORKSPACE
     # the wait self-test needs a status word
     assert L.csa_selftest_wait_timeout(None, None, None) == csa.CSA_ERR_INVALID
+
+
+def test_fp4_page_record_layout():
+    """The test-side layout of CSA_FMT_FP4_PAGE records (include/csa.h) round
+    trips and puts a hand-computed byte where the header says."""
+    import numpy as np
+    from gpu_util import fp4_page_records, fp4_page_unpack
+    rng = np.random.default_rng(0)
+    for dim in (64, 128):
+        n = 128
+        packed = rng.integers(0, 256, (n, dim // 2), dtype=np.uint8)
+        bsc = rng.integers(0, 127, (n, dim // 16), dtype=np.uint8)
+        sc = rng.uniform(0.1, 2.0, n).astype(np.float32)
+        rec = fp4_page_records(packed, bsc, sc, dim)
+        assert rec.shape == (2, 36 * dim + 256)
+        pk, pb, ps = fp4_page_unpack(rec, dim)
+        assert np.array_equal(pk, packed) and np.array_equal(pb, bsc) and np.array_equal(ps, sc)
+        # key 73: page 1, r = 9, group 1, i = 1; groups of gb = 4.5*dim + 32 bytes
+        gb = 4 * dim + dim // 2 + 32
+        assert gb * 8 == 36 * dim + 256
+        # code byte 17: gb + (17//16)*128 + 1*16 + 17%16
+        assert rec[1, gb + 128 + 16 + 1] == packed[73, 17]
+        # its second block scale and its row scale
+        assert rec[1, gb + 4 * dim + dim // 16 + 1] == bsc[73, 1]
+        o = gb + 4 * dim + dim // 2 + 4
+        assert rec[1, o:o + 4].view(np.float32)[0] == sc[73]

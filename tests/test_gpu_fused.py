@@ -20,11 +20,11 @@ def lib():
     return csa.lib()
 
 
-def _batch(name, scale):
+def _batch(name, scale, paged=False):
     from compressed_sparse_attention_12_b200 import pipeline, synth
     w = synth.workload(name, scale)
     data = synth.draw(w, "cuda")
-    return w, pipeline.CsaBatch(w, data)
+    return w, pipeline.CsaBatch(w, data, paged_fp4=paged)
 
 
 def _separate(batch):
@@ -36,12 +36,13 @@ def _separate(batch):
     return batch.logits.clone(), batch.indices.clone(), batch.raw_indices.clone()
 
 
-@pytest.mark.parametrize("name,scale", [("tiny", 1.0), ("decode_128k", 1 / 64),
-                                        ("decode_128k", 1.0), ("decode_1m", 1.0),
-                                        ("decode_1m_wide", 1 / 16), ("ragged", 1 / 32),
-                                        ("prefill", 1 / 16)])
-def test_fused_equals_separate(name, scale):
-    w, batch = _batch(name, scale)
+@pytest.mark.parametrize("name,scale,paged", [("tiny", 1.0, False), ("decode_128k", 1 / 64, False),
+                                              ("decode_128k", 1.0, False), ("decode_1m", 1.0, False),
+                                              ("decode_1m_wide", 1 / 16, False),
+                                              ("ragged", 1 / 32, False), ("prefill", 1 / 16, False),
+                                              ("decode_1m_wide", 1 / 16, True)])
+def test_fused_equals_separate(name, scale, paged):
+    w, batch = _batch(name, scale, paged)
     lg, idx, raw = _separate(batch)
     batch.logits.fill_(float("nan"))
     batch.indices.fill_(-7)
@@ -68,10 +69,10 @@ def test_select_then_merge_equals_fused(name, scale):
     batch.raw_indices.fill_(-7)
     ws = torch.empty_like(batch.fused_ws)
     csa.csa_indexer_select(batch.q_codes, batch.q_bsc, batch.w_fold, w.idx_heads, w.idx_dim,
-                           batch.idx_fmt, batch.k_codes, batch.k_bsc, batch.k_scales,
+                           batch.key_fmt, batch.k_codes, batch.k_bsc, batch.k_scales,
                            batch.page_table, batch.c4_lens, batch.cu_q, batch.q_pos, batch.max_c4,
                            batch.logits, ws, num_slots=batch.c4_slots_n, status=batch.status)
-    csa.csa_topk512_merge(w.num_q, w.idx_heads, w.idx_dim, batch.idx_fmt, batch.c4_lens,
+    csa.csa_topk512_merge(w.num_q, w.idx_heads, w.idx_dim, batch.key_fmt, batch.c4_lens,
                           batch.cu_q, batch.q_pos, batch.page_table, batch.c4_slots_n,
                           batch.max_c4, batch.indices, ws, raw_indices=batch.raw_indices,
                           status=batch.status)
@@ -87,7 +88,7 @@ def test_fused_workspace_is_checked():
     small = torch.empty(16, dtype=torch.uint8, device="cuda")
     with pytest.raises(csa.CsaError) as e:
         csa.csa_indexer_topk512(batch.q_codes, batch.q_bsc, batch.w_fold, w.idx_heads,
-                                w.idx_dim, batch.idx_fmt, batch.k_codes, batch.k_bsc,
+                                w.idx_dim, batch.key_fmt, batch.k_codes, batch.k_bsc,
                                 batch.k_scales, batch.page_table, batch.c4_lens, batch.cu_q,
                                 batch.q_pos, batch.max_c4, batch.logits, batch.indices,
                                 batch.raw_indices, small, status=batch.status)

@@ -31,14 +31,19 @@ def _gpu(d):
     return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
 
 
-@pytest.mark.parametrize("name,scale", [("tiny", 1.0), ("decode_128k", 1 / 64),
-                                        ("decode_1m", 1 / 256), ("decode_1m_wide", 1 / 256),
-                                        ("ragged", 1 / 128), ("prefill", 1 / 64)])
-def test_step_end_to_end(name, scale):
+@pytest.mark.parametrize("name,scale,paged", [("tiny", 1.0, False), ("decode_128k", 1 / 64, False),
+                                              ("decode_1m", 1 / 256, False),
+                                              ("decode_1m_wide", 1 / 256, False),
+                                              ("ragged", 1 / 128, False), ("prefill", 1 / 64, False),
+                                              ("decode_1m", 1 / 256, True),
+                                              ("ragged", 1 / 128, True)])
+def test_step_end_to_end(name, scale, paged):
+    """paged: FP4 index keys kept as CSA_FMT_FP4_PAGE records (the compressor
+    writes them, the indexer reads them)."""
     from compressed_sparse_attention_12_b200 import pipeline, synth
     w = synth.workload(name, scale)
     data = synth.draw(w, "cpu")
-    batch = pipeline.CsaBatch(w, _gpu(data))
+    batch = pipeline.CsaBatch(w, _gpu(data), paged_fp4=paged)
     batch.step()
     torch.cuda.synchronize()
     batch.check_status()
@@ -97,7 +102,8 @@ def _full_index_check(name, sample_q):
     s = np.arange(n)
     slots = np.concatenate([pt[b, s // 64].astype(np.int64) * 64 + s % 64 for b in range(bs)])
     n_slots = w.num_pages * 64
-    kc, kb, ks = index_arrays(kq, w.idx_fmt, Di, n_slots, slots)
+    kfmt = w.idx_fmt
+    kc, kb, ks = index_arrays(kq, kfmt, Di, n_slots, slots)
     qx = rng.standard_normal((bs, Hi, Di))
     qq = orc.index_quantise(qx, w.idx_fmt)
     qc, qb, qs = index_arrays(qq, w.idx_fmt, Di, bs * Hi)
@@ -109,9 +115,9 @@ def _full_index_check(name, sample_q):
     c4 = dev(w.c4_lens.astype(np.int32))
     cu_q = dev(w.cu_q)
     q_pos = dev(w.q_pos)
-    fmt = csa.FMT[w.idx_fmt]
+    fmt = csa.FMT[kfmt]
     csa.csa_indexer_logits(qc, qb, dev(wf), Hi, Di, fmt, kc, kb, ks, dev(pt), c4, cu_q, q_pos, n,
-                           logits, status=st)
+                           logits, num_slots=n_slots, status=st)
     torch.cuda.synchronize()
     assert st.item() == 0
     got = logits.cpu().numpy()[:, :n]
@@ -191,7 +197,8 @@ def _full_ragged_check(name, sample_q):
     slots = np.concatenate([pt[b, np.arange(c4[b]) // 64].astype(np.int64) * 64 +
                             np.arange(c4[b]) % 64 for b in range(bs)])
     n_slots = w.num_pages * 64
-    kc, kb, ks = index_arrays(kq, w.idx_fmt, Di, n_slots, slots)
+    kfmt = w.idx_fmt
+    kc, kb, ks = index_arrays(kq, kfmt, Di, n_slots, slots)
     qx = rng.standard_normal((nq, Hi, Di))
     qq = orc.index_quantise(qx, w.idx_fmt)
     qc, qb, qs = index_arrays(qq, w.idx_fmt, Di, nq * Hi)
@@ -202,8 +209,8 @@ def _full_ragged_check(name, sample_q):
     logits = torch.empty((nq, stride), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     c4_d, cu_q, q_pos = dev(c4.astype(np.int32)), dev(w.cu_q), dev(w.q_pos)
-    csa.csa_indexer_logits(qc, qb, dev(wf), Hi, Di, csa.FMT[w.idx_fmt], kc, kb, ks, dev(pt), c4_d,
-                           cu_q, q_pos, max_c4, logits, status=st)
+    csa.csa_indexer_logits(qc, qb, dev(wf), Hi, Di, csa.FMT[kfmt], kc, kb, ks, dev(pt), c4_d,
+                           cu_q, q_pos, max_c4, logits, num_slots=n_slots, status=st)
     torch.cuda.synchronize()
     assert st.item() == 0
     got = logits.cpu().numpy()
@@ -322,7 +329,8 @@ def test_full_size_prefill_indexer_shared_codes():
     s = np.arange(n)
     slots = pt[0, s // 64].astype(np.int64) * 64 + s % 64
     n_slots = w.num_pages * 64
-    kc, kb, ks = index_arrays(kq, w.idx_fmt, Di, n_slots, slots)
+    kfmt = w.idx_fmt
+    kc, kb, ks = index_arrays(kq, kfmt, Di, n_slots, slots)
     qx = rng.standard_normal((nq, Hi, Di))
     qq = orc.index_quantise(qx, w.idx_fmt)
     qc, qb, qs = index_arrays(qq, w.idx_fmt, Di, nq * Hi)

@@ -24,7 +24,7 @@ from oracle import oracle as orc
 
 pytestmark = pytest.mark.gpu
 
-FMT = {"bf16": 0, "fp8": 1, "fp4": 2}
+FMT = {"bf16": 0, "fp8": 1, "fp4": 2, "fp4p": 4}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -155,6 +155,42 @@ def test_hadamard_quant_row_map_scatter():
     assert (got[r[v]] == ref["codes"][v]).mean() > 0.999
     untouched = np.setdiff1d(np.arange(n_out), r[v])
     assert (got[untouched] == 0x55).all() and (sc.cpu().numpy()[untouched] == -1.0).all()
+
+
+@pytest.mark.parametrize("dim", [64, 128])
+def test_hadamard_quant_fp4_page_records(dim):
+    """Index keys quantised straight into paged records equal the plain FP4
+    arrays of the same call laid out as records, byte for byte, and untouched
+    slots stay as they were."""
+    from gpu_util import fp4_page_unpack
+    csa = _csa()
+    g = torch.Generator().manual_seed(11 + dim)
+    rows, pages = 700, 20
+    n_slots = pages * 64
+    x = torch.randn(rows, dim, generator=g) * 3.0
+    rmap = torch.randperm(n_slots, generator=g)[:rows].int()
+    w = torch.rand(rows, generator=g)
+    codes = torch.zeros((n_slots, dim // 2), dtype=torch.uint8, device="cuda")
+    bsc = torch.zeros((n_slots, dim // 16), dtype=torch.uint8, device="cuda")
+    sc = torch.ones(n_slots, dtype=torch.float32, device="cuda")
+    wo = torch.empty(rows, dtype=torch.float32, device="cuda")
+    rec = torch.full((pages, csa.index_record_bytes(dim)), 0x5A, dtype=torch.uint8, device="cuda")
+    wo2 = torch.empty(rows, dtype=torch.float32, device="cuda")
+    st = zstatus()
+    csa.csa_hadamard_quant(x.cuda(), FMT["fp4"], codes, bsc, sc, row_map=rmap.cuda(),
+                           w_in=w.cuda(), w_out=wo, status=st)
+    csa.csa_hadamard_quant(x.cuda(), FMT["fp4p"], rec, None, None, row_map=rmap.cuda(),
+                           w_in=w.cuda(), w_out=wo2, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    pk, pb, ps = fp4_page_unpack(rec.cpu().numpy(), dim)
+    r = rmap.numpy()
+    assert np.array_equal(pk[r], codes.cpu().numpy()[r])
+    assert np.array_equal(pb[r], bsc.cpu().numpy()[r])
+    assert np.array_equal(ps[r].view(np.uint32), sc.cpu().numpy()[r].view(np.uint32))
+    assert np.array_equal(wo.cpu().numpy(), wo2.cpu().numpy())
+    untouched = np.setdiff1d(np.arange(n_slots), r)
+    assert (pk[untouched] == 0x5A).all() and (pb[untouched] == 0x5A).all()
 
 
 # ------------------------------------------------------------------ compressor
@@ -297,6 +333,32 @@ def test_c4_compress_index(fmt, dim):
     _compare_codes(gc, gb, gs, ref, fmt, dim, y.shape[0])
 
 
+@pytest.mark.parametrize("dim", [64, 128])
+def test_c4_compress_index_fp4_page(dim):
+    """The compressor writing index keys into paged FP4 records gives the same
+    bytes per slot as the compressor writing the plain FP4 arrays."""
+    from gpu_util import fp4_page_unpack
+    csa = _csa()
+    x, gate, bias, cu, start, pt, n_slots, new = _compress_setup(dim, 40 + dim)
+    codes = torch.zeros((n_slots, dim // 2), dtype=torch.uint8, device="cuda")
+    bsc = torch.zeros((n_slots, dim // 16), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(n_slots, dtype=torch.float32, device="cuda")
+    rec = torch.zeros((n_slots // 64, csa.index_record_bytes(dim)), dtype=torch.uint8,
+                      device="cuda")
+    st = zstatus()
+    args = (dev(x), dev(gate), dev(bias), dev(cu), dev(start.astype(np.int32)), int(new.max()),
+            dev(pt))
+    csa.csa_c4_compress(*args, csa.CSA_OUT_INDEX_FP4, codes, bsc, sc, status=st)
+    csa.csa_c4_compress(*args, csa.CSA_OUT_INDEX_FP4_PAGE, rec, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    pk, pb, ps = fp4_page_unpack(rec.cpu().numpy(), dim)
+    assert np.array_equal(pk, codes.cpu().numpy())
+    assert np.array_equal(pb, bsc.cpu().numpy())
+    assert np.array_equal(ps.view(np.uint32), sc.cpu().numpy().view(np.uint32))
+    assert (ps != 0).sum() > 0
+
+
 # ------------------------------------------------------------------ indexer
 
 def _indexer_case(fmt, dim, heads, seed, c4_lens, q_lens, dist="normal"):
@@ -324,10 +386,11 @@ def _indexer_case(fmt, dim, heads, seed, c4_lens, q_lens, dist="normal"):
         slots.append(pt[b, s // 64].astype(np.int64) * 64 + s % 64)
     keys = np.concatenate(key_rows) if key_rows else np.zeros((0, dim))
     slots = np.concatenate(slots).astype(np.int64)
-    kq = orc.index_quantise(keys, fmt)
+    ofmt = "fp4" if fmt == "fp4p" else fmt      # paged records hold the FP4 values
+    kq = orc.index_quantise(keys, ofmt)
     nq = int(q_lens.sum())
     qx = rng.standard_normal((nq, heads, dim))
-    qq = orc.index_quantise(qx, fmt)
+    qq = orc.index_quantise(qx, ofmt)
     w = rng.uniform(size=(nq, heads)).astype(np.float32)
     cu_q = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
     q_pos = np.concatenate([np.arange(L[b] - q_lens[b], L[b]) for b in range(bs)]).astype(np.int32)
@@ -336,16 +399,18 @@ def _indexer_case(fmt, dim, heads, seed, c4_lens, q_lens, dist="normal"):
 
 
 INDEXER_CASES = [("bf16", 64, 8), ("fp8", 128, 64), ("fp4", 64, 8), ("fp4", 128, 64),
-                 ("fp8", 64, 16), ("bf16", 128, 32), ("fp8", 128, 8)]
+                 ("fp8", 64, 16), ("bf16", 128, 32), ("fp8", 128, 8), ("fp4p", 64, 8),
+                 ("fp4p", 128, 64), ("fp4p", 64, 16)]
 
 
 @pytest.mark.parametrize("fmt,dim,heads", INDEXER_CASES)
 def test_indexer_logits(fmt, dim, heads):
     csa = _csa()
     c = _indexer_case(fmt, dim, heads, seed=dim + heads, c4_lens=[0, 1, 63, 64, 65, 1000, 5000, 2049],
-                      q_lens=[1, 1, 5, 1, 2, 1, 5, 3], dist="t3" if fmt == "fp4" else "normal")
+                      q_lens=[1, 1, 5, 1, 2, 1, 5, 3],
+                      dist="t3" if fmt in ("fp4", "fp4p") else "normal")
     kc, kb, ks = index_arrays(c["keys"], fmt, dim, c["n_slots"], c["slots"])
-    qc, qb, qs = index_arrays(c["qq"], fmt, dim, c["nq"] * heads)
+    qc, qb, qs = index_arrays(c["qq"], "fp4" if fmt == "fp4p" else fmt, dim, c["nq"] * heads)
     wf = c["w"] * (c["qq"]["scales"].reshape(c["nq"], heads) if fmt != "bf16" else 1.0)
     wf = wf.astype(np.float32)
     max_c4 = int(c["c4"].max())
