@@ -809,7 +809,7 @@ def measure_csa(args, name, world, rank, local, dev, full=True):
         if not fused[0]:
             ev_i0.record(s)
             c.csa_indexer_logits(batch_q.q_codes, batch_q.q_bsc, batch_q.w_fold, w.idx_heads,
-                                 w.idx_dim, batch_q.idx_fmt, batch_q.k_codes, batch_q.k_bsc,
+                                 w.idx_dim, batch_q.key_fmt, batch_q.k_codes, batch_q.k_bsc,
                                  batch_q.k_scales, batch_q.page_table, batch_q.c4_lens,
                                  batch_q.cu_q, batch_q.q_pos, batch_q.max_c4, batch_q.logits,
                                  status=batch_q.status, stream=s)
@@ -819,12 +819,12 @@ def measure_csa(args, name, world, rank, local, dev, full=True):
             return
         ev_i0.record(s)
         c.csa_indexer_select(batch_q.q_codes, batch_q.q_bsc, batch_q.w_fold, w.idx_heads,
-                             w.idx_dim, batch_q.idx_fmt, batch_q.k_codes, batch_q.k_bsc,
+                             w.idx_dim, batch_q.key_fmt, batch_q.k_codes, batch_q.k_bsc,
                              batch_q.k_scales, batch_q.page_table, batch_q.c4_lens, batch_q.cu_q,
                              batch_q.q_pos, batch_q.max_c4, batch_q.logits, batch_q.fused_ws,
                              num_slots=batch_q.c4_slots_n, status=batch_q.status, stream=s)
         ev_i1.record(s)
-        c.csa_topk512_merge(w.num_q, w.idx_heads, w.idx_dim, batch_q.idx_fmt, batch_q.c4_lens,
+        c.csa_topk512_merge(w.num_q, w.idx_heads, w.idx_dim, batch_q.key_fmt, batch_q.c4_lens,
                             batch_q.cu_q, batch_q.q_pos, batch_q.page_table, batch_q.c4_slots_n,
                             batch_q.max_c4, batch_q.indices, batch_q.fused_ws,
                             raw_indices=batch_q.raw_indices, status=batch_q.status, stream=s)
