@@ -379,17 +379,48 @@ def pack_inputs(batch, names, dev):
     return arena
 
 
-def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_bytes):
+def _cudart():
+    """The CUDA runtime torch is linked against (for host<->device copies
+    recorded into a graph)."""
+    import ctypes
+    import glob
+    import torch
+    for name in ("libcudart.so.12", "libcudart.so"):
+        try:
+            return ctypes.CDLL(name)
+        except OSError:
+            pass
+    base = os.path.dirname(torch.__file__)
+    for pat in (os.path.join(base, "..", "nvidia", "cuda_runtime", "lib", "libcudart.so*"),
+                os.path.join(base, "lib", "libcudart*.so*")):
+        for f in sorted(glob.glob(pat)):
+            return ctypes.CDLL(f)
+    raise RuntimeError("CUDA runtime library not found")
+
+
+def _copy_async(rt, dst, src, nbytes, kind, stream):
+    """cudaMemcpyAsync(dst, src, nbytes, kind, stream); kind 1 = host to
+    device, 2 = device to host."""
+    import ctypes
+    rc = rt.cudaMemcpyAsync(ctypes.c_void_p(dst.data_ptr()), ctypes.c_void_p(src.data_ptr()),
+                            ctypes.c_size_t(nbytes), ctypes.c_int(kind),
+                            ctypes.c_void_p(stream.cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"cudaMemcpyAsync failed: {rc}")
+
+
+def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_bytes, body):
     """The step end to end: every step copies its inputs (the packed arena)
-    from pinned host memory, replays the graph and copies the output back to
+    from pinned host memory, runs the step and copies the output back to
     pinned host memory, all inside the timed region.
 
     Reported, when the step's working set (step_bytes) is larger than L2: the
-    pipelined loop a serving process runs (two staging buffers on each side:
-    the copy of step i+1's inputs and the read-back of step i-1's output run
-    on their own streams while step i computes; no L2 flush is needed), and
-    beside it the one-step-at-a-time loop with an L2 flush before every step.
-    Smaller steps report the one-step-at-a-time loop only."""
+    pipelined loop a serving process runs -- two staging buffers on each
+    side; each step is one launch of a graph whose three branches copy step
+    i+1's inputs in, run step i (`body`), and read step i-1's output back,
+    so that both copies run while step i computes; no L2 flush is needed --
+    and beside it the one-step-at-a-time loop with an L2 flush before every
+    step.  Smaller steps report the one-step-at-a-time loop only."""
     import torch
     h_in = arena.cpu().pin_memory()
     h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
@@ -410,6 +441,7 @@ def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_byte
             e1.synchronize()
             if i >= args.warmup:
                 ms.append(e0.elapsed_time(e1))
+    ref = h_out[0].clone()
     t_seq = sum(ms) / len(ms) / 1e3
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     if step_bytes <= l2:
@@ -417,57 +449,73 @@ def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_byte
         return {"value": world * num_q / t_seq, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": t_seq * 1e3,
                 "pipelined": None}
-    # pipelined, depth 2
+    # pipelined, depth 2: graph b runs step i (i % 2 == b) from stage_in[b]
+    # into stage_out[b], copies step i+1's inputs into stage_in[1-b] and
+    # reads step i-1's output back from stage_out[1-b]
+    rt = _cudart()
     c_in = torch.cuda.Stream(device=dev)
     c_out = torch.cuda.Stream(device=dev)
     stage_in = [torch.empty_like(arena) for _ in range(2)]
     stage_out = [torch.empty_like(out) for _ in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_in_free = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out_free = [torch.cuda.Event() for _ in range(2)]
+    out_bytes = out.numel() * out.element_size()
+
+    def pipeline_graph(b):
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gp, stream=stream):
+                c_in.wait_stream(stream)
+                c_out.wait_stream(stream)
+                _copy_async(rt, stage_in[1 - b], h_in, h2d, 1, c_in)
+                _copy_async(rt, h_out[1 - b], stage_out[1 - b], out_bytes, 2, c_out)
+                arena.copy_(stage_in[b])
+                body(stream)
+                stage_out[b].copy_(out)
+                stream.wait_stream(c_in)
+                stream.wait_stream(c_out)
+        return gp
+
+    graphs = [pipeline_graph(0), pipeline_graph(1)]
 
     def run(n, timed):
         torch.cuda.synchronize()
-        for e in ev_in_free + ev_out_free:
-            e.record(stream)
-        if timed:
-            e0.record(stream)
-        for i in range(n):
-            b = i & 1
-            c_in.wait_event(ev_in_free[b])
-            with torch.cuda.stream(c_in):
-                stage_in[b].copy_(h_in, non_blocking=True)
-            ev_in[b].record(c_in)
-            stream.wait_event(ev_in[b])
-            with torch.cuda.stream(stream):
-                arena.copy_(stage_in[b])
-                ev_in_free[b].record(stream)
-                g.replay()
-                stream.wait_event(ev_out_free[b])
-                stage_out[b].copy_(out)
-                ev_done[b].record(stream)
-            c_out.wait_event(ev_done[b])
-            with torch.cuda.stream(c_out):
-                h_out[b].copy_(stage_out[b], non_blocking=True)
-            ev_out_free[b].record(c_out)
-        if timed:
-            e1.record(c_out)
+        with torch.cuda.stream(stream):
+            if timed:
+                e0.record(stream)
+            _copy_async(rt, stage_in[0], h_in, h2d, 1, stream)       # step 0's inputs
+            for i in range(n):
+                graphs[i & 1].replay()
+            _copy_async(rt, h_out[(n - 1) & 1], stage_out[(n - 1) & 1], out_bytes, 2,
+                        stream)                                     # the last step's output
+            if timed:
+                e1.record(stream)
         torch.cuda.synchronize()
 
     run(args.warmup, False)
     run(args.steps, True)
+    if not torch.equal(h_out[(args.steps - 1) & 1], ref):
+        raise RuntimeError("pipelined end-to-end output differs from the one-step run")
     t = e0.elapsed_time(e1) / 1e3 / args.steps
+    # the input copy alone, for reference (the pipelined step cannot beat it)
+    cp = []
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            e0.record(stream)
+            _copy_async(rt, stage_in[0], h_in, h2d, 1, stream)
+            e1.record(stream)
+            e1.synchronize()
+            cp.append(e0.elapsed_time(e1))
+    t_h2d = statistics.median(cp) / 1e3
     t, t_seq = max_over_ranks([t, t_seq], world, dev)
     return {"value": world * num_q / t, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": t * 1e3,
-            "pipelined": f"depth 2: inputs of step i+1 copied in and outputs of step i-1 read "
-                         f"back while step i computes; no L2 flush between steps, so this is "
-                         f"a warm-L2 figure (working set {step_bytes / 1e6:.0f} MB, L2 "
-                         f"{l2 / 1e6:.0f} MB: part of it stays resident); the flushed "
-                         f"one-step-at-a-time figure is beside it",
+            "pipelined": f"depth 2, one graph launch per step: inputs of step i+1 copied in "
+                         f"and outputs of step i-1 read back while step i computes; no L2 "
+                         f"flush between steps, so this is a warm-L2 figure (working set "
+                         f"{step_bytes / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB: part of it stays "
+                         f"resident); the flushed one-step-at-a-time figure is beside it",
             "l2": "warm (pipelined)",
-            "ms_per_step_one_at_a_time": t_seq * 1e3}
+            "ms_per_step_one_at_a_time": t_seq * 1e3,
+            "h2d_copy_ms": t_h2d * 1e3}
 
 
 def cpu_baseline(w, data, pt, budget_s=20.0):
@@ -619,7 +667,7 @@ def main_hca(args, world, rank, local, dev):
     e2e = None
     if not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
-                       hca_step_alg_bytes(w, int(batch.new_tokens.sum())))
+                       hca_step_alg_bytes(w, int(batch.new_tokens.sum())), body)
     split = csa.csa_hca_attention_workspace_size(w.num_q, w.heads, w.window, batch.decode,
                                                  batch.max_hca) > 0
     tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0    # merges its own splits
@@ -719,7 +767,7 @@ def main_dsa(args, world, rank, local, dev):
     e2e = None
     if not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
-                       dsa_step_alg_bytes(w))
+                       dsa_step_alg_bytes(w), body)
     split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, 0, batch.decode) > 0
     tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0    # merges its own splits
     launches = 2 + 1 + 1 + 2 + (1 if tc_attention or not split else 2)
@@ -874,8 +922,10 @@ def measure_csa(args, name, world, rank, local, dev, full=True):
     # or plain), top-k (merge, or one or two launches), attention (the tensor-core
     # kernel for FP8 rows and 64-head groups merges its splits itself; the
     # warp-level kernels add a combine launch when they split)
-    # the top-512 is one launch for rows of at most 49152 keys, else two
-    topk_launches = 1 if batch.max_c4 <= 49152 else 2
+    # the top-512 is one launch for rows of at most 49152 keys; longer rows take
+    # the bound-first selection (3 launches) for at most 64 rows, else the
+    # per-chunk selection and merge (2)
+    topk_launches = 1 if batch.max_c4 <= 49152 else (3 if w.num_q <= 64 else 2)
     tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0
     split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, w.window, batch.decode) > 0
     launches_per_step = (2 if batch.max_new >= 4 else 0) + 1 + 1 + (1 if fused[0] else topk_launches) + \
@@ -888,7 +938,7 @@ def measure_csa(args, name, world, rank, local, dev, full=True):
     e2e = None
     if full and not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
-                       step_alg_bytes(w))
+                       step_alg_bytes(w), step_body)
 
     if rank == 0:
         hbm, src = peaks()
