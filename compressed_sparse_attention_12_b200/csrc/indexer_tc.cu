@@ -787,7 +787,9 @@ static TcPlan plan_tc(const IndexerArgs &a, bool fuse) {
     p.qg = a.num_q <= a.bs ? 1 : n_max / p.hi_pad;
     if (p.qg < 1) p.qg = 1;
     if (p.qg > 4) p.qg = 4;
-    if (fp4 && p.qg * p.hi_pad > 64) p.qg = p.hi_pad >= 64 ? 1 : 64 / p.hi_pad;
+    // (FP4 query groups stay within N = 128: the block-scaled MMA's query
+    // scale factors are laid out for 128 columns)
+    if (fp4 && p.qg * p.hi_pad > 128) p.qg = p.hi_pad >= 128 ? 1 : 128 / p.hi_pad;
     p.n = p.qg * p.hi_pad;
     // four epilogue groups (two per accumulator, each reducing half of the
     // query rows) for the wide accumulators
