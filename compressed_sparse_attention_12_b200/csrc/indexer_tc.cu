@@ -427,7 +427,18 @@ indexer_tc_kernel(const IndexerArgs a, const __grid_constant__ CUtensorMap kmap,
                 }
                 tc::cp_async_commit();
             }
-            if (lane == 0) {
+            if (!kPaged && G::kChunks == 1) {
+                // one box per page: lanes 0 and 1 issue the tile's two pages
+                // in one instruction
+                if (lane == 0) tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
+                __syncwarp();
+                if (lane < 2) {
+                    int page = pg_s[i * 2 + lane];
+                    if (page < 0 || page >= p.num_pages) page = 0;   // epilogue reports visible keys
+                    tc::tma_load_2d(tc::saddr(stage_buf + s * kStage + lane * 64 * G::kSpan),
+                                    &kmap, 0, page * kC4Page, tc::saddr(&full[s]));
+                }
+            } else if (lane == 0) {
                 if constexpr (kPaged) tc::mbar_expect_tx(tc::saddr(&sfull[s]), kStage);
                 else tc::mbar_expect_tx(tc::saddr(&full[s]), G::kStageBytes);
 #pragma unroll
