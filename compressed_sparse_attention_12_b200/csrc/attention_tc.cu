@@ -39,8 +39,8 @@
 // memory, so the softmax of tile j overlaps the score MMAs of tile j+1, the
 // conversion of tile j+2 and the copies of tile j+3.
 // The splits of one query form a thread-block cluster and merge their
-// partial outputs inside the kernel (through an L2-resident workspace, after
-// a cluster barrier; no second kernel).
+// partial outputs inside the kernel, through distributed shared memory (no
+// second kernel).
 #include "attention.cuh"
 #include "tc.cuh"
 
@@ -73,10 +73,11 @@ constexpr uint32_t kTcOCol = 160;              // O: TMEM columns 160..415, both
 constexpr float kTcRaise = 8.0f;               // log2 headroom of p before the maximum is raised
 constexpr float kTcLog2e = 1.4426950408889634f;
 
-static_assert(kTcQBytes + kTcBufs * kTcTileBytes >= kTcHeads * kLatent * 4,
-              "the split merge receives every split's slice in the Q and tile buffers");
-static_assert(2 * kTcPBytes + kTcStages * kTcStageBytes >= kTcHeads * 256 * 4,
-              "the split merge stages an outgoing slice in the P and staging buffers");
+// the split merge's fp16 slices (64 heads x 512/splits dims each): the
+// splits-1 receive slots at the end of the buffers and at least one outgoing
+// slice below them
+static_assert(kTcHeads * kLatent * 2 <= kTcMiscOff,
+              "the split merge's slices fit in the CTA's buffers");
 static_assert(kTcBufs * kTcTileBytes == kTcHeads * kKvDim * 2,
               "the query's bf16 rows are staged in the tile buffers");
 
@@ -88,6 +89,8 @@ struct TcMisc {
     float qmul[kTcHeads];            // power of two applied to each head's query row
     float ml[kTcMaxSplits][kTcHeads][2];   // (running max, sum) per split and head (merge)
     float fct[kTcHeads];             // per head, this split's factor in the merged output
+    float vmax[kTcMaxSplits];        // per split: the largest block scale of its rows (merge)
+    float vrun;                      // largest block scale of the tiles converted so far
     union {
         float qpart[kTcHeads][6];    // set-up: per head, the largest |q| of each sixth of the row
         float mx[2][2][kTcHeads];    // main loop: tile maximum per (tile parity, warpgroup, head)
@@ -210,6 +213,10 @@ __device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
+}
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
 }
 
 __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
@@ -398,6 +405,7 @@ __device__ __forceinline__ void tc_store(const TcLoad &L, int c, uint8_t *tile, 
         if (lane == 0) {
             ms.smax[buf] = mx;
             ms.vmask[buf] = live;
+            ms.vrun = fmaxf(ms.vrun, mx);      // always the same thread
         }
     }
 }
@@ -443,6 +451,7 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
             tc::mbar_init(tc::saddr(&ms.drain), 1);
             tc::mbar_init(tc::saddr(&ms.recv_full), 1);
             ms.abort = 0;
+            ms.vrun = 0.0f;
             tc::fence_mbar_init();
         }
     }
@@ -796,15 +805,22 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
         }
     } else {
         // Split merge through distributed shared memory.  The (max, sum) of
-        // every head are exchanged first; then each split, for every other
-        // split in turn, stages that split's 512/splits output dims of its O
-        // (rescaled to the merged softmax, fp32, 16-byte chunks XOR-swizzled
-        // by head) in its own shared memory and pushes them with one bulk
-        // copy into the owner's receive buffer; the owner adds its own slice
-        // from TMEM and writes the bf16 outputs.
+        // every head and each split's largest block scale are exchanged
+        // first; then each split, for every other split in turn, stages that
+        // split's 512/splits output dims of its O (rescaled to the merged
+        // softmax, fp16, 16-byte chunks XOR-swizzled by head) in its own
+        // shared memory and pushes them with one bulk copy into the owner's
+        // receive buffer; the owner adds its own slice from TMEM (fp32) and
+        // writes the bf16 outputs.
+        // fp16 range: a split's share of a merged output is a weighted mean of
+        // value dims with weights summing to at most 1, so its magnitude is at
+        // most the largest |code x block scale| of the query's rows, < 448 x
+        // the largest block scale.  Slices are sent times the power of two
+        // that maps that bound into [2^14, 2^15) (exact scaling; fp16 keeps
+        // 11 significant bits of every value down to 2^-28 of the bound).
         const int dpo = kLatent / splits;                       // dims per owner
-        const uint32_t slice = (uint32_t)(kTcHeads * dpo * 4);  // bytes of one slice
-        const int cpr = dpo / 4;                                // 16-byte chunks per row
+        const uint32_t slice = (uint32_t)(kTcHeads * dpo * 2);  // bytes of one slice
+        const int cpr = dpo / 8;                                // 16-byte chunks per row
         // receive buffer at the end of the CTA's buffers: one slot per other
         // split (slot of split r: r, or r-1 for splits after this one);
         // outgoing slices staged from the start, as many as fit below it
@@ -816,6 +832,7 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
             const uint32_t src = tc::saddr(&ms.ml[sp][h][0]);
             for (int r = 0; r < splits; r++) st_cluster_f32x2(cluster_map(src, r), m_ref, l_sum);
         }
+        if (tid < splits) st_cluster_f32(cluster_map(tc::saddr(&ms.vmax[sp]), tid), ms.vrun);
         if (tid == 0) tc::mbar_expect_tx(tc::saddr(&ms.recv_full), (uint32_t)(splits - 1) * slice);
         cluster_sync();          // every split's MMAs are done and its (max, sum) delivered
         if (warp < 4 && rh == 0) {
@@ -832,6 +849,10 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
                 a.lse[orow0 + h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
         }
         __syncthreads();
+        float vb = 0.0f;
+        for (int r = 0; r < splits; r++) vb = fmaxf(vb, ms.vmax[r]);
+        const float f16s = fit_pow2(448.0f * vb, 15);          // slices are sent times f16s
+        const float f16r = 1.0f / f16s;                         // exact (a power of two)
         // warps 0-15: four per TMEM lane quarter; each 16x32bx2 load gives a
         // thread 16 columns of head hq (threads 16-31 the next 16)
         const int q4 = warp & 3, wq = warp >> 2;                // wq = 0..3 for warps 0-15
@@ -852,7 +873,8 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
 #pragma unroll
             for (int i = 0; i < 16; i++) o[i] = __uint_as_float(v[i]) * f;
         };
-        // byte offset of 16-byte chunk j of head row hh in a slice
+        // byte offset of 16-byte chunk j (8 fp16 dims) of head row hh in a
+        // slice (cpr >= 8: at most 8 splits)
         auto slot = [&](int hh, int j) {
             return (uint32_t)((hh * cpr + (j ^ (hh & 7))) * 16);
         };
@@ -868,11 +890,14 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
                     for (int c32 = 32 * wq; c32 < dpo; c32 += 128) {
                         const int dl = c32 + 16 * chalf;         // this thread's 16 dims
                         float o[16];
-                        read_o(owner * dpo + dl, fq, o);
+                        read_o(owner * dpo + dl, fq * f16s, o);
 #pragma unroll
-                        for (int v4 = 0; v4 < 4; v4++)
-                            *reinterpret_cast<float4 *>(out_slice + slot(hq, dl / 4 + v4)) =
-                                make_float4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+                        for (int v8 = 0; v8 < 2; v8++)
+                            *reinterpret_cast<uint4 *>(out_slice + slot(hq, dl / 8 + v8)) =
+                                make_uint4(pack_f16(o[8 * v8], o[8 * v8 + 1]),
+                                           pack_f16(o[8 * v8 + 2], o[8 * v8 + 3]),
+                                           pack_f16(o[8 * v8 + 4], o[8 * v8 + 5]),
+                                           pack_f16(o[8 * v8 + 6], o[8 * v8 + 7]));
                     }
                 }
             }
@@ -899,13 +924,17 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
                 read_o(sp * dpo + dl, fq, o);
                 for (int r = 0; r < splits - 1; r++) {
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; v4++) {
-                        const float4 x = *reinterpret_cast<const float4 *>(
-                            recv + r * slice + slot(hq, dl / 4 + v4));
-                        o[4 * v4] += x.x;
-                        o[4 * v4 + 1] += x.y;
-                        o[4 * v4 + 2] += x.z;
-                        o[4 * v4 + 3] += x.w;
+                    for (int v8 = 0; v8 < 2; v8++) {
+                        const uint4 x = *reinterpret_cast<const uint4 *>(
+                            recv + r * slice + slot(hq, dl / 8 + v8));
+                        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            const float2 f = __half22float2(
+                                *reinterpret_cast<const __half2 *>(&w[k]));
+                            o[8 * v8 + 2 * k] = fmaf(f.x, f16r, o[8 * v8 + 2 * k]);
+                            o[8 * v8 + 2 * k + 1] = fmaf(f.y, f16r, o[8 * v8 + 2 * k + 1]);
+                        }
                     }
                 }
                 __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +

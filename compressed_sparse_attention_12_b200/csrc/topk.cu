@@ -368,6 +368,242 @@ topk_reg_kernel(const float *__restrict__ logits, int64_t stride, const int32_t 
     }
 }
 
+// ------------------------------------------------------------------ cluster rows
+//
+// A few rows of at most kTkRegMax logits (decode batches): a cluster of C CTAs
+// per row, so that the sweeps over the row's keys run on C SMs instead of one.
+// CTA c of the cluster holds keys [c*chunk, (c+1)*chunk), chunk = kTkRegMax/C,
+// in registers, in the layout of ordered_starts (16-byte slices of 4
+// consecutive keys; warps, slices and lanes in index order).
+//   1. The groups are the slices.  How many non-empty groups each CTA has
+//      follows from the row length alone, so every CTA knows every CTA's quota
+//      K_c = floor(512 * groups_c / groups_total) (CTA 0 also takes the
+//      remainder, so the quotas sum to 512), and CTA c finds L_c, the lower
+//      edge of the radix bin holding its K_c-th largest group maximum (one
+//      pass).  With L the smallest L_c over the CTAs with a quota, at least
+//      512 groups hold a key >= L, so every key of the top 512 is >= L (L = 0
+//      when the row has fewer than 512 groups).  A CTA holding only a few
+//      groups gets no quota, so its keys do not lower L.
+//   2. Through distributed shared memory the CTAs exchange (L_c, largest
+//      key), then their counts of keys >= L, and write those keys and their
+//      indices, in index order, into CTA 0's candidate buffer.
+//   3. CTA 0 selects the top 512 among the candidates as the one-CTA kernels
+//      do, with the page transform and -1 padding.  If the candidates overflow
+//      its buffer (heavy ties), CTA 0 stages the whole row there instead and
+//      selects from it.
+// Every CTA takes the same cluster barriers (branches depend on cluster-wide
+// values only); every remote write lands before a barrier that its target
+// passes, and no CTA is written to after it has passed its last barrier.
+constexpr int kClThreads = 512;
+constexpr int kClMaxC = 4;
+constexpr int kClCap = 16384;                    // candidates in CTA 0 (key + index)
+constexpr size_t kClSmem = (size_t)kClCap * 8;   // also holds a whole row of floats
+constexpr int kClMinLen = 8192;                  // shorter rows: one CTA per row
+constexpr int kClSms = 148;                      // CTAs of one wave (SMs of a B200)
+static_assert(kClSmem >= (size_t)kTkRegMax * 4, "the fallback stages a whole row");
+using TkClShared = TkSharedT<kClThreads>;
+
+struct ClMail {
+    uint32_t lc[kClMaxC];       // per CTA: its bound L_c (all ones: no bound)
+    uint32_t kmax[kClMaxC];     // per CTA: its largest key
+    uint32_t cnt[kClMaxC];      // per CTA: its keys >= L
+};
+
+// Address of `p` (this CTA's shared memory) in the shared memory of CTA
+// `rank` of the cluster.
+__device__ __forceinline__ uint32_t cl_map(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                 : "=r"(r)
+                 : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cl_st(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Every thread of every CTA of the cluster arrives; writes before it are
+// visible to reads after it anywhere in the cluster.
+__device__ __forceinline__ void cl_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int C>
+__global__ void __launch_bounds__(kClThreads, 1)
+topk_cluster_kernel(const float *__restrict__ logits, int64_t stride, const int32_t *c4_lens,
+                    int bs, const int32_t *cu_q, const int32_t *q_pos, int max_c4_len,
+                    const int32_t *page_table, int pt_stride, int64_t num_slots,
+                    int32_t *out_phys, int32_t *out_raw, int32_t *status, int ratio) {
+    constexpr int NT = kClThreads, KPT = kTkRegMax / (C * NT), NS = KPT / 4;
+    constexpr int kChunk = NT * KPT;
+    static_assert(C >= 2 && C <= kClMaxC && KPT % 4 == 0 && NS <= 32, "cluster layout");
+    __shared__ TkClShared sh;
+    __shared__ ClMail mail;
+    extern __shared__ __align__(16) uint8_t cl_smem[];
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(cl_smem);
+    int32_t *cand_idx = reinterpret_cast<int32_t *>(cl_smem + (size_t)kClCap * 4);
+    // this CTA has started (the wait before the first remote write pairs with it)
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    pdl_trigger();
+    const int crank = blockIdx.x, t = blockIdx.y;
+    const RowInfo ri = row_info<NT>(t, cu_q, bs, q_pos, c4_lens, max_c4_len, pt_stride, status,
+                                    crank == 0, sh, ratio);
+    pdl_wait();
+    const int len = min(ri.n_vis, kTkRegMax);     // the host keeps max_c4_len <= kTkRegMax
+    const float *row = logits + (int64_t)t * stride;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // slice j of lane l in warp w: keys lo + 32*KPT*w + 128j + 4l .. +3
+    const int w0 = crank * kChunk + warp * (32 * KPT) + 4 * lane;
+    auto index_of = [&](int kk) { return w0 + 128 * (kk >> 2) + (kk & 3); };
+    const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+    uint32_t keys[KPT];
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        const int i0 = w0 + 128 * j;
+        if (vec && i0 + 4 <= len) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(row + i0);
+            keys[4 * j] = x.x;
+            keys[4 * j + 1] = x.y;
+            keys[4 * j + 2] = x.z;
+            keys[4 * j + 3] = x.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; e++)
+                keys[4 * j + e] = i0 + e < len ? __float_as_uint(row[i0 + e]) : 0u;
+        }
+    }
+    // keys, slice maxima, the CTA's smallest slice maximum and largest key
+    uint32_t gm[NS];
+    uint32_t gpres = 0;          // bit j: slice j holds a key
+    uint32_t gmin = 0xffffffffu, kmx = 0u;
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        gm[j] = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int kk = 4 * j + e;
+            const bool p = index_of(kk) < len;
+            const uint32_t k = p ? order_key(__uint_as_float(keys[kk]), status) : 0u;
+            keys[kk] = k;
+            if (p) gm[j] = max(gm[j], k);
+        }
+        if (index_of(4 * j) < len) {
+            gpres |= 1u << j;
+            gmin = min(gmin, gm[j]);
+            kmx = max(kmx, gm[j]);
+        }
+    }
+    block_minmax<NT>(gmin, kmx, sh);
+    // this CTA's bound L_c
+    auto groups_of = [&](int c) {
+        const int m = min(len, (c + 1) * kChunk) - c * kChunk;
+        return m > 0 ? (m + 3) >> 2 : 0;
+    };
+    int g_total = 0;
+#pragma unroll
+    for (int c = 0; c < C; c++) g_total += groups_of(c);
+    const int K = min(kTopK, len);
+    uint32_t Lc = 0u;
+    if (len > kTopK && g_total >= kTopK) {
+        Lc = 0xffffffffu;
+        // quotas floor(512 g_c / total), the remainder to CTA 0 (which has the
+        // most groups: chunks fill in order); they sum to 512 and K_c <= g_c
+        int Kc = (int)((int64_t)kTopK * groups_of(crank) / g_total);
+        if (crank == 0) {
+            int floors = 0;
+#pragma unroll
+            for (int c = 0; c < C; c++) floors += (int)((int64_t)kTopK * groups_of(c) / g_total);
+            Kc += kTopK - floors;
+        }
+        if (Kc > 0) {
+            int unused;
+            radix_threshold_regs<NT, NS>(gm, [&](int j) { return ((gpres >> j) & 1u) != 0u; },
+                                         Kc, gmin, kmx, sh, &Lc, &unused, true);
+        }
+    }
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");    // every CTA has started
+    if ((int)threadIdx.x < C) {
+        cl_st(cl_map(&mail.lc[crank], threadIdx.x), Lc);
+        cl_st(cl_map(&mail.kmax[crank], threadIdx.x), kmx);
+    }
+    cl_sync();
+    uint32_t L = 0xffffffffu, kmax_all = 0u;
+#pragma unroll
+    for (int c = 0; c < C; c++) {
+        L = min(L, mail.lc[c]);
+        kmax_all = max(kmax_all, mail.kmax[c]);
+    }
+    // this CTA's candidates (keys >= L): counts per slice, then index-order offsets
+    uint32_t at[NS];
+#pragma unroll
+    for (int j = 0; j < NS; j++) {
+        at[j] = 0;
+#pragma unroll
+        for (int e = 0; e < 4; e++)
+            at[j] += (index_of(4 * j + e) < len && keys[4 * j + e] >= L) ? 1u : 0u;
+    }
+    const uint32_t n_c = ordered_starts<NT, NS>(at, sh);
+    if ((int)threadIdx.x < C) cl_st(cl_map(&mail.cnt[crank], threadIdx.x), n_c);
+    cl_sync();
+    uint32_t n_cand = 0, off = 0;
+#pragma unroll
+    for (int c = 0; c < C; c++) {
+        off += c < crank ? mail.cnt[c] : 0u;
+        n_cand += mail.cnt[c];
+    }
+    const int32_t *pt_row = page_table + (int64_t)ri.b * pt_stride;
+    int32_t *op = out_phys + (int64_t)t * kTopK;
+    int32_t *orw = out_raw ? out_raw + (int64_t)t * kTopK : nullptr;
+    auto emit = [&](int pos, int s) {
+        const int32_t page = pt_row[s / kC4Page];
+        const int64_t slot = (int64_t)page * kC4Page + s % kC4Page;
+        int32_t phys = (int32_t)slot;
+        if (page < 0 || slot >= num_slots) {
+            report(status, CSA_ERR_BOUNDS);
+            phys = -1;
+        }
+        op[pos] = phys;
+        if (orw) orw[pos] = s;
+    };
+    if (n_cand <= (uint32_t)kClCap) {            // uniform over the cluster
+#pragma unroll
+        for (int j = 0; j < NS; j++) {
+            uint32_t a = off + at[j];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int kk = 4 * j + e;
+                if (index_of(kk) < len && keys[kk] >= L) {
+                    cl_st(cl_map(&cand_key[a], 0), keys[kk]);
+                    cl_st(cl_map(&cand_idx[a], 0), (uint32_t)index_of(kk));
+                    a++;
+                }
+            }
+        }
+        cl_sync();
+        if (crank != 0) return;
+        uint32_t T = 0;
+        int need_eq = (int)n_cand;
+        if (len > kTopK) radix_threshold<NT>(cand_key, (int)n_cand, K, L, kmax_all, sh, &T, &need_eq);
+        ordered_compact<NT>(cand_key, (int)n_cand, T, need_eq, sh,
+                            [&](int pos, int i, uint32_t) { emit(pos, cand_idx[i]); });
+    } else {
+        // heavy ties: CTA 0 selects from the whole row, staged in its buffer
+        if (crank != 0) return;
+        uint32_t *skeys = reinterpret_cast<uint32_t *>(cl_smem);
+        stage_row_keys<NT>(skeys, row, len);
+        __syncthreads();
+        uint32_t T, km;
+        select_top512<NT>(skeys, len, sh, status, &T, &km,
+                          [&](int pos, int i, uint32_t) { emit(pos, i); });
+    }
+    for (int p = K + threadIdx.x; p < kTopK; p += NT) {
+        op[p] = -1;
+        if (orw) orw[p] = -1;
+    }
+}
+
 // ------------------------------------------------------------------ bound-first selection
 //
 // For a few long rows (decode batches): three launches spread over every SM
@@ -643,6 +879,33 @@ static cudaError_t launch_topk_bound_first(const TopkArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// One cluster of C CTAs per query row (rows of at most kTkRegMax logits).
+template <int C>
+static cudaError_t launch_topk_cluster(const TopkArgs &a, cudaStream_t s) {
+    static int done[64] = {0};
+    cudaError_t e = ensure_max_smem((const void *)topk_cluster_kernel<C>, (int)kClSmem, done);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, a.num_q);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.dynamicSmemBytes = kClSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<C>, a.logits, a.logits_stride, a.c4_seq_lens,
+                           a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.page_table, a.pt_stride,
+                           a.num_slots, a.out_phys, a.out_raw, a.status, a.ratio);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 static int topk_max_chunks(int max_c4_len) {
     return max_c4_len <= 0 ? 1 : (max_c4_len + kTkChunk - 1) / kTkChunk;
 }
@@ -655,12 +918,18 @@ static size_t two_stage_bytes(int num_q, int max_c4_len) {
 }
 
 // Which selection runs for these sizes: the bound-first launches for a few
-// long rows (when their workspace fits `limit`), else one CTA per row for rows
-// of at most kTkRowMax keys, else the two-stage merge.
-enum TopkKind { kTopkReg, kTopkRow, kTopkBound, kTopkTwoStage };
+// long rows (when their workspace fits `limit`); a cluster of 4 or 2 CTAs per
+// row for up to one wave of such CTAs with rows of kClMinLen .. kTkRegMax
+// keys; else one CTA per row for rows of at most kTkRowMax keys; else the
+// two-stage merge.
+enum TopkKind { kTopkCluster4, kTopkCluster2, kTopkReg, kTopkRow, kTopkBound, kTopkTwoStage };
 
 static TopkKind topk_kind(int num_q, int max_c4_len, size_t limit) {
     if (tb_applies(num_q, max_c4_len) && tb_bytes(num_q, max_c4_len) <= limit) return kTopkBound;
+    if (max_c4_len > kClMinLen && max_c4_len <= kTkRegMax) {
+        if ((int64_t)num_q * 4 <= kClSms) return kTopkCluster4;
+        if ((int64_t)num_q * 2 <= kClSms) return kTopkCluster2;
+    }
     if (max_c4_len <= kTkRegMax) return kTopkReg;
     if (max_c4_len <= kTkRowMax) return kTopkRow;
     return kTopkTwoStage;
@@ -697,6 +966,8 @@ static cudaError_t launch_topk512_limited(const TopkArgs &a, cudaStream_t s, siz
     if (a.num_q == 0) return cudaSuccess;
     const TopkKind kind = topk_kind(a.num_q, a.max_c4_len, limit);
     if (kind == kTopkBound) return launch_topk_bound_first(a, s);
+    if (kind == kTopkCluster4) return launch_topk_cluster<4>(a, s);
+    if (kind == kTopkCluster2) return launch_topk_cluster<2>(a, s);
     if (kind == kTopkReg) {
         launch_k(topk_reg_kernel, a.num_q, kTkRowThreads, 0, s, a.logits, a.logits_stride,
                  a.c4_seq_lens, a.bs, a.cu_q, a.q_pos, a.max_c4_len, a.page_table, a.pt_stride,

@@ -234,6 +234,11 @@ csa_status_t csa_indexer_logits(const void *q_codes, const uint8_t *q_block_scal
  *   workspace      >= csa_topk512_workspace_size(num_q, max_c4_len) bytes
  *                  (always checked; written only when max_c4_len > 49152, the
  *                  rows shorter than that being selected in one launch)
+ * Up to 74 rows of 8193..32768 keys are selected by a thread-block cluster
+ * of 4 CTAs per row (2 CTAs above 37 rows) that share the row's keys: their
+ * group maxima give each CTA a bound, the keys above the lowest bound are
+ * gathered into the first CTA through distributed shared memory, and it
+ * selects among them.  Other rows of at most 49152 keys take one CTA per row.
  * Rows longer than 49152 keys are selected in several launches: with at most
  * 64 rows, a bound-first selection spread over every SM (the maxima of about
  * 1024-2048 groups of consecutive keys give a lower bound of the 512th key,

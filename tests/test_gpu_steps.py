@@ -489,6 +489,15 @@ def _topk_case(case, rng):
         c4, ql = [32769, 31000], [1, 1]
     elif case == "allequal_reg":
         c4, ql = [32768, 9000], [1, 1]
+    elif case == "cluster2":
+        # 40 rows: two CTAs per row (the four-CTA form takes up to 37 rows)
+        c4, ql = [32768, 20000, 8193, 12000, 30001], [8, 8, 8, 8, 8]
+    elif case == "cluster_edge":
+        # rows that end just inside the second, third and fourth CTA's keys
+        c4, ql = [8197, 16385, 24577, 9000, 32767], [1, 1, 1, 1, 1]
+    elif case == "reg_many":
+        # 80 rows: one CTA per row
+        c4, ql = [32768, 9000, 20000, 1200], [20, 20, 20, 20]
     elif case == "rowmax":
         # the longest rows the one-launch top-k stages whole (49152 keys), with ties
         c4, ql = [49152, 30000, 4], [1, 3, 1]
@@ -517,11 +526,13 @@ def _topk_case(case, rng):
     stride_l = max_c4 + 3
     lg = np.full((nq, stride_l), np.nan, dtype=np.float32)
     for t in range(nq):
-        if case in ("ties", "rowmax", "rowmax1", "regmax", "regmax1"):
+        if case in ("ties", "rowmax", "rowmax1", "regmax", "regmax1", "cluster2"):
             v = np.round(rng.standard_normal(max_c4) * 3) / 2
             v[rng.integers(0, max_c4, 50)] = -0.0
         elif case in ("allequal", "allequal_reg"):
             v = np.full(max_c4, 2.5)
+        elif case == "cluster_edge":
+            v = np.maximum(rng.standard_normal(max_c4), 0.0) * 3
         elif case == "long":
             v = rng.standard_t(3, max_c4)
             v[rng.integers(0, max_c4, 100)] = -np.inf
@@ -538,7 +549,8 @@ def _topk_case(case, rng):
 
 
 @pytest.mark.parametrize("case", ["short", "ties", "long", "causal", "allequal", "rowmax",
-                                  "rowmax1", "regmax", "regmax1", "allequal_reg"])
+                                  "rowmax1", "regmax", "regmax1", "allequal_reg", "cluster2",
+                                  "cluster_edge", "reg_many"])
 def test_topk512_bit_exact(case):
     csa = _csa()
     c = _topk_case(case, np.random.default_rng(len(case)))
