@@ -814,8 +814,8 @@ sparse_mqa_tc_kernel(const AttnArgs a, int splits, int tiles_per_split) {
         // writes the bf16 outputs.
         // fp16 range: a split's share of a merged output is a weighted mean of
         // value dims with weights summing to at most 1, so its magnitude is at
-        // most the largest |code x block scale| of the query's rows, < 448 x
-        // the largest block scale.  Slices are sent times the power of two
+        // most the largest |code x block scale| of the query's rows, at most
+        // 448 x the largest block scale.  Slices are sent times the power of two
         // that maps that bound into [2^14, 2^15) (exact scaling; fp16 keeps
         // 11 significant bits of every value down to 2^-28 of the bound).
         const int dpo = kLatent / splits;                       // dims per owner

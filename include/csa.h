@@ -380,7 +380,9 @@ csa_status_t csa_topk512_merge(int32_t num_q, int32_t idx_heads, int32_t idx_dim
  * query's rows across CTAs (few queries, many rows each), _prefill gives each
  * query its own CTA (many queries).  FP8 rows with heads a multiple of 64 run
  * on the tensor-core kernel, whose splits (a thread-block cluster of at most 8
- * CTAs per query) merge inside the kernel and use no workspace; the other
+ * CTAs per query) merge inside the kernel and use no workspace (the partial
+ * outputs cross the cluster as fp16 under a shared power of two, rounded to
+ * at most 2^-11 relative, and are summed in fp32); the other
  * cases write split partials to the workspace and merge them in a second
  * launch.
  * Ordering: like every kernel of the library this one is launched with
