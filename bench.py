@@ -371,12 +371,24 @@ def pack_inputs(batch, names, dev):
         offs.append(total)
         total += (t.numel() * t.element_size() + 255) // 256 * 256
     arena = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
+    layout = []
     for (n, t), o in zip(items, offs):
         nb = t.numel() * t.element_size()
         view = arena[o:o + nb].view(t.dtype).view(t.shape)
         view.copy_(t)
         setattr(batch, n, view)
+        layout.append((n, o, nb, t.dtype, tuple(t.shape)))
+    arena.input_layout = layout  # lets the pipelined loop bind the inputs to other buffers
     return arena
+
+
+def bind_inputs(batch, arena_like, layout, out):
+    """Points the step inputs batch.<name> at the same offsets of another
+    buffer of the arena's size, and batch.out at `out` (before capturing a
+    graph that should read and write those buffers)."""
+    for n, o, nb, dt, shape in layout:
+        setattr(batch, n, arena_like[o:o + nb].view(dt).view(shape))
+    batch.out = out
 
 
 def _cudart():
@@ -409,7 +421,7 @@ def _copy_async(rt, dst, src, nbytes, kind, stream):
         raise RuntimeError(f"cudaMemcpyAsync failed: {rc}")
 
 
-def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_bytes, body):
+def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_bytes, body, batch):
     """The step end to end: every step copies its inputs (the packed arena)
     from pinned host memory, runs the step and copies the output back to
     pinned host memory, all inside the timed region.
@@ -417,10 +429,12 @@ def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_byte
     Reported, when the step's working set (step_bytes) is larger than L2: the
     pipelined loop a serving process runs -- two staging buffers on each
     side; each step is one launch of a graph whose three branches copy step
-    i+1's inputs in, run step i (`body`), and read step i-1's output back,
-    so that both copies run while step i computes; no L2 flush is needed --
-    and beside it the one-step-at-a-time loop with an L2 flush before every
-    step.  Smaller steps report the one-step-at-a-time loop only."""
+    i+1's inputs in, run step i (`body`, captured with batch's inputs and
+    output bound to staging buffer i % 2, so no device-side copies), and
+    read step i-1's output back, so that both copies run while step i
+    computes; no L2 flush is needed -- and beside it the one-step-at-a-time
+    loop with an L2 flush before every step.  Smaller steps report the
+    one-step-at-a-time loop only."""
     import torch
     h_in = arena.cpu().pin_memory()
     h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
@@ -460,6 +474,7 @@ def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_byte
     out_bytes = out.numel() * out.element_size()
 
     def pipeline_graph(b):
+        bind_inputs(batch, stage_in[b], arena.input_layout, stage_out[b])
         gp = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             with torch.cuda.graph(gp, stream=stream):
@@ -467,14 +482,13 @@ def time_e2e(g, stream, args, l2_flush, arena, out, world, dev, num_q, step_byte
                 c_out.wait_stream(stream)
                 _copy_async(rt, stage_in[1 - b], h_in, h2d, 1, c_in)
                 _copy_async(rt, h_out[1 - b], stage_out[1 - b], out_bytes, 2, c_out)
-                arena.copy_(stage_in[b])
                 body(stream)
-                stage_out[b].copy_(out)
                 stream.wait_stream(c_in)
                 stream.wait_stream(c_out)
         return gp
 
     graphs = [pipeline_graph(0), pipeline_graph(1)]
+    bind_inputs(batch, arena, arena.input_layout, out)  # the step graph's own buffers again
 
     def run(n, timed):
         torch.cuda.synchronize()
@@ -667,7 +681,7 @@ def main_hca(args, world, rank, local, dev):
     e2e = None
     if not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
-                       hca_step_alg_bytes(w, int(batch.new_tokens.sum())), body)
+                       hca_step_alg_bytes(w, int(batch.new_tokens.sum())), body, batch)
     split = csa.csa_hca_attention_workspace_size(w.num_q, w.heads, w.window, batch.decode,
                                                  batch.max_hca) > 0
     tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0    # merges its own splits
@@ -767,7 +781,7 @@ def main_dsa(args, world, rank, local, dev):
     e2e = None
     if not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
-                       dsa_step_alg_bytes(w), body)
+                       dsa_step_alg_bytes(w), body, batch)
     split = csa.csa_sparse_mqa_workspace_size(w.num_q, w.heads, 0, batch.decode) > 0
     tc_attention = w.kv_fmt == "fp8" and w.heads % 64 == 0    # merges its own splits
     launches = 2 + 1 + 1 + 2 + (1 if tc_attention or not split else 2)
@@ -938,7 +952,7 @@ def measure_csa(args, name, world, rank, local, dev, full=True):
     e2e = None
     if full and not args.profile:
         e2e = time_e2e(g, stream, args, l2_flush, arena, batch.out, world, dev, w.num_q,
-                       step_alg_bytes(w), step_body)
+                       step_alg_bytes(w), step_body, batch)
 
     if rank == 0:
         hbm, src = peaks()
