@@ -71,3 +71,28 @@ def test_decode_roofline_is_hbm_bound():
     assert line["logit_bytes_per_launch"] == 32 * 32768 * 4
     assert line["traffic"] == 144419328
     assert line["intensity_flop_per_byte"] < line["ridge_flop_per_byte"]
+
+
+def test_pack_inputs_and_rebinding_keep_each_input_at_its_offset():
+    # the step inputs move into one buffer (256-byte aligned views); binding
+    # them to another buffer of the same size keeps names, shapes and offsets
+    import torch
+
+    class B:
+        pass
+
+    b = B()
+    b.q = torch.arange(6, dtype=torch.float32).reshape(2, 3)
+    b.w = torch.arange(5, dtype=torch.int32)
+    b.out = torch.zeros(4)
+    arena = bench.pack_inputs(b, ["q", "w", "missing"], "cpu")
+    assert [e[0] for e in arena.input_layout] == ["q", "w"]
+    assert [e[1] % 256 for e in arena.input_layout] == [0, 0]
+    assert torch.equal(b.q, torch.arange(6, dtype=torch.float32).reshape(2, 3))
+    assert b.q.data_ptr() == arena.data_ptr()
+    other = arena.clone()
+    out2 = torch.ones(4)
+    bench.bind_inputs(b, other, arena.input_layout, out2)
+    assert b.q.data_ptr() == other.data_ptr() and b.out is out2
+    assert torch.equal(b.w, torch.arange(5, dtype=torch.int32))
+    assert b.w.data_ptr() == other.data_ptr() + arena.input_layout[1][1]
