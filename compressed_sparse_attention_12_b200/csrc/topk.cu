@@ -7,16 +7,25 @@
 // (logit descending, logical index ascending); outputs are listed in
 // ascending logical index and padded with -1.
 //
-// Two launches, no inter-CTA waits:
-//   stage 1: each CTA takes a chunk of logits of one query row into shared
-//            memory and writes the chunk's top-512 (key, index) pairs in index
-//            order plus (512th key, largest key) to the workspace
-//            (select_chunk in topk.cuh; the indexer kernel can run the same
-//            step on its own chunk instead).
-//   stage 2: one CTA per query row selects among the row's concatenated
-//            candidates (every element of the global top-512 is in its chunk's
-//            top-512 under the same total order) and writes physical slots
-//            page_table[s/64]*64 + s%64 and raw indices.
+// Forms, chosen on the host by the batch's row count and longest row
+// (launch_topk512):
+//   * a thread-block cluster of 4 or 2 CTAs per row (up to one wave of them,
+//     rows of 8193..32768 logits): topk_cluster_kernel;
+//   * one CTA per row holding the row in registers (rows of at most 32768
+//     logits) or in shared memory (at most 49152): topk_reg_kernel,
+//     topk_row_kernel;
+//   * for at most 64 longer rows, a bound from group maxima applied by every
+//     chunk's CTA, then one CTA per row: the three topk_tb_* kernels;
+//   * otherwise two launches:
+//     stage 1: each CTA takes a chunk of logits of one query row into shared
+//              memory and writes the chunk's top-512 (key, index) pairs in
+//              index order plus (512th key, largest key) to the workspace
+//              (select_chunk in topk.cuh; the indexer kernel can run the same
+//              step on its own chunk instead);
+//     stage 2: one CTA per query row selects among the row's concatenated
+//              candidates (every element of the global top-512 is in its
+//              chunk's top-512 under the same total order).
+// Every form writes physical slots page_table[s/64]*64 + s%64 and raw indices.
 #include "common.cuh"
 #include "launch.h"
 #include <atomic>
